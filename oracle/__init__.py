@@ -1,0 +1,169 @@
+"""Test infrastructure: the fp64 CPU oracle for top-p routed block-sparse attention.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline /
+reference leg may import this package.  The product (``top_routed_block_b200``)
+never does, and the oracle shares no code with it.
+
+The arithmetic lives in ``fvattn_oracle.c`` (plain C loops, fp64, index-order
+sums, compiled with ``-ffp-contract=off``).  This module only builds that file
+and marshals numpy arrays into it.  Sources, per function, are cited in the C
+file: the FVAttn review, §1 Key Terms (top-p routing) and §1 RLB / §3 (per-head
+work after the mask), and the FlashAttention review, §Background "Motivation"
+(S = QK^T, P = softmax(S), O = PV) and §Model "Tiling Softmax".
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "fvattn_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle shared library in-tree (gcc, -O2, no FP contraction)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        cmd = ["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared",
+               "-pthread", _SRC, "-o", _LIB + ".tmp", "-lm"]
+        subprocess.check_call(cmd)
+        os.replace(_LIB + ".tmp", _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB)
+        P = ctypes.c_void_p
+        i32, i64, dbl = ctypes.c_int, ctypes.c_int64, ctypes.c_double
+        lib.oracle_pool.argtypes = [P, i64, i32, i32, i32, P, i32]
+        lib.oracle_route.argtypes = [P, P, i32, i32, i32, i32, i32, dbl, P, P, i64, P, P, i32]
+        lib.oracle_attn_rows.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, P, P, P, i64, P, P, i32]
+        lib.oracle_attn_tiled.argtypes = lib.oracle_attn_rows.argtypes
+        lib.oracle_lpt_order.argtypes = [P, i64, P]
+        for f in ("oracle_pool", "oracle_route", "oracle_attn_rows", "oracle_attn_tiled", "oracle_lpt_order"):
+            getattr(lib, f).restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def default_threads() -> int:
+    return max(1, os.cpu_count() or 1)
+
+
+def _bits(x: np.ndarray) -> np.ndarray:
+    """bf16 tensors travel as their uint16 bit patterns."""
+    x = np.ascontiguousarray(x)
+    if x.dtype != np.uint16:
+        raise TypeError("oracle inputs are bf16 bit patterns (uint16)")
+    return x
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def pool(X: np.ndarray, bs: int, nthreads: int | None = None) -> np.ndarray:
+    """Mean of each block of ``bs`` tokens over the tokens that exist: X [B,H,N,d] -> [B,H,nb,d] fp64."""
+    X = _bits(X)
+    B, H, N, d = X.shape
+    nb = -(-N // bs)
+    out = np.empty((B, H, nb, d), dtype=np.float64)
+    rc = _load().oracle_pool(_ptr(X), B * H, N, d, bs, _ptr(out), nthreads or default_threads())
+    if rc != 0:
+        raise ValueError(f"oracle_pool failed ({rc})")
+    return out
+
+
+class Route:
+    """CSR block mask from the oracle, with per-row diagnostics.
+
+    ``diag[r]`` = (mass kept, mass without the last kept block, last kept score,
+    first dropped score, last kept probability, first dropped probability).
+    """
+
+    def __init__(self, row_ptr, col_idx, head_counts, diag):
+        self.row_ptr, self.col_idx, self.head_counts, self.diag = row_ptr, col_idx, head_counts, diag
+
+    @property
+    def counts(self) -> np.ndarray:
+        return np.diff(self.row_ptr)
+
+
+def route(Q: np.ndarray, K: np.ndarray, p: float, bs: int, nthreads: int | None = None) -> Route:
+    Q, K = _bits(Q), _bits(K)
+    B, H, N, d = Q.shape
+    if K.shape != Q.shape:
+        raise ValueError("Q and K shapes differ")
+    nb = -(-N // bs)
+    rows = B * H * nb
+    row_ptr = np.empty(rows + 1, dtype=np.int32)
+    cap = rows * nb
+    col_idx = np.empty(max(cap, 1), dtype=np.int32)
+    head_counts = np.empty(B * H, dtype=np.int32)
+    diag = np.empty((rows, 6), dtype=np.float64)
+    rc = _load().oracle_route(_ptr(Q), _ptr(K), B, H, N, d, bs, float(p), _ptr(row_ptr), _ptr(col_idx), cap,
+                              _ptr(head_counts), _ptr(diag), nthreads or default_threads())
+    if rc != 0:
+        raise ValueError(f"oracle_route failed ({rc})")
+    return Route(row_ptr, col_idx[: row_ptr[-1]].copy(), head_counts, diag)
+
+
+def _attn(fn, Q, K, V, bs, causal, row_ptr, col_idx, tokens, nthreads):
+    Q, K, V = _bits(Q), _bits(K), _bits(V)
+    B, H, N, d = Q.shape
+    tokens = np.ascontiguousarray(tokens, dtype=np.int64)
+    row_ptr = np.ascontiguousarray(row_ptr, dtype=np.int32)
+    col_idx = np.ascontiguousarray(col_idx, dtype=np.int32)
+    if col_idx.size == 0:
+        col_idx = np.zeros(1, dtype=np.int32)
+    O = np.empty((tokens.size, d), dtype=np.float64)
+    LSE = np.empty(tokens.size, dtype=np.float64)
+    rc = fn(_ptr(Q), _ptr(K), _ptr(V), B, H, N, d, bs, 1 if causal else 0, _ptr(row_ptr), _ptr(col_idx),
+            _ptr(tokens), tokens.size, _ptr(O), _ptr(LSE), nthreads or default_threads())
+    if rc != 0:
+        raise ValueError(f"oracle attention failed ({rc})")
+    return O, LSE
+
+
+def attn_rows(Q, K, V, bs, causal, row_ptr, col_idx, tokens, nthreads=None):
+    """Row-wise definition. ``tokens`` are flat indices (b*H + h)*N + t. Returns O [n,d], LSE [n] (fp64)."""
+    return _attn(_load().oracle_attn_rows, Q, K, V, bs, causal, row_ptr, col_idx, tokens, nthreads)
+
+
+def attn_tiled(Q, K, V, bs, causal, row_ptr, col_idx, tokens, nthreads=None):
+    """Block-by-block online softmax; equal to :func:`attn_rows` up to rounding."""
+    return _attn(_load().oracle_attn_tiled, Q, K, V, bs, causal, row_ptr, col_idx, tokens, nthreads)
+
+
+def lpt_order(row_ptr: np.ndarray) -> np.ndarray:
+    """Rows sorted by selected-block count descending, ties by row id ascending."""
+    row_ptr = np.ascontiguousarray(row_ptr, dtype=np.int32)
+    rows = row_ptr.size - 1
+    order = np.empty(max(rows, 1), dtype=np.int32)
+    rc = _load().oracle_lpt_order(_ptr(row_ptr), rows, _ptr(order))
+    if rc != 0:
+        raise ValueError("oracle_lpt_order failed")
+    return order[:rows]
+
+
+def dense_csr(B: int, H: int, N: int, bs: int, causal: bool = False):
+    """Every key block for every query block (lower triangle of blocks if causal)."""
+    nb = -(-N // bs)
+    counts = []
+    cols = []
+    for _bh in range(B * H):
+        for i in range(nb):
+            js = list(range(i + 1)) if causal else list(range(nb))
+            counts.append(len(js))
+            cols.extend(js)
+    row_ptr = np.zeros(len(counts) + 1, dtype=np.int32)
+    row_ptr[1:] = np.cumsum(counts)
+    return row_ptr, np.asarray(cols, dtype=np.int32)

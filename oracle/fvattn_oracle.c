@@ -1,0 +1,482 @@
+/*
+ * fvattn_oracle.c -- TEST INFRASTRUCTURE, not part of the product.
+ *
+ * A plain, slow, fp64 CPU statement of what top-p routed block-sparse attention
+ * computes.  Only the test suite, the smoke check and the benchmark's CPU
+ * baseline leg load this library.  It shares no code, header, table or helper
+ * with the CUDA library; the two meet only in the seeded input generators.
+ *
+ * Sources (page title, then section):
+ *  [FVAttn]  "[논문리뷰] FVAttn: Adaptive Sparse Attention with Runtime Load
+ *            Balancing for Video Generation", §1 Key Terms (Top-p routing):
+ *            for every query block, key blocks are taken in order of an
+ *            importance score until their cumulative probability reaches p.
+ *            §1 (RLB) and §2: the per-head amount of work is what is balanced.
+ *  [FA]      "FlashAttention - Fast and Memory-Efficient Exact Attention with
+ *            IO-Awareness" review, §Background [3] Motivation: S = QK^T,
+ *            P = softmax(S), O = PV; §Model "Tiling Softmax": the row softmax
+ *            is computed block by block and the partial results are combined
+ *            exactly.
+ *
+ * The pages name the routing score but never define it.  This library fixes
+ * it as: mean-pool every block of `bs` tokens of Q and of K (over the tokens
+ * that exist), score = qbar . kbar / sqrt(d), softmax over all key blocks,
+ * and keep the shortest prefix of key blocks -- sorted by descending score,
+ * equal scores by ascending index -- whose probability mass is >= p
+ * (p >= 1 keeps every block).
+ *
+ * Precision: bf16 inputs are widened to fp64 exactly; every sum runs in fp64
+ * in index order.  Compile with -ffp-contract=off so that a*b+c is two
+ * roundings, exactly as written.
+ *
+ * Parity pins (what this file is checked against, in tests/):
+ *   pool        closed forms (constant and ramp blocks, ragged last block)
+ *   route       top-p invariants, K = 0 uniform closed form (tie-break),
+ *               one-hot block, p -> 0+ argmax, p = 1 all blocks, monotone in p,
+ *               exhaustive subset search on tiny rows
+ *   attn_rows   high-precision Decimal brute force on tiny inputs, closed
+ *               forms (single key, K = 0 mean of V, constant V)
+ *   attn_tiled  equals attn_rows (the "exact" tiling identity of [FA])
+ *   lpt_order   brute-force sort on small inputs
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ---------------------------------------------------------------- helpers */
+
+static double bf16_bits_to_double(uint16_t h) {
+    uint32_t u = ((uint32_t)h) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f; /* float -> double is exact */
+}
+
+static int64_t num_blocks(int N, int bs) { return ((int64_t)N + bs - 1) / bs; }
+
+/* Simple parallel-for over [0, n) with a fixed number of threads. */
+typedef void (*range_fn)(void *ctx, int64_t begin, int64_t end);
+typedef struct {
+    range_fn fn;
+    void *ctx;
+    int64_t begin, end;
+} range_job;
+
+static void *range_trampoline(void *arg) {
+    range_job *j = (range_job *)arg;
+    j->fn(j->ctx, j->begin, j->end);
+    return NULL;
+}
+
+static void parallel_for(int64_t n, int nthreads, range_fn fn, void *ctx) {
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > 256) nthreads = 256;
+    if (n < nthreads) nthreads = (int)(n > 0 ? n : 1);
+    if (nthreads == 1) {
+        fn(ctx, 0, n);
+        return;
+    }
+    pthread_t th[256];
+    range_job jobs[256];
+    int started[256];
+    int64_t chunk = (n + nthreads - 1) / nthreads;
+    for (int i = 0; i < nthreads; ++i) {
+        jobs[i].fn = fn;
+        jobs[i].ctx = ctx;
+        jobs[i].begin = i * chunk < n ? i * chunk : n;
+        jobs[i].end = (i + 1) * chunk < n ? (i + 1) * chunk : n;
+        started[i] = pthread_create(&th[i], NULL, range_trampoline, &jobs[i]) == 0;
+        if (!started[i]) fn(ctx, jobs[i].begin, jobs[i].end);
+    }
+    for (int i = 0; i < nthreads; ++i)
+        if (started[i]) pthread_join(th[i], NULL);
+}
+
+/* ------------------------------------------------------------ mean pooling */
+/*
+ * out[bh, i, c] = (1/n_i) * sum_{t in block i, t < N} X[bh, t, c]
+ * n_i counts only the tokens that exist (the last block may be ragged).
+ */
+typedef struct {
+    const uint16_t *X;
+    int N, d, bs;
+    int64_t nb;
+    double *out;
+} pool_ctx;
+
+static void pool_range(void *vctx, int64_t begin, int64_t end) {
+    pool_ctx *c = (pool_ctx *)vctx;
+    for (int64_t u = begin; u < end; ++u) { /* u = bh * nb + i */
+        int64_t bh = u / c->nb, i = u % c->nb;
+        int64_t t0 = i * c->bs, t1 = t0 + c->bs;
+        if (t1 > c->N) t1 = c->N;
+        double *o = c->out + u * c->d;
+        for (int ch = 0; ch < c->d; ++ch) {
+            double s = 0.0;
+            for (int64_t t = t0; t < t1; ++t)
+                s = s + bf16_bits_to_double(c->X[(bh * c->N + t) * c->d + ch]);
+            o[ch] = s / (double)(t1 - t0);
+        }
+    }
+}
+
+int oracle_pool(const uint16_t *X, int64_t BH, int N, int d, int bs, double *out, int nthreads) {
+    if (!X || !out || BH < 0 || N < 1 || d < 1 || bs < 1) return -1;
+    pool_ctx c = {X, N, d, bs, num_blocks(N, bs), out};
+    parallel_for(BH * c.nb, nthreads, pool_range, &c);
+    return 0;
+}
+
+/* ------------------------------------------------------------ top-p routing */
+
+typedef struct {
+    double s; /* score */
+    int j;    /* key-block index */
+} scored_block;
+
+/* Descending score; equal scores by ascending index. */
+static int by_score_desc_index_asc(const void *a, const void *b) {
+    const scored_block *x = (const scored_block *)a, *y = (const scored_block *)b;
+    if (x->s > y->s) return -1;
+    if (x->s < y->s) return 1;
+    return (x->j > y->j) - (x->j < y->j);
+}
+
+typedef struct {
+    const double *qbar, *kbar; /* [BH, nb, d] */
+    int d;
+    int64_t nb;
+    double p, scale;
+    int32_t *counts;  /* [rows] */
+    uint8_t *chosen;  /* [rows, nb] 0/1 */
+    double *diag;     /* [rows, 6] or NULL */
+} route_ctx;
+
+/*
+ * One row = one (b, h, query block i).  Steps in the order of [FVAttn] §1:
+ * importance score per key block, probability by softmax, then key blocks in
+ * descending order until the cumulative probability reaches p.
+ */
+static void route_range(void *vctx, int64_t begin, int64_t end) {
+    route_ctx *c = (route_ctx *)vctx;
+    int64_t nb = c->nb;
+    scored_block *sb = (scored_block *)malloc(sizeof(scored_block) * nb);
+    double *prob = (double *)malloc(sizeof(double) * nb);
+    if (!sb || !prob) {
+        free(sb);
+        free(prob);
+        return;
+    }
+    for (int64_t row = begin; row < end; ++row) {
+        int64_t bh = row / nb;
+        const double *q = c->qbar + row * c->d;
+        /* scores s_j = (qbar_i . kbar_j) * (1/sqrt(d)) */
+        double smax = -INFINITY;
+        for (int64_t j = 0; j < nb; ++j) {
+            const double *k = c->kbar + (bh * nb + j) * c->d;
+            double dot = 0.0;
+            for (int ch = 0; ch < c->d; ++ch) dot = dot + q[ch] * k[ch];
+            sb[j].s = dot * c->scale;
+            sb[j].j = (int)j;
+            if (sb[j].s > smax) smax = sb[j].s;
+        }
+        /* softmax over key blocks */
+        double z = 0.0;
+        for (int64_t j = 0; j < nb; ++j) {
+            prob[j] = exp(sb[j].s - smax);
+            z = z + prob[j];
+        }
+        for (int64_t j = 0; j < nb; ++j) prob[j] = prob[j] / z;
+        /* order by score, cut where the cumulative mass first reaches p */
+        qsort(sb, (size_t)nb, sizeof(scored_block), by_score_desc_index_asc);
+        int64_t k = nb - 1; /* p >= 1, or mass never reaches p: all blocks */
+        double cum = 0.0, cum_prev = 0.0, cum_at_k = 0.0;
+        if (c->p < 1.0) {
+            for (int64_t r = 0; r < nb; ++r) {
+                cum_prev = cum;
+                cum = cum + prob[sb[r].j];
+                if (cum >= c->p) {
+                    k = r;
+                    break;
+                }
+            }
+            cum_at_k = cum;
+        } else {
+            for (int64_t r = 0; r < nb; ++r) {
+                cum_prev = cum;
+                cum = cum + prob[sb[r].j];
+            }
+            cum_at_k = cum;
+        }
+        uint8_t *ch = c->chosen + row * nb;
+        for (int64_t j = 0; j < nb; ++j) ch[j] = 0;
+        for (int64_t r = 0; r <= k; ++r) ch[sb[r].j] = 1;
+        c->counts[row] = (int32_t)(k + 1);
+        if (c->diag) {
+            double *g = c->diag + row * 6;
+            g[0] = cum_at_k;                                     /* mass kept */
+            g[1] = cum_prev;                                     /* mass without the last kept block */
+            g[2] = sb[k].s;                                      /* last kept score */
+            g[3] = (k + 1 < nb) ? sb[k + 1].s : -INFINITY;       /* first dropped score */
+            g[4] = prob[sb[k].j];                                /* last kept probability */
+            g[5] = (k + 1 < nb) ? prob[sb[k + 1].j] : 0.0;       /* first dropped probability */
+        }
+    }
+    free(sb);
+    free(prob);
+}
+
+/*
+ * Full routing: pooled Q and K, scores, softmax, top-p selection, CSR with
+ * ascending column indices inside each row, and per-head selected-block counts.
+ * Returns 0, -1 on bad arguments, -4 when col_capacity is too small.
+ */
+int oracle_route(const uint16_t *Q, const uint16_t *K, int B, int H, int N, int d, int bs, double p,
+                 int32_t *row_ptr, int32_t *col_idx, int64_t col_capacity, int32_t *head_counts,
+                 double *diag, int nthreads) {
+    if (!Q || !K || !row_ptr || !head_counts || B < 1 || H < 1 || N < 1 || d < 1 || bs < 1) return -1;
+    if (!(p > 0.0) || p > 1.0) return -1;
+    int64_t BH = (int64_t)B * H, nb = num_blocks(N, bs), rows = BH * nb;
+    double *qbar = (double *)malloc(sizeof(double) * rows * d);
+    double *kbar = (double *)malloc(sizeof(double) * rows * d);
+    int32_t *counts = (int32_t *)malloc(sizeof(int32_t) * rows);
+    uint8_t *chosen = (uint8_t *)malloc((size_t)(rows * nb));
+    int rc = 0;
+    if (!qbar || !kbar || !counts || !chosen) {
+        rc = -1;
+        goto done;
+    }
+    oracle_pool(Q, BH, N, d, bs, qbar, nthreads);
+    oracle_pool(K, BH, N, d, bs, kbar, nthreads);
+    route_ctx c = {qbar, kbar, d, nb, p, 1.0 / sqrt((double)d), counts, chosen, diag};
+    parallel_for(rows, nthreads, route_range, &c);
+    /* CSR: exclusive prefix sum of the row counts, columns ascending */
+    int64_t total = 0;
+    for (int64_t r = 0; r < rows; ++r) {
+        row_ptr[r] = (int32_t)total;
+        total += counts[r];
+    }
+    row_ptr[rows] = (int32_t)total;
+    if (total > col_capacity || !col_idx) {
+        rc = -4;
+    } else {
+        for (int64_t r = 0; r < rows; ++r) {
+            int64_t w = row_ptr[r];
+            for (int64_t j = 0; j < nb; ++j)
+                if (chosen[r * nb + j]) col_idx[w++] = (int32_t)j;
+        }
+    }
+    for (int64_t bh = 0; bh < BH; ++bh) {
+        int64_t s = 0;
+        for (int64_t i = 0; i < nb; ++i) s += counts[bh * nb + i];
+        head_counts[bh] = (int32_t)s;
+    }
+done:
+    free(qbar);
+    free(kbar);
+    free(counts);
+    free(chosen);
+    return rc;
+}
+
+/* ------------------------------------------------- attention, row by row */
+
+typedef struct {
+    const uint16_t *Q, *K, *V;
+    int H, N, d, bs, causal;
+    int64_t nb;
+    const int32_t *row_ptr, *col_idx;
+    const int64_t *tokens; /* global token index bh*N + t */
+    double *O, *LSE;
+    double scale;
+} attn_ctx;
+
+/*
+ * The textbook definition of [FA] §Motivation, restricted to the key tokens
+ * of the blocks listed in the query token's CSR row (and u <= t if causal):
+ *   s_u = q_t . k_u / sqrt(d),  O_t = sum_u softmax(s)_u v_u,
+ *   LSE_t = ln sum_u exp(s_u).
+ * An empty key set gives O = 0 and LSE = -inf.
+ */
+static void attn_rows_range(void *vctx, int64_t begin, int64_t end) {
+    attn_ctx *c = (attn_ctx *)vctx;
+    int d = c->d;
+    double *q = (double *)malloc(sizeof(double) * d);
+    double *acc = (double *)malloc(sizeof(double) * d);
+    int64_t cap = c->nb * c->bs;
+    double *s = (double *)malloc(sizeof(double) * cap);
+    int64_t *u_of = (int64_t *)malloc(sizeof(int64_t) * cap);
+    if (!q || !acc || !s || !u_of) goto out;
+    for (int64_t it = begin; it < end; ++it) {
+        int64_t g = c->tokens[it], bh = g / c->N, t = g % c->N;
+        int64_t row = bh * c->nb + t / c->bs;
+        for (int ch = 0; ch < d; ++ch) q[ch] = bf16_bits_to_double(c->Q[g * d + ch]);
+        int64_t n = 0;
+        double m = -INFINITY;
+        for (int32_t e = c->row_ptr[row]; e < c->row_ptr[row + 1]; ++e) {
+            int64_t kb = c->col_idx[e];
+            for (int64_t u = kb * c->bs; u < (kb + 1) * c->bs && u < c->N; ++u) {
+                if (c->causal && u > t) continue;
+                const uint16_t *k = c->K + (bh * c->N + u) * d;
+                double dot = 0.0;
+                for (int ch = 0; ch < d; ++ch) dot = dot + q[ch] * bf16_bits_to_double(k[ch]);
+                s[n] = dot * c->scale;
+                u_of[n] = u;
+                if (s[n] > m) m = s[n];
+                ++n;
+            }
+        }
+        double *o = c->O + it * d;
+        if (n == 0) {
+            for (int ch = 0; ch < d; ++ch) o[ch] = 0.0;
+            c->LSE[it] = -INFINITY;
+            continue;
+        }
+        double z = 0.0;
+        for (int ch = 0; ch < d; ++ch) acc[ch] = 0.0;
+        for (int64_t a = 0; a < n; ++a) {
+            double w = exp(s[a] - m);
+            z = z + w;
+            const uint16_t *v = c->V + (bh * c->N + u_of[a]) * d;
+            for (int ch = 0; ch < d; ++ch) acc[ch] = acc[ch] + w * bf16_bits_to_double(v[ch]);
+        }
+        for (int ch = 0; ch < d; ++ch) o[ch] = acc[ch] / z;
+        c->LSE[it] = m + log(z);
+    }
+out:
+    free(q);
+    free(acc);
+    free(s);
+    free(u_of);
+}
+
+int oracle_attn_rows(const uint16_t *Q, const uint16_t *K, const uint16_t *V, int B, int H, int N, int d, int bs,
+                     int causal, const int32_t *row_ptr, const int32_t *col_idx, const int64_t *tokens,
+                     int64_t ntok, double *O, double *LSE, int nthreads) {
+    if (!Q || !K || !V || !row_ptr || !col_idx || !tokens || !O || !LSE) return -1;
+    if (B < 1 || H < 1 || N < 1 || d < 1 || bs < 1) return -1;
+    int64_t total = (int64_t)B * H * N;
+    for (int64_t i = 0; i < ntok; ++i)
+        if (tokens[i] < 0 || tokens[i] >= total) return -1;
+    attn_ctx c = {Q, K, V, H, N, d, bs, causal ? 1 : 0, num_blocks(N, bs), row_ptr, col_idx, tokens, O, LSE,
+                  1.0 / sqrt((double)d)};
+    parallel_for(ntok, nthreads, attn_rows_range, &c);
+    return 0;
+}
+
+/* -------------------------------------- attention, tiled online softmax */
+
+/*
+ * The same quantity, computed the way [FA] §Model "Tiling Softmax" describes:
+ * one key block at a time, keeping a running maximum m, a running sum l and
+ * an unnormalised output; when the maximum grows from m to m', the old sum
+ * and output are scaled by exp(m - m').  In exact arithmetic this equals
+ * attn_rows; the tests pin the two against each other.
+ */
+static void attn_tiled_range(void *vctx, int64_t begin, int64_t end) {
+    attn_ctx *c = (attn_ctx *)vctx;
+    int d = c->d;
+    double *q = (double *)malloc(sizeof(double) * d);
+    double *acc = (double *)malloc(sizeof(double) * d);
+    double *s = (double *)malloc(sizeof(double) * c->bs);
+    int64_t *u_of = (int64_t *)malloc(sizeof(int64_t) * c->bs);
+    if (!q || !acc || !s || !u_of) goto out;
+    for (int64_t it = begin; it < end; ++it) {
+        int64_t g = c->tokens[it], bh = g / c->N, t = g % c->N;
+        int64_t row = bh * c->nb + t / c->bs;
+        for (int ch = 0; ch < d; ++ch) {
+            q[ch] = bf16_bits_to_double(c->Q[g * d + ch]);
+            acc[ch] = 0.0;
+        }
+        double m = -INFINITY, l = 0.0;
+        for (int32_t e = c->row_ptr[row]; e < c->row_ptr[row + 1]; ++e) {
+            int64_t kb = c->col_idx[e];
+            int n = 0;
+            double mt = -INFINITY;
+            for (int64_t u = kb * c->bs; u < (kb + 1) * c->bs && u < c->N; ++u) {
+                if (c->causal && u > t) continue;
+                const uint16_t *k = c->K + (bh * c->N + u) * d;
+                double dot = 0.0;
+                for (int ch = 0; ch < d; ++ch) dot = dot + q[ch] * bf16_bits_to_double(k[ch]);
+                s[n] = dot * c->scale;
+                u_of[n] = u;
+                if (s[n] > mt) mt = s[n];
+                ++n;
+            }
+            if (n == 0) continue;
+            double mn = mt > m ? mt : m;
+            double alpha = (m == -INFINITY) ? 0.0 : exp(m - mn);
+            l = l * alpha;
+            for (int ch = 0; ch < d; ++ch) acc[ch] = acc[ch] * alpha;
+            for (int a = 0; a < n; ++a) {
+                double w = exp(s[a] - mn);
+                l = l + w;
+                const uint16_t *v = c->V + (bh * c->N + u_of[a]) * d;
+                for (int ch = 0; ch < d; ++ch) acc[ch] = acc[ch] + w * bf16_bits_to_double(v[ch]);
+            }
+            m = mn;
+        }
+        double *o = c->O + it * d;
+        if (l == 0.0) {
+            for (int ch = 0; ch < d; ++ch) o[ch] = 0.0;
+            c->LSE[it] = -INFINITY;
+        } else {
+            for (int ch = 0; ch < d; ++ch) o[ch] = acc[ch] / l;
+            c->LSE[it] = m + log(l);
+        }
+    }
+out:
+    free(q);
+    free(acc);
+    free(s);
+    free(u_of);
+}
+
+int oracle_attn_tiled(const uint16_t *Q, const uint16_t *K, const uint16_t *V, int B, int H, int N, int d, int bs,
+                      int causal, const int32_t *row_ptr, const int32_t *col_idx, const int64_t *tokens,
+                      int64_t ntok, double *O, double *LSE, int nthreads) {
+    if (!Q || !K || !V || !row_ptr || !col_idx || !tokens || !O || !LSE) return -1;
+    if (B < 1 || H < 1 || N < 1 || d < 1 || bs < 1) return -1;
+    int64_t total = (int64_t)B * H * N;
+    for (int64_t i = 0; i < ntok; ++i)
+        if (tokens[i] < 0 || tokens[i] >= total) return -1;
+    attn_ctx c = {Q, K, V, H, N, d, bs, causal ? 1 : 0, num_blocks(N, bs), row_ptr, col_idx, tokens, O, LSE,
+                  1.0 / sqrt((double)d)};
+    parallel_for(ntok, nthreads, attn_tiled_range, &c);
+    return 0;
+}
+
+/* ----------------------------------------------- longest-first work order */
+
+typedef struct {
+    int64_t count;
+    int64_t id;
+} work_item;
+
+static int by_count_desc_id_asc(const void *a, const void *b) {
+    const work_item *x = (const work_item *)a, *y = (const work_item *)b;
+    if (x->count != y->count) return x->count > y->count ? -1 : 1;
+    return (x->id > y->id) - (x->id < y->id);
+}
+
+/*
+ * Work items are the CSR rows (one query block of one head).  The order is
+ * longest first -- descending selected-block count, equal counts by ascending
+ * row id -- the single-GPU counterpart of balancing per-head work after the
+ * mask is known ([FVAttn] §1 RLB, §3).
+ */
+int oracle_lpt_order(const int32_t *row_ptr, int64_t rows, int32_t *order) {
+    if (!row_ptr || !order || rows < 0) return -1;
+    work_item *w = (work_item *)malloc(sizeof(work_item) * (rows > 0 ? rows : 1));
+    if (!w) return -1;
+    for (int64_t r = 0; r < rows; ++r) {
+        w[r].count = (int64_t)row_ptr[r + 1] - row_ptr[r];
+        w[r].id = r;
+    }
+    qsort(w, (size_t)rows, sizeof(work_item), by_count_desc_id_asc);
+    for (int64_t r = 0; r < rows; ++r) order[r] = (int32_t)w[r].id;
+    free(w);
+    return 0;
+}

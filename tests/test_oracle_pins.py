@@ -1,0 +1,415 @@
+"""Pins for the fp64 CPU oracle (no GPU).
+
+Each test checks the oracle against something other than itself: exact
+rational or 50-digit Decimal brute force of the definitions, closed forms and
+the invariants of the top-p rule.
+
+Definitions followed (page title, section):
+  * FVAttn review, §1 Key Terms "Top-p routing": key blocks are added in order
+    of importance until the cumulative probability reaches p.
+  * FlashAttention review, §Background "Motivation": S = QK^T, P = softmax(S),
+    O = PV; §Model "Tiling Softmax": block-wise softmax combines exactly.
+The routing score itself (mean-pooled blocks, qbar.kbar/sqrt(d), softmax over
+key blocks, ties to the lower index) is this library's reading, since the
+pages only name it.
+"""
+from __future__ import annotations
+
+import itertools
+import math
+from decimal import Decimal, getcontext
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+from workloads import bf16_bits_to_f32, f32_to_bf16_bits
+
+getcontext().prec = 60
+
+
+def bf16(a) -> np.ndarray:
+    return f32_to_bf16_bits(np.asarray(a, dtype=np.float32))
+
+
+def rand_bf16(rng, shape, scale=1.0):
+    return bf16(rng.standard_normal(shape).astype(np.float32) * scale)
+
+
+def fvals(bits: np.ndarray) -> np.ndarray:
+    return bf16_bits_to_f32(bits).astype(np.float64)
+
+
+# ----------------------------------------------------------------- pooling
+
+def test_pool_constant_blocks(oracle_mod):
+    N, bs, d = 200, 64, 8
+    X = np.zeros((1, 2, N, d), np.float32)
+    for h in range(2):
+        for i in range(4):
+            X[0, h, i * bs:(i + 1) * bs] = (h * 4 + i) * 0.5 - 1.25
+    out = oracle_mod.pool(bf16(X), bs)
+    for h in range(2):
+        for i in range(4):
+            assert np.all(out[0, h, i] == (h * 4 + i) * 0.5 - 1.25)
+
+
+def test_pool_ragged_block_divides_by_valid_tokens(oracle_mod):
+    N, bs, d = 70, 64, 4
+    X = np.zeros((1, 1, N, d), np.float32)
+    for t in range(N):
+        for c in range(d):
+            X[0, 0, t, c] = (t % 7) - 3 + 0.25 * c
+    out = oracle_mod.pool(bf16(X), bs)
+    for i, (t0, t1) in enumerate([(0, 64), (64, 70)]):
+        for c in range(d):
+            exact = sum(Fraction(float(X[0, 0, t, c])) for t in range(t0, t1)) / (t1 - t0)
+            assert abs(Fraction(out[0, 0, i, c]) - exact) <= abs(exact) * Fraction(1, 2**50) + Fraction(1, 2**60)
+    # the last block holds 6 tokens; dividing by the block size would be 64/6 times smaller
+    assert out[0, 0, 1, 0] != 0.0
+
+
+# ------------------------------------------------------- attention (rows)
+
+def decimal_attention(q, keys, vals):
+    """50-digit brute force of softmax(q.k/sqrt(d)) v over the given keys."""
+    d = len(q)
+    if not keys:
+        return [Decimal(0)] * d, None
+    scale = Decimal(1) / Decimal(d).sqrt()
+    s = [sum(Decimal(float(q[c])) * Decimal(float(k[c])) for c in range(d)) * scale for k in keys]
+    m = max(s)
+    w = [(x - m).exp() for x in s]
+    z = sum(w)
+    out = [sum(w[a] * Decimal(float(vals[a][c])) for a in range(len(vals))) / z for c in range(d)]
+    return out, m + z.ln()
+
+
+def random_csr(rng, rows, nb, p_keep=0.5, allow_empty=True):
+    row_ptr = [0]
+    cols = []
+    for r in range(rows):
+        sel = [j for j in range(nb) if rng.random() < p_keep]
+        if not sel and not allow_empty:
+            sel = [int(rng.integers(nb))]
+        cols.extend(sel)
+        row_ptr.append(len(cols))
+    return np.asarray(row_ptr, np.int32), np.asarray(cols, np.int32)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N,bs,d", [(11, 4, 4), (8, 4, 8), (1, 4, 4), (9, 3, 2)])
+def test_attn_rows_matches_decimal_brute_force(oracle_mod, N, bs, d, causal):
+    rng = np.random.default_rng(N * 100 + bs * 10 + d + causal)
+    B, H = 1, 2
+    Q, K, V = (rand_bf16(rng, (B, H, N, d)) for _ in range(3))
+    nb = -(-N // bs)
+    row_ptr, col_idx = random_csr(rng, B * H * nb, nb)
+    # the first row empty and the second row full, whatever the draw
+    counts = np.diff(row_ptr).tolist()
+    rows_cols = [list(col_idx[row_ptr[r]:row_ptr[r + 1]]) for r in range(len(counts))]
+    rows_cols[0] = []
+    if len(rows_cols) > 1:
+        rows_cols[1] = list(range(nb))
+    row_ptr = np.zeros(len(rows_cols) + 1, np.int32)
+    row_ptr[1:] = np.cumsum([len(c) for c in rows_cols])
+    col_idx = np.asarray([j for c in rows_cols for j in c], np.int32)
+    tokens = np.arange(B * H * N, dtype=np.int64)
+    O, LSE = oracle_mod.attn_rows(Q, K, V, bs, causal, row_ptr, col_idx, tokens)
+    Ot, LSEt = oracle_mod.attn_tiled(Q, K, V, bs, causal, row_ptr, col_idx, tokens)
+    Qf, Kf, Vf = fvals(Q), fvals(K), fvals(V)
+    for g in tokens:
+        bh, t = divmod(int(g), N)
+        b, h = divmod(bh, H)
+        row = bh * nb + t // bs
+        keys = []
+        for e in range(row_ptr[row], row_ptr[row + 1]):
+            kb = int(col_idx[e])
+            for u in range(kb * bs, min(N, kb * bs + bs)):
+                if causal and u > t:
+                    continue
+                keys.append(u)
+        ref_o, ref_lse = decimal_attention(Qf[b, h, t], [Kf[b, h, u] for u in keys], [Vf[b, h, u] for u in keys])
+        for impl_o, impl_lse in ((O, LSE), (Ot, LSEt)):
+            assert np.allclose(impl_o[g], [float(x) for x in ref_o], rtol=0, atol=1e-12)
+            if ref_lse is None:
+                assert impl_lse[g] == -np.inf
+            else:
+                assert abs(impl_lse[g] - float(ref_lse)) <= 1e-12
+
+
+def test_attn_closed_form_zero_keys_gives_mean_of_values(oracle_mod):
+    rng = np.random.default_rng(7)
+    B, H, N, d, bs = 1, 1, 40, 8, 16
+    Q = rand_bf16(rng, (B, H, N, d))
+    K = bf16(np.zeros((B, H, N, d)))
+    V = rand_bf16(rng, (B, H, N, d))
+    nb = 3
+    row_ptr = np.array([0, 1, 3, 6], np.int32)
+    col_idx = np.array([2, 0, 2, 0, 1, 2], np.int32)
+    tokens = np.arange(N, dtype=np.int64)
+    O, LSE = oracle_mod.attn_rows(Q, K, V, bs, False, row_ptr, col_idx, tokens)
+    Vf = fvals(V)[0, 0]
+    for t in range(N):
+        row = t // bs
+        keys = [u for e in range(row_ptr[row], row_ptr[row + 1])
+                for u in range(col_idx[e] * bs, min(N, col_idx[e] * bs + bs))]
+        for c in range(d):
+            exact = sum(Fraction(Vf[u, c]) for u in keys) / len(keys)
+            assert abs(O[t, c] - float(exact)) <= 1e-14
+        assert abs(LSE[t] - math.log(len(keys))) <= 1e-14
+    assert nb == 3
+
+
+def test_attn_closed_form_single_key_and_constant_values(oracle_mod):
+    Q = bf16([[[[0.5, -1.0, 2.0, 0.25]]]])
+    K = bf16([[[[1.0, 1.0, -0.5, 4.0]]]])
+    V = bf16([[[[3.0, -2.0, 0.125, 7.0]]]])
+    O, LSE = oracle_mod.attn_rows(Q, K, V, 64, False, np.array([0, 1], np.int32), np.array([0], np.int32),
+                                  np.array([0], np.int64))
+    assert np.array_equal(O[0], [3.0, -2.0, 0.125, 7.0])
+    assert LSE[0] == (0.5 - 1.0 - 1.0 + 1.0) / 2.0
+    rng = np.random.default_rng(3)
+    Q, K = rand_bf16(rng, (1, 1, 100, 16)), rand_bf16(rng, (1, 1, 100, 16), 3.0)
+    V = bf16(np.full((1, 1, 100, 16), 1.5))
+    row_ptr, col_idx = oracle_mod.dense_csr(1, 1, 100, 32)
+    O, _ = oracle_mod.attn_rows(Q, K, V, 32, False, row_ptr, col_idx, np.arange(100, dtype=np.int64))
+    assert np.max(np.abs(O - 1.5)) <= 1e-14
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_tiled_online_softmax_equals_row_softmax(oracle_mod, causal):
+    rng = np.random.default_rng(11)
+    B, H, N, d, bs = 1, 2, 300, 32, 64
+    Q, K, V = rand_bf16(rng, (B, H, N, d), 2.0), rand_bf16(rng, (B, H, N, d), 2.0), rand_bf16(rng, (B, H, N, d))
+    row_ptr, col_idx = random_csr(rng, B * H * 5, 5, p_keep=0.6)
+    tokens = np.arange(B * H * N, dtype=np.int64)
+    O, L = oracle_mod.attn_rows(Q, K, V, bs, causal, row_ptr, col_idx, tokens)
+    Ot, Lt = oracle_mod.attn_tiled(Q, K, V, bs, causal, row_ptr, col_idx, tokens)
+    assert np.max(np.abs(O - Ot)) <= 1e-12
+    fin = np.isfinite(L)
+    assert np.array_equal(fin, np.isfinite(Lt))
+    assert np.max(np.abs(L[fin] - Lt[fin])) <= 1e-12
+
+
+# ------------------------------------------------------------------ routing
+
+def check_csr(route, rows, nb):
+    rp, ci = route.row_ptr, route.col_idx
+    assert rp[0] == 0 and rp.size == rows + 1 and np.all(np.diff(rp) >= 1)
+    for r in range(rows):
+        cols = ci[rp[r]:rp[r + 1]]
+        assert np.all(np.diff(cols) > 0) and cols[0] >= 0 and cols[-1] < nb
+
+
+def test_route_uniform_scores_select_lowest_indices(oracle_mod):
+    """K = 0 makes every score 0 and every probability 1/nb: the kept set is the
+    first ceil(p*nb) blocks by index -- this pins the tie-break."""
+    rng = np.random.default_rng(5)
+    B, H, N, d, bs = 1, 2, 640, 16, 64
+    Q = rand_bf16(rng, (B, H, N, d))
+    K = bf16(np.zeros((B, H, N, d)))
+    for p, expect in ((0.35, 4), (0.55, 6), (0.73, 8), (0.05, 1)):
+        r = oracle_mod.route(Q, K, p, bs)
+        check_csr(r, B * H * 10, 10)
+        assert np.all(r.counts == expect)
+        for row in range(B * H * 10):
+            assert list(r.col_idx[r.row_ptr[row]:r.row_ptr[row + 1]]) == list(range(expect))
+        assert np.all(r.head_counts == 10 * expect)
+
+
+def test_route_reaching_p_exactly_counts(oracle_mod):
+    """Eight uniform blocks (probability 1/8, exact in binary): with p = 1/2 the
+    mass of four blocks equals p exactly, and "reaches p" keeps four, not five."""
+    rng = np.random.default_rng(6)
+    Q = rand_bf16(rng, (1, 1, 512, 16))
+    K = bf16(np.zeros((1, 1, 512, 16)))
+    r = oracle_mod.route(Q, K, 0.5, 64)
+    assert np.all(r.counts == 4)
+    assert np.all(r.diag[:, 0] == 0.5)
+
+
+def test_route_worked_example_by_hand(oracle_mod):
+    """Hand-derived instance.  Q tokens all (1,0,0,0); K block means in channel 0
+    are (0, 2, 1, 2) for blocks 0..3 (d=4, so scale 1/2): scores (0, 1, .5, 1).
+    Probabilities e^s/Z with Z = 1 + 2e + e^.5 are (.1237, .3362, .2039, .3362).
+    Order by score, equal scores by index: 1, 3, 2, 0; cumulative mass
+    .3362, .6724, .8763, 1.  Hence p=.3 -> {1}; p=.5 -> {1,3}; p=.7 -> {1,2,3};
+    p=.9 -> {0,1,2,3}."""
+    N, bs, d = 8, 2, 4
+    Q = np.zeros((1, 1, N, d), np.float32)
+    Q[..., 0] = 1.0
+    K = np.zeros((1, 1, N, d), np.float32)
+    K[0, 0, 2:4, 0] = [1.0, 3.0]   # mean 2
+    K[0, 0, 4:6, 0] = [0.5, 1.5]   # mean 1
+    K[0, 0, 6:8, 0] = [2.0, 2.0]   # mean 2
+    K[0, 0, 0:2, 1] = [5.0, -5.0]  # block 0 mean 0 in every channel
+    z = 1 + 2 * math.e + math.exp(0.5)
+    probs = [1 / z, math.e / z, math.exp(0.5) / z, math.e / z]
+    assert abs(probs[1] + probs[3] - 0.6724) < 1e-4
+    for p, want in ((0.3, [1]), (0.5, [1, 3]), (0.7, [1, 2, 3]), (0.9, [0, 1, 2, 3])):
+        r = oracle_mod.route(bf16(Q), bf16(K), p, bs)
+        for row in range(4):
+            assert list(r.col_idx[r.row_ptr[row]:r.row_ptr[row + 1]]) == want
+        assert r.head_counts[0] == 4 * len(want)
+
+
+def test_route_one_hot_block(oracle_mod):
+    B, H, N, d, bs = 1, 1, 640, 16, 64
+    Q = bf16(np.ones((B, H, N, d)))
+    Kf = np.zeros((B, H, N, d), np.float32)
+    Kf[0, 0, 5 * bs:6 * bs] = 4.0   # score 4*16/4 = 16 against 0 elsewhere
+    r = oracle_mod.route(Q, bf16(Kf), 0.99, bs)
+    assert np.all(r.counts == 1) and np.all(r.col_idx == 5)
+
+
+def test_route_p_to_zero_is_argmax_with_lowest_index(oracle_mod):
+    B, H, N, d, bs = 1, 1, 640, 16, 64
+    Q = bf16(np.ones((B, H, N, d)))
+    Kf = np.zeros((B, H, N, d), np.float32)
+    Kf[0, 0, 2 * bs:3 * bs] = 1.0
+    Kf[0, 0, 7 * bs:8 * bs] = 1.0
+    r = oracle_mod.route(Q, bf16(Kf), 1e-300, bs)
+    assert np.all(r.counts == 1) and np.all(r.col_idx == 2)
+
+
+def test_route_p_one_keeps_every_block(oracle_mod):
+    rng = np.random.default_rng(9)
+    Q, K = rand_bf16(rng, (2, 3, 500, 32), 3.0), rand_bf16(rng, (2, 3, 500, 32), 3.0)
+    r = oracle_mod.route(Q, K, 1.0, 64)
+    nb = 8
+    assert np.all(r.counts == nb)
+    rp, ci = oracle_mod.dense_csr(2, 3, 500, 64)
+    assert np.array_equal(r.row_ptr, rp) and np.array_equal(r.col_idx, ci)
+
+
+def test_route_invariants_and_monotone_in_p(oracle_mod):
+    from workloads import Workload, generate
+    w = Workload("t", B=1, H=4, N=24 * 32, d=32, bs=32, p=0.9, dist="structured", grid=(3, 16, 16),
+                 head_scale=("uniform", 0.5, 4.0), seed=21)
+    Q, K, _ = generate(w)
+    prev = None
+    for p in (0.1, 0.3, 0.5, 0.7, 0.9, 0.95, 0.99):
+        r = oracle_mod.route(Q, K, p, w.bs)
+        check_csr(r, w.rows, w.nb)
+        g = r.diag
+        assert np.all(g[:, 0] >= p)                       # kept mass reaches p
+        assert np.all(g[:, 1] < p)                        # one block fewer does not
+        assert np.all(g[:, 2] >= g[:, 3])                 # kept scores >= dropped scores
+        assert np.all(g[:, 4] >= g[:, 5])                 # kept probability >= dropped
+        hc = r.counts.reshape(w.B * w.H, w.nb).sum(1)
+        assert np.array_equal(hc, r.head_counts)
+        if prev is not None:
+            assert np.all(r.counts >= prev)
+        prev = r.counts
+
+
+def exact_route_row(qbar, kbars, p):
+    """Exact scores (d a perfect square) and 60-digit probabilities; the shortest
+    set reaching p found by exhaustive search over subsets."""
+    d = len(qbar)
+    root = math.isqrt(d)
+    assert root * root == d
+    s = [sum(qbar[c] * k[c] for c in range(d)) / root for k in kbars]
+    m = max(s)
+    e = [(Decimal(x.numerator) / Decimal(x.denominator) - Decimal(m.numerator) / Decimal(m.denominator)).exp()
+         for x in s]
+    z = sum(e)
+    prob = [x / z for x in e]
+    nb = len(kbars)
+    P = Decimal(repr(p))
+    for size in range(1, nb + 1):
+        best = None
+        for sub in itertools.combinations(range(nb), size):
+            mass = sum(prob[j] for j in sub)
+            if mass >= P and (best is None or mass > best[0]):
+                best = (mass, sub)
+        if best is not None:
+            order = sorted(range(nb), key=lambda j: (-s[j], j))
+            chosen = sorted(order[:size])
+            top_mass = sum(prob[j] for j in chosen)
+            near = min(abs(top_mass - P), abs(top_mass - prob[order[size - 1]] - P))
+            return chosen, near
+    return list(range(nb)), Decimal(0)
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2, 3])
+def test_route_matches_exhaustive_exact_search(oracle_mod, seed):
+    rng = np.random.default_rng(seed)
+    B, H, N, d, bs = 1, 2, 6 * 4 - 1, 16, 4      # 6 blocks, the last ragged
+    Q, K = rand_bf16(rng, (B, H, N, d), 2.0), rand_bf16(rng, (B, H, N, d), 2.0)
+    Qf, Kf = fvals(Q), fvals(K)
+    nb = 6
+
+    def pooled(X, bh, i):
+        t0, t1 = i * bs, min(N, i * bs + bs)
+        return [sum(Fraction(X[0, bh, t, c]) for t in range(t0, t1)) / (t1 - t0) for c in range(d)]
+
+    for p in (0.2, 0.5, 0.8, 0.95):
+        r = oracle_mod.route(Q, K, p, bs)
+        for bh in range(H):
+            kb = [pooled(Kf, bh, j) for j in range(nb)]
+            for i in range(nb):
+                want, near = exact_route_row(pooled(Qf, bh, i), kb, p)
+                if near < Decimal("1e-9"):
+                    continue
+                row = bh * nb + i
+                assert list(r.col_idx[r.row_ptr[row]:r.row_ptr[row + 1]]) == want
+
+
+# -------------------------------------------------------------- LPT order
+
+def test_lpt_order_brute_force(oracle_mod):
+    rng = np.random.default_rng(4)
+    for rows in (0, 1, 7, 300):
+        counts = rng.integers(0, 12, size=rows)
+        rp = np.zeros(rows + 1, np.int32)
+        rp[1:] = np.cumsum(counts)
+        got = oracle_mod.lpt_order(rp)
+        want = sorted(range(rows), key=lambda r: (-int(counts[r]), r))
+        assert list(got) == want
+
+
+# ------------------------------------------------------ stored fixtures
+
+def test_golden_tiny_route_unchanged(oracle_mod):
+    """tests/golden/tiny_route.json was written by tests/golden/make_golden.py
+    (oracle only); the oracle must keep reproducing it."""
+    import json
+    import os
+    from workloads import TINY, generate
+    with open(os.path.join(os.path.dirname(__file__), "golden", "tiny_route.json")) as f:
+        g = json.load(f)
+    Q, K, _ = generate(TINY)
+    r = oracle_mod.route(Q, K, TINY.p, TINY.bs)
+    assert r.row_ptr.tolist() == g["row_ptr"]
+    assert r.col_idx.tolist() == g["col_idx"]
+    assert r.head_counts.tolist() == g["head_counts"]
+
+
+def test_workload_generators_are_seeded_and_shaped():
+    from workloads import ALL, TINY, Workload, generate
+    a = generate(TINY)
+    b = generate(TINY)
+    assert all(np.array_equal(x, y) for x, y in zip(a, b))
+    assert a[0].shape == (1, 2, 512, 64) and a[0].dtype == np.uint16
+    w = Workload("s", B=1, H=3, N=4 * 6 * 8, d=16, bs=32, p=0.9, dist="structured", grid=(4, 6, 8),
+                 head_scale=("uniform", 0.5, 4.0), seed=5)
+    Q, K, V = generate(w)
+    assert Q.shape == (1, 3, 192, 16)
+    qf, kf, vf = (bf16_bits_to_f32(x).astype(np.float64) for x in (Q, K, V))
+    assert qf.std() > 1.0                                  # noise plus the per-head field
+    assert np.corrcoef(qf.ravel(), kf.ravel())[0, 1] > 0.2  # Q and K share the field
+    assert abs(np.corrcoef(qf.ravel(), vf.ravel())[0, 1]) < 0.1
+    assert ALL["video_dit"].N == 32760 and ALL["video_dit"].nb == 256
+    assert ALL["long_video"].N == 118800 and ALL["long_video"].nb == 929
+    assert len([k for k in ALL if k.startswith("sweep")]) == 20
+
+
+def test_bf16_rounding_is_nearest_even():
+    x = np.array([1.0, 1.0 + 2**-8, 1.0 + 3 * 2**-8, -2.5, 0.0, 1e-30], np.float32)
+    b = f32_to_bf16_bits(x)
+    back = bf16_bits_to_f32(b)
+    assert back[0] == 1.0 and back[1] == 1.0          # tie rounds to even
+    assert back[2] == 1.0 + 2**-6                       # tie rounds up to even
+    assert back[3] == -2.5 and back[4] == 0.0
