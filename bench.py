@@ -1,0 +1,363 @@
+"""Benchmark: one step = top-p routing + longest-first ordering + block-sparse
+attention forward over one synthetic video-latent-like input (B1 H40 N32760
+d128, block 128, p 0.9), with the inputs resident in HBM.
+
+    python bench.py [--gpus N --steps K --warmup W] [--impl reference] [--workload NAME]
+
+Prints one JSON line (rank 0).  Under torchrun every rank runs its own input
+(weak scaling, no data-path collective); time is the max over ranks.
+
+Metric: effective TFLOP/s = 4 * block^2 * d * (selected blocks) / time, the
+work of the selected key blocks counted as full tiles.  ``value`` uses the
+whole step (routing + ordering + attention); ``roofline`` reports the
+attention call alone against the measured bf16 tensor peak.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "effective TFLOP/s & tensor-pipe % of peak (sparse attn fwd, p=0.9); routing ms"
+UNIT = "TFLOP/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+ROUTE_KERNELS_PER_CALL = 4      # pool, select, CSR scan, CSR scatter
+FWD_KERNELS_PER_CALL = 4        # LPT rank, LPT offsets, LPT scatter, attention
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def eff_flops(nnz: int, w: W.Workload) -> float:
+    return 4.0 * w.bs * w.bs * w.d * float(nnz)
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples taken during the timed region."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: str):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu_index), f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.out,
+                                         stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.out.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        mx = [num(r[2]) for r in rows if num(r[2]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def gpu_selector(dev) -> str:
+    """nvidia-smi -i argument for this device (its UUID when torch exposes it)."""
+    import torch
+    try:
+        u = str(torch.cuda.get_device_properties(dev).uuid)
+        if u:
+            return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        pass
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        return vis.split(",")[dev.index or 0].strip()
+    return str(dev.index or 0)
+
+
+def dist_setup(n_gpus: int):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    return rank, world, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# --------------------------------------------------------------- CPU oracle
+
+def oracle_sample(w: W.Workload, Q, K, V, budget_s: float, seed: int = 7):
+    """Times the oracle on a bounded sample: full routing, then whole query blocks
+    (128 rows each) drawn at random until the time budget is spent."""
+    import oracle
+    threads = oracle.default_threads()
+    t0 = time.perf_counter()
+    r = oracle.route(Q, K, w.p, w.bs, nthreads=threads)
+    t_route = time.perf_counter() - t0
+    counts = r.counts
+    rng = np.random.default_rng(seed)
+    items = rng.permutation(w.rows)
+    done_flops = 0.0
+    t_attn = 0.0
+    n_items = 0
+    for row in items:
+        if t_attn >= budget_s:
+            break
+        bh, qb = divmod(int(row), w.nb)
+        t_lo, t_hi = qb * w.bs, min(w.N, (qb + 1) * w.bs)
+        toks = bh * w.N + np.arange(t_lo, t_hi, dtype=np.int64)
+        t1 = time.perf_counter()
+        oracle.attn_rows(Q, K, V, w.bs, w.causal, r.row_ptr, r.col_idx, toks, nthreads=threads)
+        t_attn += time.perf_counter() - t1
+        done_flops += eff_flops(int(counts[row]), w)
+        n_items += 1
+    frac = n_items / w.rows
+    total_t = t_attn + t_route * frac
+    return {
+        "value": done_flops / total_t / 1e12,
+        "unit": UNIT,
+        "cores": threads,
+        "kind": "oracle",
+        "sample": (f"{w.name}: full fp64 routing ({t_route:.2f} s, prorated by {frac:.4f}) + {n_items} of "
+                   f"{w.rows} query blocks of attention ({t_attn:.1f} s)"),
+        "route_s_full": t_route,
+    }
+
+
+def run_reference(args, w, rank, world):
+    if rank != 0:
+        return
+    Q, K, V = W.generate(w)
+    for _ in range(args.warmup):
+        pass  # the oracle has no warm-up state
+    vals = []
+    cb = None
+    per_step = max(2.0, 20.0 / max(1, args.steps))
+    for s in range(args.steps):
+        cb = oracle_sample(w, Q, K, V, budget_s=per_step, seed=1000 + s)
+        vals.append(cb["value"])
+    v = float(np.mean(vals))
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "block": w.bs, "p": w.p,
+                       "causal": w.causal, "l2": "inputs larger than L2"},
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": cb["cores"], "kind": "oracle",
+                             "sample": cb["sample"]},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------ GPU (ours)
+
+def run_ours(args, w, rank, world, local):
+    import torch
+
+    import top_routed_block_b200 as fv
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    Qh, Kh, Vh = W.generate(w, seed=w.seed + rank)
+
+    def pinned(a):
+        t = torch.from_numpy(a.view(np.int16)).view(torch.bfloat16)
+        return t.pin_memory()
+    hQ, hK, hV = pinned(Qh), pinned(Kh), pinned(Vh)
+    dQ, dK, dV = (h.to(dev, non_blocking=True) for h in (hQ, hK, hV))
+    torch.cuda.synchronize(dev)
+    plan = fv.FvattnPlan(w.B, w.H, w.N, w.d, w.bs, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        plan.run_route(dQ, dK, w.p, stream=stream)
+        plan.run_fwd(dQ, dK, dV, w.causal, stream=stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    plan.check()
+    nnz = int(plan.route.row_ptr[-1].item())
+    flops = eff_flops(nnz, w)
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    sampler = ClockSampler(gpu_selector(dev))
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for s in range(args.steps):
+        e0, e1, e2 = ev[s]
+        e0.record(stream)
+        plan.run_route(dQ, dK, w.p, stream=stream)
+        e1.record(stream)
+        plan.run_fwd(dQ, dK, dV, w.causal, stream=stream)
+        e2.record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    clocks = sampler.stop()
+    plan.check()
+    total_ms = t_start.elapsed_time(t_end)
+    route_ms = [a.elapsed_time(b) for a, b, _ in ev]
+    fwd_ms = [b.elapsed_time(c) for _, b, c in ev]
+    total_ms_max = max_over_ranks(total_ms, world)
+    ms_per_step = total_ms_max / args.steps
+    value = world * flops * args.steps / (total_ms_max * 1e-3) / 1e12
+    attn_ms = statistics.mean(fwd_ms)
+    attn_tflops = flops / (attn_ms * 1e-3) / 1e12
+    r_ms = statistics.mean(route_ms)
+
+    # end to end through the host-buffer entry point
+    hO = torch.empty((w.B, w.H, w.N, w.d), dtype=torch.bfloat16).pin_memory()
+    hL = torch.empty((w.B, w.H, w.N), dtype=torch.float32).pin_memory()
+    fv.fvattn_attention_host(hQ, hK, hV, w.p, w.bs, w.causal, plan=plan, dQ=dQ, dK=dK, dV=dV, hO=hO, hLSE=hL,
+                             stream=stream)
+    e2e_steps = max(1, min(args.steps, 5))
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(e2e_steps):
+        fv.fvattn_attention_host(hQ, hK, hV, w.p, w.bs, w.causal, plan=plan, dQ=dQ, dK=dK, dV=dV, hO=hO, hLSE=hL,
+                                 stream=stream)
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(a.elapsed_time(b), world) / e2e_steps
+    elem = w.B * w.H * w.N * w.d
+    h2d = 3 * elem * 2
+    d2h = elem * 2 + w.B * w.H * w.N * 4 + 8
+
+    if rank != 0:
+        return
+    peaks, peak_src = load_peaks()
+    peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+    burst = float(peaks["bf16_tflops"])
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        cpu = oracle_sample(w, Qh, Kh, Vh, budget_s=args.cpu_budget)
+        cpu.pop("route_s_full", None)
+    counts = plan.route.head_counts.cpu().numpy()
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": max(3, args.warmup), "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "block": w.bs, "p": w.p,
+                   "causal": w.causal, "nnz_blocks": nnz, "density": nnz / (w.B * w.H * w.nb * w.nb),
+                   "l2": "inputs larger than L2 (each of Q, K, V is %d MB)" % (elem * 2 // 10**6),
+                   "parallelism": f"replicas x{world}"},
+        "attn_tflops": attn_tflops, "attn_ms": attn_ms, "route_ms": r_ms,
+        "route_frac": r_ms / (r_ms + attn_ms),
+        "tensor_frac_of_burst_peak": attn_tflops / burst,
+        "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peak, "unit": "TFLOP/s",
+                     "frac": attn_tflops / peak, "traffic": None,
+                     "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside back-to-back steps)",
+                     "note": "achieved = 4*block^2*d*nnz / mean CUDA-event time of the fvattn_sparse_fwd call "
+                             "(its 3 small ordering kernels included)"},
+        "route_roofline": {"bound": "hbm", "pool_bytes": 2 * elem * 2,
+                           "achieved_gbs_whole_route": 2 * elem * 2 / (r_ms * 1e-3) / 1e9,
+                           "peak": float(peaks["hbm_gbs"]), "unit": "GB/s"},
+        "head_counts": {"min": int(counts.min()), "max": int(counts.max()), "mean": float(counts.mean())},
+        "e2e": {"value": flops / (e2e_ms * 1e-3) / 1e12 * world, "unit": UNIT, "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": args.steps * (ROUTE_KERNELS_PER_CALL + FWD_KERNELS_PER_CALL),
+        "clocks": clocks,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=W.VIDEO.name, choices=sorted(W.ALL))
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    w = W.ALL[args.workload]
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        run_reference(args, w, rank, world)
+        return
+    rank, world, local = dist_setup(args.gpus)
+    try:
+        run_ours(args, w, rank, world, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

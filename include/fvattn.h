@@ -1,0 +1,185 @@
+/*
+ * fvattn.h -- C ABI of libfvattn.so: top-p routed block-sparse attention
+ * forward for NVIDIA B200 (sm_100a).
+ *
+ * What it computes (page title, section):
+ *   - FVAttn review ("[논문리뷰] FVAttn: Adaptive Sparse Attention with Runtime
+ *     Load Balancing for Video Generation"), §1 Key Terms "Top-p routing":
+ *     every query block keeps key blocks, most important first, until their
+ *     cumulative probability reaches p.  §1 "RLB" and §3: the per-head amount
+ *     of work is known once the mask is fixed and is balanced at run time.
+ *   - FlashAttention review ("FlashAttention - Fast and Memory-Efficient Exact
+ *     Attention with IO-Awareness"), §Background "Motivation" (S = QK^T,
+ *     P = softmax(S), O = PV) and §Model (one fused kernel, tiled matmul,
+ *     "Tiling Softmax"): exact attention computed tile by tile without writing
+ *     S or P to memory.
+ * The pages name the routing score without defining it; this library fixes
+ * it as: mean of each block of `block` tokens of Q and of K (over the tokens
+ * that exist), score = qbar . kbar / sqrt(d), softmax over all key blocks,
+ * and keep the shortest prefix of key blocks sorted by descending score
+ * (equal scores: lower index first) whose mass is >= p; p = 1 keeps all.
+ *
+ * Conventions shared by every call:
+ *   - Tensors Q, K, V, O are bf16, contiguous [B, H, N, d] (d fastest).
+ *     LSE is fp32 [B, H, N], natural logarithm.
+ *   - nb = ceil(N / block); a "row" is one (b, h, query block i), numbered
+ *     r = (b*H + h)*nb + i.  The CSR block mask is row_ptr int32[rows + 1]
+ *     and col_idx int32[row_ptr[rows]] with strictly ascending key-block
+ *     indices inside a row.
+ *   - The caller owns and allocates every buffer (device memory unless a
+ *     parameter says "host").  The library allocates nothing and keeps no
+ *     state between calls apart from cached device attributes; calls on
+ *     different streams with disjoint buffers may run concurrently.
+ *   - Every device call is asynchronous on `stream` (a cudaStream_t; NULL is
+ *     the legacy default stream) and never synchronises the host, except
+ *     fvattn_attention_host, which synchronises before returning.
+ *   - Errors: the return value reports argument and launch errors found on
+ *     the host (fvattn_status, negative).  Errors found on the device (a
+ *     column index out of range or not ascending, CSR capacity exceeded, a
+ *     bounded wait that timed out) are written to *dev_status (int32 in
+ *     device memory; the call sets it to 0 first).  Read it after the stream
+ *     has completed.  The first device error wins.
+ *   - Supported: d in {64, 128}; block in {64, 128}; 0 < p <= 1; 1 <= N;
+ *     nb <= 4096 (nb <= 1024 for fvattn_route); B*H*nb < 2^31.  Tensor and
+ *     workspace pointers 16-byte aligned, int32/fp32 arrays 4-byte aligned.
+ */
+#ifndef FVATTN_H
+#define FVATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define FVATTN_API __attribute__((visibility("default")))
+#else
+#define FVATTN_API
+#endif
+
+typedef struct CUstream_st *fvattn_stream_t; /* identical to cudaStream_t */
+
+typedef enum {
+    FVATTN_OK = 0,
+    FVATTN_ERR_INVALID_ARG = -1,    /* null pointer, bad size, p outside (0, 1] */
+    FVATTN_ERR_UNSUPPORTED = -2,    /* d or block not supported, no sm_100 device */
+    FVATTN_ERR_ALIGNMENT = -3,      /* a pointer is not 16-byte aligned */
+    FVATTN_ERR_CAPACITY = -4,       /* workspace or col_idx capacity too small */
+    FVATTN_ERR_CUDA = -5,           /* a CUDA runtime/driver call failed */
+    FVATTN_ERR_BAD_CSR = -6,        /* device: index out of range, not ascending, count > nb */
+    FVATTN_ERR_DEVICE_TIMEOUT = -7  /* device: a bounded wait gave up */
+} fvattn_status;
+
+/* Human-readable name of a status code (static string, never NULL). */
+FVATTN_API const char *fvattn_status_string(int status);
+
+/* Number of rows B*H*ceil(N/block) (0 on bad arguments). */
+FVATTN_API int64_t fvattn_num_rows(int B, int H, int N, int block);
+
+/* Largest possible nnz of a routing CSR: B*H*nb*nb (0 on bad arguments). */
+FVATTN_API int64_t fvattn_route_max_nnz(int B, int H, int N, int block);
+
+/* Device workspace fvattn_route needs, in bytes (0 on bad arguments). */
+FVATTN_API size_t fvattn_route_workspace_bytes(int B, int H, int N, int d, int block);
+
+/*
+ * fvattn_route -- top-p routing (FVAttn review §1 "Top-p routing"), then the
+ * CSR block mask and per-head selected-block counts.
+ *
+ *   Q, K          bf16 [B,H,N,d], read only.
+ *   p             threshold in (0, 1]; p = 1 selects every block.
+ *   row_ptr       out, int32[rows + 1].
+ *   col_idx       out, int32[col_capacity]; row_ptr[rows] entries are written,
+ *                 ascending within each row.  If the selection needs more than
+ *                 col_capacity entries, *dev_status = FVATTN_ERR_CAPACITY and
+ *                 col_idx is left incomplete (row_ptr is still complete).
+ *                 col_capacity >= fvattn_route_max_nnz() never overflows.
+ *   head_counts   out, int32[B*H]: selected blocks of each head (its work).
+ *   workspace     device scratch of ws_bytes >= fvattn_route_workspace_bytes().
+ *   dev_status    device int32, see above.
+ * Steps: mean pooling (fp64 accumulation of the bf16 inputs), fp64 scores and
+ * softmax, sort by (score desc, index asc), prefix sum to p, CSR emission.
+ */
+FVATTN_API int fvattn_route(const void *Q, const void *K, int B, int H, int N, int d, int block, double p,
+                 int32_t *row_ptr, int32_t *col_idx, int64_t col_capacity, int32_t *head_counts,
+                 void *workspace, size_t ws_bytes, int32_t *dev_status, fvattn_stream_t stream);
+
+/* Device workspace fvattn_sparse_fwd needs, in bytes (0 on bad arguments). */
+FVATTN_API size_t fvattn_fwd_workspace_bytes(int B, int H, int N, int block);
+
+/* Device workspace fvattn_lpt_order needs for `rows` rows with counts <= max_count. */
+FVATTN_API size_t fvattn_lpt_workspace_bytes(int64_t rows, int max_count);
+
+/*
+ * fvattn_lpt_order -- longest-first order of the rows of a CSR block mask:
+ * rows sorted by selected-block count descending, equal counts by ascending
+ * row id.  This is the single-GPU counterpart of FVAttn's run-time balancing
+ * of per-head work (§1 "RLB", §3): the attention kernel hands rows to SMs in
+ * this order.
+ *
+ *   row_ptr     int32[rows + 1], read only; counts must lie in [0, max_count].
+ *   max_count   largest allowed count (nb for a routing mask), <= 4096.
+ *   order       out, int32[rows].
+ *   workspace   >= fvattn_lpt_workspace_bytes(rows, max_count) bytes.
+ * A count outside [0, max_count] sets *dev_status = FVATTN_ERR_BAD_CSR and is
+ * clamped.
+ */
+FVATTN_API int fvattn_lpt_order(const int32_t *row_ptr, int64_t rows, int max_count, int32_t *order, void *workspace,
+                     size_t ws_bytes, int32_t *dev_status, fvattn_stream_t stream);
+
+/*
+ * fvattn_sparse_fwd -- exact attention restricted to the CSR block mask
+ * (FlashAttention review §Model: one fused kernel, tiled matmuls, tiled
+ * online softmax; FVAttn review §1: only the selected key blocks are read).
+ *
+ * For every query token t of row r = (b,h,i):
+ *   keys(t) = { u : u in block j for some j in col_idx[row_ptr[r]..row_ptr[r+1]),
+ *               u < N, and u <= t if causal }
+ *   O[t]   = sum_{u in keys(t)} softmax_u(q_t.k_u/sqrt(d)) v_u      (bf16 out)
+ *   LSE[t] = ln sum_{u in keys(t)} exp(q_t.k_u/sqrt(d))            (fp32 out)
+ * An empty keys(t) gives O[t] = 0 and LSE[t] = -inf.
+ *
+ *   Q, K, V     bf16 [B,H,N,d], read only.
+ *   row_ptr, col_idx  CSR as above (e.g. from fvattn_route), read only.
+ *   causal      0 or 1.
+ *   O           out, bf16 [B,H,N,d].   LSE  out, fp32 [B,H,N].
+ *   workspace   >= fvattn_fwd_workspace_bytes(B,H,N,block).
+ * Matmuls run on the tensor cores in bf16 with fp32 accumulation; softmax in
+ * fp32.  Rows are processed longest-first (fvattn_lpt_order) by a persistent
+ * grid.  Out-of-range or non-ascending column indices are skipped and set
+ * *dev_status = FVATTN_ERR_BAD_CSR.
+ */
+FVATTN_API int fvattn_sparse_fwd(const void *Q, const void *K, const void *V, const int32_t *row_ptr,
+                      const int32_t *col_idx, int B, int H, int N, int d, int block, int causal, void *O,
+                      float *LSE, void *workspace, size_t ws_bytes, int32_t *dev_status,
+                      fvattn_stream_t stream);
+
+/*
+ * fvattn_attention_host -- the whole path from host memory: copies Q, K, V
+ * (host, ideally pinned) to the device buffers dQ, dK, dV, routes with p,
+ * runs the sparse forward, and copies O (bf16) and LSE (fp32) back to the
+ * host buffers hO, hLSE; synchronises `stream` before returning.
+ *   hQ, hK, hV    host bf16 [B,H,N,d];  hO host bf16 [B,H,N,d];  hLSE host fp32 [B,H,N].
+ *   dQ, dK, dV, dO, dLSE, row_ptr, col_idx (capacity col_capacity), head_counts,
+ *   route_ws (route_ws_bytes), fwd_ws (fwd_ws_bytes): device buffers as for
+ *   fvattn_route / fvattn_sparse_fwd.  dev_status: device int32[2] (routing
+ *   status, then attention status).
+ * Returns the first host error, else the first nonzero device status read
+ * after the sync.
+ */
+FVATTN_API int fvattn_attention_host(const void *hQ, const void *hK, const void *hV, int B, int H, int N, int d, int block,
+                          double p, int causal, void *hO, float *hLSE, void *dQ, void *dK, void *dV, void *dO,
+                          float *dLSE, int32_t *row_ptr, int32_t *col_idx, int64_t col_capacity,
+                          int32_t *head_counts, void *route_ws, size_t route_ws_bytes, void *fwd_ws,
+                          size_t fwd_ws_bytes, int32_t *dev_status, fvattn_stream_t stream);
+
+/* Compiled-in build description (architecture, version), static string. */
+FVATTN_API const char *fvattn_build_info(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FVATTN_H */

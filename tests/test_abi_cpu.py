@@ -1,0 +1,109 @@
+"""Host-side checks of the C ABI (no GPU): the library loads, exports every
+function include/fvattn.h declares, and its size helpers and argument checks
+behave as documented."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from top_routed_block_b200 import _build
+    _build.build()
+    import top_routed_block_b200 as fv
+    return fv.load_library()
+
+
+def declared_functions():
+    with open(os.path.join(ROOT, "include", "fvattn.h")) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fvattn_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("fvattn_route", "fvattn_sparse_fwd", "fvattn_lpt_order", "fvattn_route_workspace_bytes",
+                     "fvattn_fwd_workspace_bytes", "fvattn_route_max_nnz", "fvattn_status_string"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+        assert isinstance(getattr(lib, name), ctypes._CFuncPtr)
+
+
+def test_only_declared_symbols_are_exported(lib):
+    import subprocess
+    from top_routed_block_b200 import LIB_PATH
+    out = subprocess.run(["nm", "-D", "--defined-only", LIB_PATH], capture_output=True, text=True).stdout
+    exported = {l.split()[-1] for l in out.splitlines() if " T " in l and l.split()[-1].startswith("fvattn_")}
+    assert exported == set(declared_functions())
+
+
+def test_status_strings(lib):
+    import top_routed_block_b200 as fv
+    assert fv.status_string(0) == "ok"
+    for code in range(-7, 0):
+        assert fv.status_string(code) not in ("", "unknown status")
+    assert fv.status_string(-99) == "unknown status"
+    assert b"sm_100a" in lib.fvattn_build_info()
+
+
+def test_size_helpers(lib):
+    import top_routed_block_b200 as fv
+    assert fv.fvattn_num_rows(1, 40, 32760, 128) == 40 * 256
+    assert fv.fvattn_route_max_nnz(1, 24, 118800, 128) == 24 * 929 * 929
+    assert fv.fvattn_route_max_nnz(0, 1, 1, 64) == 0
+    rw = fv.fvattn_route_workspace_bytes(1, 40, 32760, 128, 128)
+    # two fp64 block-mean tensors dominate: 2 * 40 * 256 * 128 * 8 bytes
+    assert rw >= 2 * 40 * 256 * 128 * 8
+    assert fv.fvattn_route_workspace_bytes(1, 1, 100, 96, 128) == 0      # d unsupported
+    assert fv.fvattn_route_workspace_bytes(1, 1, 100, 64, 32) == 0       # block unsupported
+    fw = fv.fvattn_fwd_workspace_bytes(1, 40, 32760, 128)
+    assert fw >= 40 * 256 * 4
+    assert fv.fvattn_lpt_workspace_bytes(10, 5000) == 0                  # count limit 4096
+
+
+def test_invalid_arguments_rejected_before_any_device_work(lib):
+    P = ctypes.c_void_p
+    fake = P(16)  # never dereferenced: argument checks fail first
+    # p outside (0, 1]
+    for p in (0.0, -0.5, 1.5, float("nan")):
+        rc = lib.fvattn_route(fake, fake, 1, 1, 128, 64, 64, p, fake, fake, 4, fake, fake, 1 << 20, fake, None)
+        assert rc == -1
+    # unsupported head dim / block
+    assert lib.fvattn_route(fake, fake, 1, 1, 128, 96, 64, 0.5, fake, fake, 4, fake, fake, 1 << 20, fake, None) == -2
+    assert lib.fvattn_sparse_fwd(fake, fake, fake, fake, fake, 1, 1, 128, 64, 32, 0, fake, fake, fake, 1 << 20,
+                                 fake, None) == -2
+    # null pointers
+    assert lib.fvattn_sparse_fwd(None, fake, fake, fake, fake, 1, 1, 128, 64, 64, 0, fake, fake, fake, 1 << 20,
+                                 fake, None) == -1
+    # misaligned tensor pointer
+    assert lib.fvattn_sparse_fwd(P(18), fake, fake, fake, fake, 1, 1, 128, 64, 64, 0, fake, fake, fake, 1 << 20,
+                                 fake, None) == -3
+    # workspace too small
+    assert lib.fvattn_sparse_fwd(fake, fake, fake, fake, fake, 1, 1, 128, 64, 64, 0, fake, fake, fake, 8,
+                                 fake, None) == -4
+    # causal must be 0 or 1
+    assert lib.fvattn_sparse_fwd(fake, fake, fake, fake, fake, 1, 1, 128, 64, 64, 2, fake, fake, fake, 1 << 20,
+                                 fake, None) == -1
+    # routing supports at most 1024 blocks per sequence
+    assert lib.fvattn_route(fake, fake, 1, 1, 1025 * 64, 64, 64, 0.5, fake, fake, 4, fake, fake, 1 << 30, fake,
+                            None) == -2
+
+
+def test_binding_fails_loudly_without_library(tmp_path):
+    import top_routed_block_b200 as fv
+    saved = fv._lib
+    try:
+        fv._lib = None
+        with pytest.raises(fv.FvattnError):
+            fv.load_library(str(tmp_path / "missing.so"))
+    finally:
+        fv._lib = saved

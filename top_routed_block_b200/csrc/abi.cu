@@ -1,0 +1,289 @@
+// abi.cu -- the extern "C" surface of libfvattn.so (declared in include/fvattn.h):
+// argument checks, workspace carving, TMA descriptor encoding and launches.
+// All compute runs in the kernels of route.cu, lpt.cu and attn_fwd.cu.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/fvattn.h"
+#include "attn_fwd.cuh"
+#include "common.cuh"
+#include "lpt.cuh"
+#include "route.cuh"
+
+using namespace fvattn;
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+struct DeviceInfo {
+    int sms = 0;
+    int major = 0;
+    bool ok = false;
+};
+
+// Cached per device: multiprocessor count and compute capability.
+bool device_info(DeviceInfo *out) {
+    static std::mutex mu;
+    static DeviceInfo cache[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+    std::lock_guard<std::mutex> g(mu);
+    if (!cache[dev].ok) {
+        DeviceInfo d;
+        if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return false;
+        if (cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return false;
+        d.ok = true;
+        cache[dev] = d;
+    }
+    *out = cache[dev];
+    return true;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_shape(int B, int H, int N, int d, int block) {
+    if (B < 1 || H < 1 || N < 1) return FVATTN_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return FVATTN_ERR_UNSUPPORTED;
+    if (block != 64 && block != 128) return FVATTN_ERR_UNSUPPORTED;
+    const int64_t nb = ceil_div(N, block);
+    if (nb > kMaxCount) return FVATTN_ERR_UNSUPPORTED;
+    const int64_t rows = static_cast<int64_t>(B) * H * nb;
+    if (rows >= (1LL << 31)) return FVATTN_ERR_UNSUPPORTED;
+    return FVATTN_OK;
+}
+
+int check_device() {
+    DeviceInfo info;
+    if (!device_info(&info)) return FVATTN_ERR_CUDA;
+    if (info.major != 10) return FVATTN_ERR_UNSUPPORTED;
+    return FVATTN_OK;
+}
+
+// 3-D map over a contiguous bf16 [B*H, N, d] tensor; box = 64 columns (128 bytes,
+// the swizzle width) x `rows` tokens x 1 head; out-of-range rows read as zero.
+bool make_map(CUtensorMap *m, const void *base, int64_t BH, int N, int d, int rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(N) * d * 2};
+    cuuint32_t box[3] = {64, static_cast<cuuint32_t>(rows), 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct FwdWorkspace {
+    size_t order, counter, lpt, total;
+};
+
+FwdWorkspace fwd_layout(int64_t rows, int max_count) {
+    FwdWorkspace w{};
+    Carver c;
+    w.order = c.take<int32_t>(static_cast<size_t>(rows));
+    w.counter = c.take<int32_t>(64);
+    w.lpt = align_up(c.off, 256);
+    w.total = w.lpt + lpt_workspace_layout(rows, max_count).total;
+    return w;
+}
+
+int from_cuda(cudaError_t e) { return e == cudaSuccess ? FVATTN_OK : FVATTN_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+const char *fvattn_status_string(int status) {
+    switch (status) {
+        case FVATTN_OK: return "ok";
+        case FVATTN_ERR_INVALID_ARG: return "invalid argument";
+        case FVATTN_ERR_UNSUPPORTED: return "unsupported configuration or device";
+        case FVATTN_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+        case FVATTN_ERR_CAPACITY: return "workspace or output capacity too small";
+        case FVATTN_ERR_CUDA: return "CUDA error";
+        case FVATTN_ERR_BAD_CSR: return "malformed CSR block mask";
+        case FVATTN_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+        default: return "unknown status";
+    }
+}
+
+const char *fvattn_build_info(void) { return "libfvattn 0.1 sm_100a (tcgen05/TMA/TMEM)"; }
+
+int64_t fvattn_num_rows(int B, int H, int N, int block) {
+    if (B < 1 || H < 1 || N < 1 || block < 1) return 0;
+    return static_cast<int64_t>(B) * H * ceil_div(N, block);
+}
+
+int64_t fvattn_route_max_nnz(int B, int H, int N, int block) {
+    if (B < 1 || H < 1 || N < 1 || block < 1) return 0;
+    const int64_t nb = ceil_div(N, block);
+    return static_cast<int64_t>(B) * H * nb * nb;
+}
+
+size_t fvattn_route_workspace_bytes(int B, int H, int N, int d, int block) {
+    if (check_shape(B, H, N, d, block) != FVATTN_OK) return 0;
+    const int nb = static_cast<int>(ceil_div(N, block));
+    return route_workspace_layout(static_cast<int64_t>(B) * H, nb, d).total;
+}
+
+size_t fvattn_lpt_workspace_bytes(int64_t rows, int max_count) {
+    if (rows < 0 || max_count < 0 || max_count > kMaxCount) return 0;
+    return lpt_workspace_layout(rows, max_count).total;
+}
+
+size_t fvattn_fwd_workspace_bytes(int B, int H, int N, int block) {
+    if (B < 1 || H < 1 || N < 1 || (block != 64 && block != 128)) return 0;
+    const int64_t nb = ceil_div(N, block);
+    if (nb > kMaxCount) return 0;
+    return fwd_layout(static_cast<int64_t>(B) * H * nb, static_cast<int>(nb)).total;
+}
+
+int fvattn_route(const void *Q, const void *K, int B, int H, int N, int d, int block, double p, int32_t *row_ptr,
+                 int32_t *col_idx, int64_t col_capacity, int32_t *head_counts, void *workspace, size_t ws_bytes,
+                 int32_t *dev_status, fvattn_stream_t stream) {
+    int rc = check_shape(B, H, N, d, block);
+    if (rc != FVATTN_OK) return rc;
+    if (!Q || !K || !row_ptr || !col_idx || !head_counts || !workspace || !dev_status) return FVATTN_ERR_INVALID_ARG;
+    if (!(p > 0.0) || p > 1.0 || std::isnan(p)) return FVATTN_ERR_INVALID_ARG;
+    if (col_capacity < 0) return FVATTN_ERR_INVALID_ARG;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(workspace)) return FVATTN_ERR_ALIGNMENT;
+    if ((reinterpret_cast<uintptr_t>(row_ptr) | reinterpret_cast<uintptr_t>(col_idx) |
+         reinterpret_cast<uintptr_t>(head_counts) | reinterpret_cast<uintptr_t>(dev_status)) & 3u)
+        return FVATTN_ERR_ALIGNMENT;
+    const int nb = static_cast<int>(ceil_div(N, block));
+    if (nb > kMaxRouteBlocks) return FVATTN_ERR_UNSUPPORTED;
+    if (ws_bytes < fvattn_route_workspace_bytes(B, H, N, d, block)) return FVATTN_ERR_CAPACITY;
+    if ((rc = check_device()) != FVATTN_OK) return rc;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if ((rc = from_cuda(cudaMemsetAsync(dev_status, 0, sizeof(int32_t), s))) != FVATTN_OK) return rc;
+    return from_cuda(launch_route(Q, K, static_cast<int64_t>(B) * H, N, d, block, nb, p, row_ptr, col_idx,
+                                  col_capacity, head_counts, workspace, dev_status, s));
+}
+
+int fvattn_lpt_order(const int32_t *row_ptr, int64_t rows, int max_count, int32_t *order, void *workspace,
+                     size_t ws_bytes, int32_t *dev_status, fvattn_stream_t stream) {
+    if (!row_ptr || !order || !workspace || !dev_status || rows < 0 || rows >= (1LL << 31))
+        return FVATTN_ERR_INVALID_ARG;
+    if (max_count < 0 || max_count > kMaxCount) return FVATTN_ERR_UNSUPPORTED;
+    if (!aligned16(workspace)) return FVATTN_ERR_ALIGNMENT;
+    if (ws_bytes < fvattn_lpt_workspace_bytes(rows, max_count)) return FVATTN_ERR_CAPACITY;
+    int rc = check_device();
+    if (rc != FVATTN_OK) return rc;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if ((rc = from_cuda(cudaMemsetAsync(dev_status, 0, sizeof(int32_t), s))) != FVATTN_OK) return rc;
+    return from_cuda(launch_lpt_order(row_ptr, rows, max_count, order, workspace, dev_status, s));
+}
+
+int fvattn_sparse_fwd(const void *Q, const void *K, const void *V, const int32_t *row_ptr, const int32_t *col_idx,
+                      int B, int H, int N, int d, int block, int causal, void *O, float *LSE, void *workspace,
+                      size_t ws_bytes, int32_t *dev_status, fvattn_stream_t stream) {
+    int rc = check_shape(B, H, N, d, block);
+    if (rc != FVATTN_OK) return rc;
+    if (!Q || !K || !V || !row_ptr || !col_idx || !O || !LSE || !workspace || !dev_status)
+        return FVATTN_ERR_INVALID_ARG;
+    if (causal != 0 && causal != 1) return FVATTN_ERR_INVALID_ARG;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(workspace))
+        return FVATTN_ERR_ALIGNMENT;
+    if ((reinterpret_cast<uintptr_t>(row_ptr) | reinterpret_cast<uintptr_t>(col_idx) |
+         reinterpret_cast<uintptr_t>(LSE) | reinterpret_cast<uintptr_t>(dev_status)) & 3u)
+        return FVATTN_ERR_ALIGNMENT;
+    if (ws_bytes < fvattn_fwd_workspace_bytes(B, H, N, block)) return FVATTN_ERR_CAPACITY;
+    if ((rc = check_device()) != FVATTN_OK) return rc;
+    DeviceInfo info;
+    if (!device_info(&info)) return FVATTN_ERR_CUDA;
+    const int64_t BH = static_cast<int64_t>(B) * H;
+    const int nb = static_cast<int>(ceil_div(N, block));
+    const int64_t rows = BH * nb;
+    const FwdWorkspace w = fwd_layout(rows, nb);
+    char *ws = static_cast<char *>(workspace);
+    int32_t *order = reinterpret_cast<int32_t *>(ws + w.order);
+    int *counter = reinterpret_cast<int *>(ws + w.counter);
+
+    CUtensorMap mq, mk, mv;
+    if (!make_map(&mq, Q, BH, N, d, block) || !make_map(&mk, K, BH, N, d, block) ||
+        !make_map(&mv, V, BH, N, d, block))
+        return FVATTN_ERR_CUDA;
+
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if ((rc = from_cuda(cudaMemsetAsync(dev_status, 0, sizeof(int32_t), s))) != FVATTN_OK) return rc;
+    if ((rc = from_cuda(launch_lpt_order(row_ptr, rows, nb, order, ws + w.lpt, dev_status, s))) != FVATTN_OK)
+        return rc;
+    if ((rc = from_cuda(cudaMemsetAsync(counter, 0, sizeof(int), s))) != FVATTN_OK) return rc;
+
+    AttnLaunch a{};
+    a.tmap_q = &mq;
+    a.tmap_k = &mk;
+    a.tmap_v = &mv;
+    a.row_ptr = row_ptr;
+    a.col_idx = col_idx;
+    a.order = order;
+    a.n_items = static_cast<int>(rows);
+    a.work_counter = counter;
+    a.N = N;
+    a.nb = nb;
+    a.causal = causal;
+    a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(d)));
+    a.O = O;
+    a.LSE = LSE;
+    a.dev_status = dev_status;
+    const int64_t max_grid = 2LL * info.sms;
+    a.grid = static_cast<int>(rows < max_grid ? rows : max_grid);
+    return from_cuda(launch_sparse_attn(a, d, block, s));
+}
+
+int fvattn_attention_host(const void *hQ, const void *hK, const void *hV, int B, int H, int N, int d, int block,
+                          double p, int causal, void *hO, float *hLSE, void *dQ, void *dK, void *dV, void *dO,
+                          float *dLSE, int32_t *row_ptr, int32_t *col_idx, int64_t col_capacity,
+                          int32_t *head_counts, void *route_ws, size_t route_ws_bytes, void *fwd_ws,
+                          size_t fwd_ws_bytes, int32_t *dev_status, fvattn_stream_t stream) {
+    int rc = check_shape(B, H, N, d, block);
+    if (rc != FVATTN_OK) return rc;
+    if (!hQ || !hK || !hV || !hO || !hLSE) return FVATTN_ERR_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const size_t bytes = static_cast<size_t>(B) * H * N * d * 2;
+    const size_t lse_bytes = static_cast<size_t>(B) * H * N * sizeof(float);
+    if (!dQ || !dK || !dV || !dO || !dLSE) return FVATTN_ERR_INVALID_ARG;
+    if ((rc = from_cuda(cudaMemcpyAsync(dQ, hQ, bytes, cudaMemcpyHostToDevice, s))) != FVATTN_OK) return rc;
+    if ((rc = from_cuda(cudaMemcpyAsync(dK, hK, bytes, cudaMemcpyHostToDevice, s))) != FVATTN_OK) return rc;
+    if ((rc = from_cuda(cudaMemcpyAsync(dV, hV, bytes, cudaMemcpyHostToDevice, s))) != FVATTN_OK) return rc;
+    rc = fvattn_route(dQ, dK, B, H, N, d, block, p, row_ptr, col_idx, col_capacity, head_counts, route_ws,
+                      route_ws_bytes, dev_status, stream);
+    if (rc != FVATTN_OK) return rc;
+    // the routing status is kept: fvattn_sparse_fwd must not clear a routing error
+    int32_t *fwd_status = dev_status + 1;
+    if ((reinterpret_cast<uintptr_t>(fwd_status) & 3u) != 0) return FVATTN_ERR_ALIGNMENT;
+    rc = fvattn_sparse_fwd(dQ, dK, dV, row_ptr, col_idx, B, H, N, d, block, causal, dO, dLSE, fwd_ws, fwd_ws_bytes,
+                           fwd_status, stream);
+    if (rc != FVATTN_OK) return rc;
+    if ((rc = from_cuda(cudaMemcpyAsync(hO, dO, bytes, cudaMemcpyDeviceToHost, s))) != FVATTN_OK) return rc;
+    if ((rc = from_cuda(cudaMemcpyAsync(hLSE, dLSE, lse_bytes, cudaMemcpyDeviceToHost, s))) != FVATTN_OK) return rc;
+    int32_t st[2] = {0, 0};
+    if ((rc = from_cuda(cudaMemcpyAsync(st, dev_status, sizeof(st), cudaMemcpyDeviceToHost, s))) != FVATTN_OK)
+        return rc;
+    if ((rc = from_cuda(cudaStreamSynchronize(s))) != FVATTN_OK) return rc;
+    return st[0] != 0 ? st[0] : st[1];
+}
+
+}  // extern "C"

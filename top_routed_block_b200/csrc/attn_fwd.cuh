@@ -1,0 +1,26 @@
+// attn_fwd.cuh -- internal interface of the sparse attention kernel (attn_fwd.cu).
+#pragma once
+
+#include <cuda.h>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace fvattn {
+
+struct AttnLaunch {
+    const CUtensorMap *tmap_q, *tmap_k, *tmap_v;  // host copies, passed by value as kernel parameters
+    const int32_t *row_ptr, *col_idx, *order;
+    int n_items;
+    int *work_counter;  // zeroed before the launch
+    int N, nb, causal;
+    float scale_log2;   // log2(e) / sqrt(d)
+    void *O;
+    float *LSE;
+    int32_t *dev_status;
+    int grid;
+};
+
+int attn_smem_bytes(int d, int bs);
+cudaError_t launch_sparse_attn(const AttnLaunch &a, int d, int bs, cudaStream_t stream);
+
+}  // namespace fvattn
