@@ -175,6 +175,38 @@ FVATTN_API int fvattn_attention_host(const void *hQ, const void *hK, const void 
                           int32_t *head_counts, void *route_ws, size_t route_ws_bytes, void *fwd_ws,
                           size_t fwd_ws_bytes, int32_t *dev_status, fvattn_stream_t stream);
 
+/* Size of the library-owned device scratch used by fvattn_sparse_fwd_noalloc. */
+#define FVATTN_NOALLOC_SCRATCH_BYTES (4u << 20)
+
+/*
+ * fvattn_sparse_fwd_noalloc -- fvattn_sparse_fwd without a caller workspace.
+ * The pages have no counterpart to this call; it exists for callers that cannot
+ * allocate device memory when they call the library: a host that hands the
+ * library a stream and its tensors but owns every allocation itself (plugin-style
+ * enqueue functions, fixed memory pools), or code that must not pay for the device
+ * synchronisation that cudaMalloc/cudaFree imply in the middle of a step.
+ *
+ * Arguments and results are those of fvattn_sparse_fwd minus workspace/ws_bytes;
+ * the caller still provides Q, K, V, the CSR, O, LSE and dev_status.  The scratch
+ * the call needs (fvattn_fwd_workspace_bytes(B,H,N,block) bytes) comes from one
+ * file-scope device array of FVATTN_NOALLOC_SCRATCH_BYTES (4 MiB) inside the
+ * library, which every device that loads the library keeps until the process
+ * exits.  Shapes that need more return FVATTN_ERR_CAPACITY without launching
+ * anything (about 400k rows B*H*ceil(N/block) at most).
+ *
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current) and caches it; make that first
+ * call before any stream capture.  The call allocates nothing: no cudaMalloc,
+ * cudaFree or allocating library routine.  All calls on a device share the one
+ * array, which keeps the previous call's contents (the parts that must start at
+ * zero are cleared on the stream by each call), so calls whose executions overlap
+ * on the GPU -- on different streams, or from different host threads -- race on it
+ * and must be serialised by the caller.
+ */
+FVATTN_API int fvattn_sparse_fwd_noalloc(const void *Q, const void *K, const void *V, const int32_t *row_ptr,
+                                         const int32_t *col_idx, int B, int H, int N, int d, int block, int causal,
+                                         void *O, float *LSE, int32_t *dev_status, fvattn_stream_t stream);
+
 /* Compiled-in build description (architecture, version), static string. */
 FVATTN_API const char *fvattn_build_info(void);
 

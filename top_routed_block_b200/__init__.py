@@ -66,6 +66,7 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         "fvattn_route": (I, [P, P, I, I, I, I, I, D, P, P, I64, P, P, SZ, P, P]),
         "fvattn_lpt_order": (I, [P, I64, I, P, P, SZ, P, P]),
         "fvattn_sparse_fwd": (I, [P, P, P, P, P, I, I, I, I, I, I, P, P, P, SZ, P, P]),
+        "fvattn_sparse_fwd_noalloc": (I, [P, P, P, P, P, I, I, I, I, I, I, P, P, P, P]),
         "fvattn_attention_host": (I, [P, P, P, I, I, I, I, I, D, I, P, P, P, P, P, P, P, P, P, I64, P, P, SZ, P, SZ,
                                       P, P]),
     }
@@ -205,6 +206,19 @@ def fvattn_sparse_fwd(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, row_ptr
                                1 if causal else 0, _ptr(O), _ptr(LSE), _ptr(workspace), workspace.numel(),
                                _ptr(dev_status), _stream_ptr(stream))
     _check(rc, "fvattn_sparse_fwd")
+    return O, LSE, dev_status
+
+
+def fvattn_sparse_fwd_noalloc(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, row_ptr: torch.Tensor,
+                              col_idx: torch.Tensor, block: int, causal: bool, *, O: torch.Tensor, LSE: torch.Tensor,
+                              dev_status: torch.Tensor, stream=None):
+    """fvattn_sparse_fwd with the library's own fixed device scratch instead of a
+    caller workspace; O, LSE and dev_status must be given (nothing is allocated)."""
+    lib = load_library()
+    B, H, N, d = _shape(Q)
+    rc = lib.fvattn_sparse_fwd_noalloc(_ptr(Q), _ptr(K), _ptr(V), _ptr(row_ptr), _ptr(col_idx), B, H, N, d, block,
+                                       1 if causal else 0, _ptr(O), _ptr(LSE), _ptr(dev_status), _stream_ptr(stream))
+    _check(rc, "fvattn_sparse_fwd_noalloc")
     return O, LSE, dev_status
 
 

@@ -287,3 +287,50 @@ int fvattn_attention_host(const void *hQ, const void *hK, const void *hV, int B,
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------------------------------
+// fvattn_sparse_fwd_noalloc: the sparse forward for callers that cannot allocate device memory
+// when they call it.  Its scratch (the longest-first order, the ordering kernels' counters and
+// the work-queue counter) lives in one statically sized device array that the library owns;
+// every device that loads the library keeps FVATTN_NOALLOC_SCRATCH_BYTES of it until exit.
+
+namespace {
+
+__device__ __align__(256) unsigned char g_fwd_scratch[FVATTN_NOALLOC_SCRATCH_BYTES];
+
+// Device address of g_fwd_scratch on the current device.  In host code the symbol
+// g_fwd_scratch is only a host-side stand-in, so the address is looked up with
+// cudaGetSymbolAddress once per device (with that device current) and cached.
+int static_scratch(void **out) {
+    static std::mutex mu;
+    static void *addr[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FVATTN_ERR_CUDA;
+    std::lock_guard<std::mutex> g(mu);
+    if (addr[dev] == nullptr) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_fwd_scratch) != cudaSuccess || p == nullptr) return FVATTN_ERR_CUDA;
+        addr[dev] = p;
+    }
+    *out = addr[dev];
+    return FVATTN_OK;
+}
+
+}  // namespace
+
+extern "C" int fvattn_sparse_fwd_noalloc(const void *Q, const void *K, const void *V, const int32_t *row_ptr,
+                                         const int32_t *col_idx, int B, int H, int N, int d, int block, int causal,
+                                         void *O, float *LSE, int32_t *dev_status, fvattn_stream_t stream) {
+    int rc = check_shape(B, H, N, d, block);
+    if (rc != FVATTN_OK) return rc;
+    const size_t need = fvattn_fwd_workspace_bytes(B, H, N, block);
+    if (need == 0) return FVATTN_ERR_INVALID_ARG;
+    if (need > FVATTN_NOALLOC_SCRATCH_BYTES) return FVATTN_ERR_CAPACITY;
+    void *scratch = nullptr;
+    if ((rc = static_scratch(&scratch)) != FVATTN_OK) return rc;
+    // Same launches as fvattn_sparse_fwd; the work-queue counter in the scratch is
+    // cleared there on the stream before the attention kernel starts, and every other
+    // scratch word is written before it is read, so stale contents never matter.
+    return fvattn_sparse_fwd(Q, K, V, row_ptr, col_idx, B, H, N, d, block, causal, O, LSE, scratch,
+                             FVATTN_NOALLOC_SCRATCH_BYTES, dev_status, stream);
+}
