@@ -9,7 +9,7 @@
 #include <cstring>
 #include <mutex>
 
-#include "../../include/fvattn.h"
+#include "fvattn.h"
 #include "attn_fwd.cuh"
 #include "common.cuh"
 #include "lpt.cuh"

@@ -46,6 +46,9 @@ constexpr int kMmaWarp = 5;
 constexpr uint32_t kTmemCols = 256;   // per CTA; two CTAs share an SM's 512 columns
 constexpr uint32_t kTmemS = 0;        // S (fp32, block columns) / P (bf16 pairs, block/2 columns)
 constexpr uint32_t kTmemO = 128;      // O (fp32, d columns)
+// S_{j+1} is written into the TMEM columns that hold P_j: the MMA warp waits for
+// PV_j to complete before issuing S_{j+1}.
+constexpr bool kWaitPvBeforeS = true;
 
 template <int D, int BS>
 struct Cfg {
@@ -70,6 +73,44 @@ struct Barriers {
     uint32_t tmem_base;
     int abort_flag;
 };
+
+constexpr float kRescaleLog2 = 8.0f;  // rescale O only when the row max grows by more than 2^8
+
+// 2^x on the MUFU unit (flushes subnormal results to zero; exp2(-inf) = 0).
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// 2^x on the FMA pipe, for finite x: x = n + f with n = round(x) and f in [-1/2, 1/2];
+// 2^f by a cubic fitted here for least maximum relative error on [-1/2, 1/2]
+// (iteratively reweighted least squares on Chebyshev nodes; max relative error
+// 7.5e-5, far below the 2^-9 rounding of the bf16 P it feeds); 2^n is added to
+// the exponent field.  x is clamped at -126, so results below 2^-126 are not
+// exact (they are then under 1.2e-38).  Adding 1.5*2^23 rounds x to an integer
+// held in the low mantissa bits of t, whose bit pattern shifted left by 23 is
+// n in the exponent field.
+constexpr float kExp2C0 = 0.99992806f, kExp2C1 = 0.69326097f, kExp2C2 = 0.24261114f, kExp2C3 = 0.05517167f;
+
+__device__ __forceinline__ float ex2_poly(float x) {
+    x = fmaxf(x, -126.0f);
+    const float t = __fadd_rn(x, 12582912.0f);
+    const float f = __fsub_rn(x, __fsub_rn(t, 12582912.0f));
+    const float p = fmaf(fmaf(fmaf(kExp2C3, f, kExp2C2), f, kExp2C1), f, kExp2C0);
+    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+// Of every 8 exponentials of a full (unmasked) block, this many run as ex2_poly on
+// the FMA pipe instead of the MUFU unit, whose throughput otherwise equals the MMA
+// time per tile.
+constexpr int kPolyOf8 = 0;
+
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -214,7 +255,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                 for (int j = 0; j < count; ++j) {
                     // S = Q K_j^T
                     if (!mbar_wait(&bar->k_full, kc & 1, abort_flag, dev_status)) { ok = false; break; }
-                    if (pv_issued > pv_seen) {
+                    if (kWaitPvBeforeS && pv_issued > pv_seen) {
                         if (!mbar_wait(&bar->pv_done, pv_seen & 1, abort_flag, dev_status)) { ok = false; break; }
                         pv_seen = pv_issued;
                     }
@@ -293,51 +334,67 @@ __global__ void __launch_bounds__(kThreads, 2)
                 if (!mbar_wait(&bar->s_full, sc & 1, abort_flag, dev_status)) { ok = false; break; }
                 ++sc;
                 tc_fence_after();
-                // pass 1: row maximum
-                float mx = -CUDART_INF_F;
+                // the whole S row of this thread: BS fp32 values
+                uint32_t v[BS];
 #pragma unroll
-                for (int c0 = 0; c0 < BS; c0 += 32) {
-                    uint32_t v[32];
-                    tmem_ld32(tS + c0, v);
-                    tmem_wait_ld();
+                for (int c0 = 0; c0 < BS; c0 += 32) tmem_ld32(tS + c0, *reinterpret_cast<uint32_t(*)[32]>(&v[c0]));
+                tmem_wait_ld();
+                if (lim < BS) {  // ragged last block, causal diagonal, or a skipped index
 #pragma unroll
-                    for (int c = 0; c < 32; ++c)
-                        if (c0 + c < lim) mx = fmaxf(mx, __uint_as_float(v[c]));
+                    for (int c = 0; c < BS; ++c)
+                        if (c >= lim) v[c] = __float_as_uint(-CUDART_INF_F);
                 }
-                const float m_new = fmaxf(m, mx * scale_log2);
-                const float m_use = (m_new == -CUDART_INF_F) ? 0.0f : m_new;
-                const float alpha = exp2f(m - m_use);
-                // pass 2: P = exp2(S*scale_log2 - m), row sum, P -> TMEM as bf16 pairs
-                float rs = 0.0f;
+                float mq[4] = {-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F};
 #pragma unroll
-                for (int c0 = 0; c0 < BS; c0 += 32) {
-                    uint32_t v[32];
-                    tmem_ld32(tS + c0, v);
-                    tmem_wait_ld();
-                    uint32_t pk[16];
+                for (int c = 0; c < BS; c += 8) {
 #pragma unroll
-                    for (int c = 0; c < 32; c += 2) {
-                        const float p0 = (c0 + c < lim) ? exp2f(fmaf(__uint_as_float(v[c]), scale_log2, -m_use)) : 0.0f;
-                        const float p1 =
-                            (c0 + c + 1 < lim) ? exp2f(fmaf(__uint_as_float(v[c + 1]), scale_log2, -m_use)) : 0.0f;
-                        rs += p0 + p1;
-                        pk[c >> 1] = pack_bf16(p0, p1);
+                    for (int q = 0; q < 4; ++q)
+                        mq[q] = max3f(mq[q], __uint_as_float(v[c + 2 * q]), __uint_as_float(v[c + 2 * q + 1]));
+                }
+                const float mxs = max3f(mq[0], mq[1], fmaxf(mq[2], mq[3])) * scale_log2;
+                // The reference maximum only moves when the row maximum exceeds it by
+                // more than 2^8: P stays below 256 and the rescale of O is rare.  O and
+                // l always share the same reference, so the final O / l is exact.
+                const bool need = mxs > m + kRescaleLog2;
+                const float m_new = need ? mxs : m;
+                const float alpha = need ? ex2_approx(m - m_new) : 1.0f;
+                const float neg_m = (m_new == -CUDART_INF_F) ? 0.0f : -m_new;
+                float rs[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+                // P packed as bf16 pairs in place: v[c/2] <- (p[c], p[c+1])
+                if (lim >= BS) {
+#pragma unroll
+                    for (int c = 0; c < BS; c += 2) {
+                        const float x0 = fmaf(__uint_as_float(v[c]), scale_log2, neg_m);
+                        const float x1 = fmaf(__uint_as_float(v[c + 1]), scale_log2, neg_m);
+                        const float p0 = ((c & 7) >= 8 - kPolyOf8) ? ex2_poly(x0) : ex2_approx(x0);
+                        const float p1 = ((c & 7) + 1 >= 8 - kPolyOf8) ? ex2_poly(x1) : ex2_approx(x1);
+                        rs[(c >> 1) & 3] += p0 + p1;
+                        v[c >> 1] = pack_bf16(p0, p1);
                     }
-                    tmem_st16(tS + (c0 >> 1), pk);
+                } else {
+#pragma unroll
+                    for (int c = 0; c < BS; c += 2) {
+                        const float p0 = ex2_approx(fmaf(__uint_as_float(v[c]), scale_log2, neg_m));
+                        const float p1 = ex2_approx(fmaf(__uint_as_float(v[c + 1]), scale_log2, neg_m));
+                        rs[(c >> 1) & 3] += p0 + p1;
+                        v[c >> 1] = pack_bf16(p0, p1);
+                    }
                 }
-                l = l * alpha + rs;
-                // rescale the running output when the maximum grew (PV_{j-1} has
-                // completed: the S_j commit tracks every earlier MMA)
-                const bool need = (j > 0) && (alpha != 1.0f);
-                if (__any_sync(0xffffffffu, need)) {
+#pragma unroll
+                for (int c0 = 0; c0 < BS / 2; c0 += 32)
+                    tmem_st32(tS + c0, *reinterpret_cast<const uint32_t(*)[32]>(&v[c0]));
+                l = l * alpha + ((rs[0] + rs[1]) + (rs[2] + rs[3]));
+                // rescale the running output (PV_{j-1} has completed: the S_j commit
+                // tracks every earlier MMA of this CTA)
+                if (__any_sync(0xffffffffu, need && j > 0)) {
 #pragma unroll
                     for (int c0 = 0; c0 < D; c0 += 32) {
-                        uint32_t v[32];
-                        tmem_ld32(tO + c0, v);
+                        uint32_t o[32];
+                        tmem_ld32(tO + c0, o);
                         tmem_wait_ld();
 #pragma unroll
-                        for (int c = 0; c < 32; ++c) v[c] = __float_as_uint(__uint_as_float(v[c]) * alpha);
-                        tmem_st32(tO + c0, v);
+                        for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+                        tmem_st32(tO + c0, o);
                     }
                 }
                 tmem_wait_st();

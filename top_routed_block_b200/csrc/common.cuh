@@ -5,7 +5,7 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 
-#include "../../include/fvattn.h"
+#include "fvattn.h"
 
 namespace fvattn {
 
