@@ -248,7 +248,7 @@ int fvattn_sparse_fwd(const void *Q, const void *K, const void *V, const int32_t
     a.O = O;
     a.LSE = LSE;
     a.dev_status = dev_status;
-    const int64_t max_grid = 2LL * info.sms;
+    const int64_t max_grid = static_cast<int64_t>(attn_ctas_per_sm()) * info.sms;
     a.grid = static_cast<int>(rows < max_grid ? rows : max_grid);
     return from_cuda(launch_sparse_attn(a, d, block, s));
 }

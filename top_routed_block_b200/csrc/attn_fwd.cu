@@ -11,15 +11,21 @@
 //   * One work item = one CSR row = one (b, h, query block).  A persistent grid
 //     of 2 CTAs per SM pops items from a longest-first queue (FVAttn §1 "RLB"
 //     balances per-head work at run time; here the SMs are balanced instead).
-//   * Per CTA, 6 warps: warps 0-3 own the 128 rows of the query tile (softmax,
-//     rescale, epilogue); warp 4 issues TMA loads; warp 5 issues tcgen05 MMAs.
+//   * Per CTA, 10 warps: warps 0-7 run the softmax, rescale and epilogue of the
+//     128-row query tile, two warps per row (warp w and w+4 address the same 32
+//     TMEM lanes and take the lower and upper half of the key columns; only the
+//     row maximum is exchanged, through shared memory, once per tile); warp 8
+//     issues TMA loads; warp 9 issues tcgen05 MMAs.
 //   * Q, K, V tiles arrive by TMA (3-D tensor maps over [B*H, N, d], 128-byte
 //     swizzle, out-of-range rows zero-filled).  K/V tiles are gathered by the
 //     CSR's column indices.
 //   * S = Q K^T accumulates in tensor memory (TMEM) in fp32 (SS MMA, M=128,
 //     N=block, K=16 steps over d).  The softmax warps read S with tcgen05.ld,
-//     write P as bf16 back into the same TMEM columns, and O += P V runs as a
-//     TS MMA with P taken from TMEM and V from shared memory (MN-major).
+//     write P as bf16 back into the first half of the S columns each of them
+//     read, and O += P V runs as a TS MMA with P taken from TMEM and V from
+//     shared memory (MN-major).  The next S is issued right behind the PV:
+//     tcgen05 MMAs of one thread execute in issue order, so the PV has read P
+//     before S overwrites those columns.
 //   * O (fp32) stays in TMEM for the whole item; the epilogue divides by l,
 //     converts to bf16 and stores; LSE = (m + log2 l) ln 2.
 //   * Every mbarrier wait is bounded; a timeout raises the CTA abort flag and
@@ -40,15 +46,17 @@ namespace {
 using namespace ptx;
 
 constexpr int kRowsM = 128;           // query rows per tile (tcgen05 M)
-constexpr int kThreads = 192;         // 4 softmax warps + TMA warp + MMA warp
-constexpr int kTmaWarp = 4;
-constexpr int kMmaWarp = 5;
+constexpr int kSoftmaxWarps = 8;      // two per 32-row lane group
+constexpr int kThreads = 320;         // 8 softmax warps + TMA warp + MMA warp
+constexpr int kTmaWarp = 8;
+constexpr int kMmaWarp = 9;
 constexpr uint32_t kTmemCols = 256;   // per CTA; two CTAs share an SM's 512 columns
 constexpr uint32_t kTmemS = 0;        // S (fp32, block columns) / P (bf16 pairs, block/2 columns)
 constexpr uint32_t kTmemO = 128;      // O (fp32, d columns)
-// S_{j+1} is written into the TMEM columns that hold P_j: the MMA warp waits for
-// PV_j to complete before issuing S_{j+1}.
-constexpr bool kWaitPvBeforeS = true;
+// S_{j+1} is written into the TMEM columns that hold P_j.  tcgen05 MMAs issued by
+// one thread run in issue order, so S_{j+1} may be queued right behind PV_j; with
+// this set the MMA warp instead waits for PV_j to complete first.
+constexpr bool kWaitPvBeforeS = false;
 
 template <int D, int BS>
 struct Cfg {
@@ -60,7 +68,10 @@ struct Cfg {
     static constexpr int OFF_K = Q_BYTES;
     static constexpr int OFF_V = Q_BYTES + KV_BYTES;
     static constexpr int TILE_BYTES = Q_BYTES + 2 * KV_BYTES;
-    static constexpr int SMEM_BYTES = TILE_BYTES + 1024 /*align slack*/ + 256 /*barriers etc*/;
+    // row-max exchange between the two warps of a lane group: buffers 0/1 alternate
+    // by tile, buffers 2/3 by item (row sums at the epilogue); each [2 halves][rows]
+    static constexpr int XCHG_BYTES = 4 * 2 * kRowsM * 4;
+    static constexpr int SMEM_BYTES = TILE_BYTES + 1024 /*align slack*/ + 256 /*barriers etc*/ + XCHG_BYTES;
     static constexpr uint32_t IDESC_S = idesc_bf16_f32(kRowsM, BS, 0, 0);
     static constexpr uint32_t IDESC_PV = idesc_bf16_f32(kRowsM, D, 0, 1);
 };
@@ -112,6 +123,11 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
     return r;
 }
 
+// Named barrier for the two warps that share a lane group (ids 1..4; 0 is __syncthreads).
+__device__ __forceinline__ void pair_sync(int group) {
+    asm volatile("bar.sync %0, 64;" ::"r"(group + 1) : "memory");
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&v);
@@ -146,13 +162,13 @@ __global__ void __launch_bounds__(kThreads, 2)
         mbar_init(&bar->v_full, 1);
         mbar_init(&bar->v_empty, 1);
         mbar_init(&bar->s_full, 1);
-        mbar_init(&bar->p_full, 4);
+        mbar_init(&bar->p_full, kSoftmaxWarps);
         mbar_init(&bar->o_full, 1);
-        mbar_init(&bar->o_empty, 4);
+        mbar_init(&bar->o_empty, kSoftmaxWarps);
         mbar_init(&bar->pv_done, 1);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&bar->sched_full[i], 1);
-            mbar_init(&bar->sched_empty[i], 1 + 4);
+            mbar_init(&bar->sched_empty[i], 1 + kSoftmaxWarps);
         }
         mbar_init(&bar->drain, 1);
         bar->abort_flag = 0;
@@ -282,8 +298,10 @@ __global__ void __launch_bounds__(kThreads, 2)
                     tc_fence_after();
 #pragma unroll
                     for (int k = 0; k < BS / 16; ++k) {
+                        // keys [16k, 16k+16): P of column half h sits at h*BS/2, packed in pairs
+                        const uint32_t pcol = 8 * k + (k / (BS / 32)) * (BS / 4);
                         const uint64_t dv = smem_desc_sw128(v0 + k * 16 * 128, BS * 128, 1024);
-                        mma_ts(tO, tS + k * 8, dv, C::IDESC_PV, (j > 0 || k > 0) ? 1u : 0u);
+                        mma_ts(tO, tS + pcol, dv, C::IDESC_PV, (j > 0 || k > 0) ? 1u : 0u);
                     }
                     mma_commit(&bar->v_empty);
                     mma_commit(&bar->pv_done);
@@ -304,10 +322,17 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
     } else {
         // ------------------------------------------------ softmax / epilogue
-        const int r = threadIdx.x;                                 // tile row = TMEM lane
-        const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-        const uint32_t tS = tmem + kTmemS + lane_base;
-        const uint32_t tO = tmem + kTmemO + lane_base;
+        // warp w: rows 32*(w%4) .. +31 (its TMEM lane quarter), key columns of half
+        // h = w/4; the two warps of a lane group exchange their row maxima.
+        constexpr int HALF = BS / 2;               // S columns per warp
+        constexpr int OHALF = D / 2;               // O columns per warp
+        const int g = warp & 3, h = warp >> 2;
+        const int r = g * 32 + lane;                               // tile row = TMEM lane
+        const uint32_t lane_base = static_cast<uint32_t>(g * 32) << 16;
+        const uint32_t tS = tmem + kTmemS + lane_base + h * HALF;  // this warp's S columns; P goes
+                                                                   // to the first HALF/2 of them
+        const uint32_t tO = tmem + kTmemO + lane_base + h * OHALF;
+        float *xchg = reinterpret_cast<float *>(smem + C::TILE_BYTES + 256);  // [4][2][kRowsM]
         uint32_t it = 0, sc = 0;
         while (true) {
             const uint32_t slot = it & 1;
@@ -320,7 +345,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             const int64_t bh = row / nb;
             const int qb = row % nb;
             const int t_row = qb * BS + r;                         // token index of this thread's row
-            float m = -CUDART_INF_F, l = 0.0f;
+            float m = -CUDART_INF_F, l = 0.0f;                     // l: this half's share of the row sum
             int prev = -1;
             bool ok = true;
             for (int j = 0; j < count; ++j) {
@@ -328,42 +353,49 @@ __global__ void __launch_bounds__(kThreads, 2)
                 const bool valid = kblk >= 0 && kblk < nb && kblk > prev;
                 if (valid) prev = kblk;
                 const int key0 = kblk * BS;
-                // keys of this block that exist and are allowed for this row
+                // keys of this block that exist and are allowed for this row, counted
+                // from the start of this warp's column half
                 int lim = valid ? min(BS, N - key0) : 0;
                 if (causal) lim = min(lim, t_row - key0 + 1);
+                lim -= h * HALF;
                 if (!mbar_wait(&bar->s_full, sc & 1, abort_flag, dev_status)) { ok = false; break; }
                 ++sc;
                 tc_fence_after();
-                // the whole S row of this thread: BS fp32 values
-                uint32_t v[BS];
+                uint32_t v[HALF];
 #pragma unroll
-                for (int c0 = 0; c0 < BS; c0 += 32) tmem_ld32(tS + c0, *reinterpret_cast<uint32_t(*)[32]>(&v[c0]));
+                for (int c0 = 0; c0 < HALF; c0 += 32)
+                    tmem_ld32(tS + c0, *reinterpret_cast<uint32_t(*)[32]>(&v[c0]));
                 tmem_wait_ld();
-                if (lim < BS) {  // ragged last block, causal diagonal, or a skipped index
+                if (lim < HALF) {  // ragged last block, causal diagonal, or a skipped index
 #pragma unroll
-                    for (int c = 0; c < BS; ++c)
+                    for (int c = 0; c < HALF; ++c)
                         if (c >= lim) v[c] = __float_as_uint(-CUDART_INF_F);
                 }
                 float mq[4] = {-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F};
 #pragma unroll
-                for (int c = 0; c < BS; c += 8) {
+                for (int c = 0; c < HALF; c += 8) {
 #pragma unroll
                     for (int q = 0; q < 4; ++q)
                         mq[q] = max3f(mq[q], __uint_as_float(v[c + 2 * q]), __uint_as_float(v[c + 2 * q + 1]));
                 }
-                const float mxs = max3f(mq[0], mq[1], fmaxf(mq[2], mq[3])) * scale_log2;
+                const float mine = max3f(mq[0], mq[1], fmaxf(mq[2], mq[3]));
+                float *xb = xchg + (j & 1) * 2 * kRowsM;
+                xb[h * kRowsM + r] = mine;
+                pair_sync(g);
+                const float mxs = fmaxf(mine, xb[(1 - h) * kRowsM + r]) * scale_log2;
                 // The reference maximum only moves when the row maximum exceeds it by
                 // more than 2^8: P stays below 256 and the rescale of O is rare.  O and
-                // l always share the same reference, so the final O / l is exact.
+                // l always share the same reference, so the final O / l is exact.  Both
+                // warps of a row take the same decision from the same values.
                 const bool need = mxs > m + kRescaleLog2;
                 const float m_new = need ? mxs : m;
                 const float alpha = need ? ex2_approx(m - m_new) : 1.0f;
                 const float neg_m = (m_new == -CUDART_INF_F) ? 0.0f : -m_new;
                 float rs[4] = {0.0f, 0.0f, 0.0f, 0.0f};
                 // P packed as bf16 pairs in place: v[c/2] <- (p[c], p[c+1])
-                if (lim >= BS) {
+                if (lim >= HALF) {
 #pragma unroll
-                    for (int c = 0; c < BS; c += 2) {
+                    for (int c = 0; c < HALF; c += 2) {
                         const float x0 = fmaf(__uint_as_float(v[c]), scale_log2, neg_m);
                         const float x1 = fmaf(__uint_as_float(v[c + 1]), scale_log2, neg_m);
                         const float p0 = ((c & 7) >= 8 - kPolyOf8) ? ex2_poly(x0) : ex2_approx(x0);
@@ -373,22 +405,26 @@ __global__ void __launch_bounds__(kThreads, 2)
                     }
                 } else {
 #pragma unroll
-                    for (int c = 0; c < BS; c += 2) {
+                    for (int c = 0; c < HALF; c += 2) {
                         const float p0 = ex2_approx(fmaf(__uint_as_float(v[c]), scale_log2, neg_m));
                         const float p1 = ex2_approx(fmaf(__uint_as_float(v[c + 1]), scale_log2, neg_m));
                         rs[(c >> 1) & 3] += p0 + p1;
                         v[c >> 1] = pack_bf16(p0, p1);
                     }
                 }
+                if constexpr (HALF / 2 >= 32) {
 #pragma unroll
-                for (int c0 = 0; c0 < BS / 2; c0 += 32)
-                    tmem_st32(tS + c0, *reinterpret_cast<const uint32_t(*)[32]>(&v[c0]));
+                    for (int c0 = 0; c0 < HALF / 2; c0 += 32)
+                        tmem_st32(tS + c0, *reinterpret_cast<const uint32_t(*)[32]>(&v[c0]));
+                } else {
+                    tmem_st16(tS, *reinterpret_cast<const uint32_t(*)[16]>(&v[0]));
+                }
                 l = l * alpha + ((rs[0] + rs[1]) + (rs[2] + rs[3]));
-                // rescale the running output (PV_{j-1} has completed: the S_j commit
-                // tracks every earlier MMA of this CTA)
+                // rescale this warp's half of the running output (PV_{j-1} has completed:
+                // the S_j commit tracks every earlier MMA of this CTA)
                 if (__any_sync(0xffffffffu, need && j > 0)) {
 #pragma unroll
-                    for (int c0 = 0; c0 < D; c0 += 32) {
+                    for (int c0 = 0; c0 < OHALF; c0 += 32) {
                         uint32_t o[32];
                         tmem_ld32(tO + c0, o);
                         tmem_wait_ld();
@@ -404,14 +440,18 @@ __global__ void __launch_bounds__(kThreads, 2)
                 m = m_new;
             }
             if (!ok) break;
-            // epilogue
+            // epilogue: row sum = both halves' shares
+            float *xl = xchg + (2 + (it & 1)) * 2 * kRowsM;
+            xl[h * kRowsM + r] = l;
+            pair_sync(g);
+            const float lsum = l + xl[(1 - h) * kRowsM + r];
             if (!mbar_wait(&bar->o_full, it & 1, abort_flag, dev_status)) break;
             tc_fence_after();
             const bool row_ok = r < BS && t_row < N;
-            const float inv_l = (l > 0.0f) ? 1.0f / l : 0.0f;
-            __nv_bfloat16 *orow = O + (bh * N + t_row) * D;
+            const float inv_l = (lsum > 0.0f) ? 1.0f / lsum : 0.0f;
+            __nv_bfloat16 *orow = O + (bh * N + t_row) * D + h * OHALF;
 #pragma unroll
-            for (int c0 = 0; c0 < D; c0 += 32) {
+            for (int c0 = 0; c0 < OHALF; c0 += 32) {
                 uint32_t v[32];
                 if (count > 0) {
                     tmem_ld32(tO + c0, v);
@@ -430,7 +470,8 @@ __global__ void __launch_bounds__(kThreads, 2)
                     for (int q = 0; q < 4; ++q) dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
                 }
             }
-            if (row_ok) LSE[bh * N + t_row] = (l > 0.0f) ? (m + __log2f(l)) * 0.69314718055994531f : -CUDART_INF_F;
+            if (row_ok && h == 0)
+                LSE[bh * N + t_row] = (lsum > 0.0f) ? (m + __log2f(lsum)) * 0.69314718055994531f : -CUDART_INF_F;
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar->o_empty);
@@ -474,3 +515,4 @@ cudaError_t launch_sparse_attn(const AttnLaunch &a, int d, int bs, cudaStream_t 
 }
 
 }  // namespace fvattn
+namespace fvattn { int attn_ctas_per_sm() { return 2; } }

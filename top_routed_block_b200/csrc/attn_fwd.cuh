@@ -21,6 +21,7 @@ struct AttnLaunch {
 };
 
 int attn_smem_bytes(int d, int bs);
+int attn_ctas_per_sm();  // resident CTAs per SM the launch grid is sized for
 cudaError_t launch_sparse_attn(const AttnLaunch &a, int d, int bs, cudaStream_t stream);
 
 }  // namespace fvattn
