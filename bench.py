@@ -135,13 +135,25 @@ def dist_setup(n_gpus: int):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """Largest value over the ranks (the step time of the slowest replica)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(flops_per_rank_step: float, world: int, steps: int, max_ms: float) -> float:
+    """Whole-job TFLOP/s: every rank runs its own replica of the workload (weak scaling)."""
+    return world * flops_per_rank_step * steps / (max_ms * 1e-3) / 1e12
+
+
+def replica_seed(w: W.Workload, rank: int) -> int:
+    """Each rank draws its own input of the same shape."""
+    return w.seed + rank
 
 
 def barrier(world: int):
@@ -222,7 +234,7 @@ def run_ours(args, w, rank, world, local):
     import top_routed_block_b200 as fv
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    Qh, Kh, Vh = W.generate(w, seed=w.seed + rank)
+    Qh, Kh, Vh = W.generate(w, seed=replica_seed(w, rank))
 
     def pinned(a):
         t = torch.from_numpy(a.view(np.int16)).view(torch.bfloat16)
@@ -269,7 +281,7 @@ def run_ours(args, w, rank, world, local):
     fwd_ms = [b.elapsed_time(c) for _, b, c in ev]
     total_ms_max = max_over_ranks(total_ms, world)
     ms_per_step = total_ms_max / args.steps
-    value = world * flops * args.steps / (total_ms_max * 1e-3) / 1e12
+    value = job_throughput(flops, world, args.steps, total_ms_max)
     attn_ms = statistics.mean(fwd_ms)
     attn_tflops = flops / (attn_ms * 1e-3) / 1e12
     r_ms = statistics.mean(route_ms)

@@ -207,6 +207,19 @@ FVATTN_API int fvattn_sparse_fwd_noalloc(const void *Q, const void *K, const voi
                                          const int32_t *col_idx, int B, int H, int N, int d, int block, int causal,
                                          void *O, float *LSE, int32_t *dev_status, fvattn_stream_t stream);
 
+/*
+ * fvattn_test_sparse_fwd_stall -- test hook for failure detection, not for
+ * production use.  Same arguments as fvattn_sparse_fwd; the CTA that takes the
+ * first work item never receives that item's Q tile, so one of its bounded
+ * waits runs out (after about one second) and the call ends with
+ * *dev_status = FVATTN_ERR_DEVICE_TIMEOUT, the rest of the grid finishing its
+ * items.  No fault, trap or hang: the CUDA context stays usable.
+ */
+FVATTN_API int fvattn_test_sparse_fwd_stall(const void *Q, const void *K, const void *V, const int32_t *row_ptr,
+                                            const int32_t *col_idx, int B, int H, int N, int d, int block,
+                                            int causal, void *O, float *LSE, void *workspace, size_t ws_bytes,
+                                            int32_t *dev_status, fvattn_stream_t stream);
+
 /* Compiled-in build description (architecture, version), static string. */
 FVATTN_API const char *fvattn_build_info(void);
 

@@ -67,6 +67,7 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         "fvattn_lpt_order": (I, [P, I64, I, P, P, SZ, P, P]),
         "fvattn_sparse_fwd": (I, [P, P, P, P, P, I, I, I, I, I, I, P, P, P, SZ, P, P]),
         "fvattn_sparse_fwd_noalloc": (I, [P, P, P, P, P, I, I, I, I, I, I, P, P, P, P]),
+        "fvattn_test_sparse_fwd_stall": (I, [P, P, P, P, P, I, I, I, I, I, I, P, P, P, SZ, P, P]),
         "fvattn_attention_host": (I, [P, P, P, I, I, I, I, I, D, I, P, P, P, P, P, P, P, P, P, I64, P, P, SZ, P, SZ,
                                       P, P]),
     }

@@ -196,9 +196,10 @@ int fvattn_lpt_order(const int32_t *row_ptr, int64_t rows, int max_count, int32_
     return from_cuda(launch_lpt_order(row_ptr, rows, max_count, order, workspace, dev_status, s));
 }
 
-int fvattn_sparse_fwd(const void *Q, const void *K, const void *V, const int32_t *row_ptr, const int32_t *col_idx,
-                      int B, int H, int N, int d, int block, int causal, void *O, float *LSE, void *workspace,
-                      size_t ws_bytes, int32_t *dev_status, fvattn_stream_t stream) {
+static int sparse_fwd_impl(const void *Q, const void *K, const void *V, const int32_t *row_ptr,
+                           const int32_t *col_idx, int B, int H, int N, int d, int block, int causal, void *O,
+                           float *LSE, void *workspace, size_t ws_bytes, int32_t *dev_status, fvattn_stream_t stream,
+                           int test_stall) {
     int rc = check_shape(B, H, N, d, block);
     if (rc != FVATTN_OK) return rc;
     if (!Q || !K || !V || !row_ptr || !col_idx || !O || !LSE || !workspace || !dev_status)
@@ -250,7 +251,23 @@ int fvattn_sparse_fwd(const void *Q, const void *K, const void *V, const int32_t
     a.dev_status = dev_status;
     const int64_t max_grid = static_cast<int64_t>(attn_ctas_per_sm()) * info.sms;
     a.grid = static_cast<int>(rows < max_grid ? rows : max_grid);
+    a.test_stall = test_stall;
     return from_cuda(launch_sparse_attn(a, d, block, s));
+}
+
+int fvattn_sparse_fwd(const void *Q, const void *K, const void *V, const int32_t *row_ptr, const int32_t *col_idx,
+                      int B, int H, int N, int d, int block, int causal, void *O, float *LSE, void *workspace,
+                      size_t ws_bytes, int32_t *dev_status, fvattn_stream_t stream) {
+    return sparse_fwd_impl(Q, K, V, row_ptr, col_idx, B, H, N, d, block, causal, O, LSE, workspace, ws_bytes,
+                           dev_status, stream, 0);
+}
+
+int fvattn_test_sparse_fwd_stall(const void *Q, const void *K, const void *V, const int32_t *row_ptr,
+                                 const int32_t *col_idx, int B, int H, int N, int d, int block, int causal, void *O,
+                                 float *LSE, void *workspace, size_t ws_bytes, int32_t *dev_status,
+                                 fvattn_stream_t stream) {
+    return sparse_fwd_impl(Q, K, V, row_ptr, col_idx, B, H, N, d, block, causal, O, LSE, workspace, ws_bytes,
+                           dev_status, stream, 1);
 }
 
 int fvattn_attention_host(const void *hQ, const void *hK, const void *hV, int B, int H, int N, int d, int block,

@@ -139,7 +139,8 @@ __global__ void __launch_bounds__(kThreads, 2)
                            const __grid_constant__ CUtensorMap tmap_v, const int32_t *__restrict__ row_ptr,
                            const int32_t *__restrict__ col_idx, const int32_t *__restrict__ order, int n_items,
                            int *__restrict__ work_counter, int N, int nb, int causal, float scale_log2,
-                           __nv_bfloat16 *__restrict__ O, float *__restrict__ LSE, int32_t *dev_status) {
+                           __nv_bfloat16 *__restrict__ O, float *__restrict__ LSE, int32_t *dev_status,
+                           int test_stall) {
     using C = Cfg<D, BS>;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     // 1024-byte alignment for the 128-byte-swizzled tiles
@@ -220,10 +221,14 @@ __global__ void __launch_bounds__(kThreads, 2)
                 const int bh = row / nb;
                 const int qb = row % nb;
                 if (!mbar_wait(&bar->q_empty, (it & 1) ^ 1, abort_flag, dev_status)) break;
-                mbar_arrive_expect_tx(&bar->q_full, C::Q_LOAD_BYTES);
-                for (int kb = 0; kb < C::KBLK; ++kb)
-                    tma_load_3d(sQ + kb * kRowsM * 128, &tmap_q, &bar->q_full, kb * 64, qb * BS, bh);
-                q_armed = it + 1;
+                // Test hook: CTA 0 leaves the Q tile of its first item unloaded, so the
+                // MMA warp's bounded wait for it runs out (exercises the timeout path).
+                if (!(test_stall && blockIdx.x == 0 && it == 0)) {
+                    mbar_arrive_expect_tx(&bar->q_full, C::Q_LOAD_BYTES);
+                    for (int kb = 0; kb < C::KBLK; ++kb)
+                        tma_load_3d(sQ + kb * kRowsM * 128, &tmap_q, &bar->q_full, kb * 64, qb * BS, bh);
+                    q_armed = it + 1;
+                }
                 int prev = -1;
                 for (int j = 0; j < count && ok; ++j) {
                     int kblk = col_idx[start + j];
@@ -503,7 +508,7 @@ static cudaError_t launch_t(const AttnLaunch &a, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     kern<<<a.grid, kThreads, Cfg<D, BS>::SMEM_BYTES, stream>>>(
         *a.tmap_q, *a.tmap_k, *a.tmap_v, a.row_ptr, a.col_idx, a.order, a.n_items, a.work_counter, a.N, a.nb,
-        a.causal, a.scale_log2, static_cast<__nv_bfloat16 *>(a.O), a.LSE, a.dev_status);
+        a.causal, a.scale_log2, static_cast<__nv_bfloat16 *>(a.O), a.LSE, a.dev_status, a.test_stall);
     return cudaGetLastError();
 }
 

@@ -18,6 +18,7 @@ struct AttnLaunch {
     float *LSE;
     int32_t *dev_status;
     int grid;
+    int test_stall;     // nonzero only from the test hook: one bounded wait runs out
 };
 
 int attn_smem_bytes(int d, int bs);
