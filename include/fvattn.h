@@ -192,7 +192,7 @@ FVATTN_API int fvattn_attention_host(const void *hQ, const void *hK, const void 
  * file-scope device array of FVATTN_NOALLOC_SCRATCH_BYTES (4 MiB) inside the
  * library, which every device that loads the library keeps until the process
  * exits.  Shapes that need more return FVATTN_ERR_CAPACITY without launching
- * anything (about 400k rows B*H*ceil(N/block) at most).
+ * anything (about 500k rows B*H*ceil(N/block) at most).
  *
  * The first call on each device looks up the array's device address
  * (cudaGetSymbolAddress, with that device current) and caches it; make that first

@@ -96,16 +96,18 @@ bool make_map(CUtensorMap *m, const void *base, int64_t BH, int N, int d, int ro
 }
 
 struct FwdWorkspace {
-    size_t order, counter, lpt, total;
+    size_t order, item_ptr, counter, lpt, total;
 };
 
-FwdWorkspace fwd_layout(int64_t rows, int max_count) {
+// items: work items of the attention kernel; max_count: largest blocks per item.
+FwdWorkspace fwd_layout(int64_t items, int max_count) {
     FwdWorkspace w{};
     Carver c;
-    w.order = c.take<int32_t>(static_cast<size_t>(rows));
+    w.order = c.take<int32_t>(static_cast<size_t>(items));
+    w.item_ptr = c.take<int32_t>(static_cast<size_t>(items) + 1);
     w.counter = c.take<int32_t>(64);
     w.lpt = align_up(c.off, 256);
-    w.total = w.lpt + lpt_workspace_layout(rows, max_count).total;
+    w.total = w.lpt + lpt_workspace_layout(items, max_count).total;
     return w;
 }
 
@@ -157,7 +159,8 @@ size_t fvattn_fwd_workspace_bytes(int B, int H, int N, int block) {
     if (B < 1 || H < 1 || N < 1 || (block != 64 && block != 128)) return 0;
     const int64_t nb = ceil_div(N, block);
     if (nb > kMaxCount) return 0;
-    return fwd_layout(static_cast<int64_t>(B) * H * nb, static_cast<int>(nb)).total;
+    return fwd_layout(attn_num_items(static_cast<int64_t>(B) * H, static_cast<int>(nb)), 2 * static_cast<int>(nb))
+        .total;
 }
 
 int fvattn_route(const void *Q, const void *K, int B, int H, int N, int d, int block, double p, int32_t *row_ptr,
@@ -217,9 +220,11 @@ static int sparse_fwd_impl(const void *Q, const void *K, const void *V, const in
     const int64_t BH = static_cast<int64_t>(B) * H;
     const int nb = static_cast<int>(ceil_div(N, block));
     const int64_t rows = BH * nb;
-    const FwdWorkspace w = fwd_layout(rows, nb);
+    const int64_t items = attn_num_items(BH, nb);
+    const FwdWorkspace w = fwd_layout(items, 2 * nb);
     char *ws = static_cast<char *>(workspace);
     int32_t *order = reinterpret_cast<int32_t *>(ws + w.order);
+    int32_t *item_ptr = reinterpret_cast<int32_t *>(ws + w.item_ptr);
     int *counter = reinterpret_cast<int *>(ws + w.counter);
 
     CUtensorMap mq, mk, mv;
@@ -229,7 +234,10 @@ static int sparse_fwd_impl(const void *Q, const void *K, const void *V, const in
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if ((rc = from_cuda(cudaMemsetAsync(dev_status, 0, sizeof(int32_t), s))) != FVATTN_OK) return rc;
-    if ((rc = from_cuda(launch_lpt_order(row_ptr, rows, nb, order, ws + w.lpt, dev_status, s))) != FVATTN_OK)
+    // work items (pairs of neighbouring query blocks) longest first
+    if ((rc = from_cuda(launch_pair_row_ptr(row_ptr, BH, nb, item_ptr, s))) != FVATTN_OK) return rc;
+    if ((rc = from_cuda(launch_lpt_order(item_ptr, items, 2 * nb, order, ws + w.lpt, dev_status, s))) !=
+        FVATTN_OK)
         return rc;
     if ((rc = from_cuda(cudaMemsetAsync(counter, 0, sizeof(int), s))) != FVATTN_OK) return rc;
 
@@ -240,7 +248,7 @@ static int sparse_fwd_impl(const void *Q, const void *K, const void *V, const in
     a.row_ptr = row_ptr;
     a.col_idx = col_idx;
     a.order = order;
-    a.n_items = static_cast<int>(rows);
+    a.n_items = static_cast<int>(items);
     a.work_counter = counter;
     a.N = N;
     a.nb = nb;
@@ -250,7 +258,7 @@ static int sparse_fwd_impl(const void *Q, const void *K, const void *V, const in
     a.LSE = LSE;
     a.dev_status = dev_status;
     const int64_t max_grid = static_cast<int64_t>(attn_ctas_per_sm()) * info.sms;
-    a.grid = static_cast<int>(rows < max_grid ? rows : max_grid);
+    a.grid = static_cast<int>(items < max_grid ? items : max_grid);
     a.test_stall = test_stall;
     return from_cuda(launch_sparse_attn(a, d, block, s));
 }

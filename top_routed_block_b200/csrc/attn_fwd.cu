@@ -8,24 +8,32 @@
 // partial output rescaled by exp(m_old - m_new) whenever the maximum grows.
 //
 // B200 design:
-//   * One work item = one CSR row = one (b, h, query block).  A persistent grid
-//     of 2 CTAs per SM pops items from a longest-first queue (FVAttn §1 "RLB"
-//     balances per-head work at run time; here the SMs are balanced instead).
-//   * Per CTA, 10 warps: warps 0-7 run the softmax, rescale and epilogue of the
-//     128-row query tile, two warps per row (warp w and w+4 address the same 32
-//     TMEM lanes and take the lower and upper half of the key columns; only the
-//     row maximum is exchanged, through shared memory, once per tile); warp 8
-//     issues TMA loads; warp 9 issues tcgen05 MMAs.
-//   * Q, K, V tiles arrive by TMA (3-D tensor maps over [B*H, N, d], 128-byte
-//     swizzle, out-of-range rows zero-filled).  K/V tiles are gathered by the
-//     CSR's column indices.
+//   * One work item = two neighbouring query blocks (2i, 2i+1) of one head:
+//     slots A and B, each with its own CSR row.  Top-p routing gives
+//     neighbouring query blocks mostly the same key blocks, so the item walks
+//     the merge of the two sorted block lists and loads every key block of the
+//     union once; a block selected by only one of the rows is computed for that
+//     row only (no wasted tensor-core work).  A persistent grid of one CTA per
+//     SM pops items longest-first (FVAttn §1 "RLB" balances per-head work at
+//     run time; here the SMs are balanced instead).
+//   * Warps 0-3 run the softmax, rescale and epilogue of slot A, warps 4-7 those
+//     of slot B (thread = query row = TMEM lane); warp 8 issues TMA loads; warp
+//     9 issues tcgen05 MMAs.  Per union block the MMA warp issues
+//     S_A, PV_B(previous B block), S_B, PV_A: while one warpgroup runs the
+//     softmax of its tile, the tensor cores run the other slot's two GEMMs.
+//   * Q tiles (one per slot) and a ring of K/V stages arrive by TMA (3-D tensor
+//     maps over [B*H, N, d], 128-byte swizzle, out-of-range rows zero-filled).
+//     The producer walks the same merge as the MMA warp, so the ring is
+//     consumed in the order it is filled; a K stage is released after its S
+//     GEMMs, a V stage after its PV GEMMs.
 //   * S = Q K^T accumulates in tensor memory (TMEM) in fp32 (SS MMA, M=128,
 //     N=block, K=16 steps over d).  The softmax warps read S with tcgen05.ld,
-//     write P as bf16 back into the first half of the S columns each of them
-//     read, and O += P V runs as a TS MMA with P taken from TMEM and V from
-//     shared memory (MN-major).  The next S is issued right behind the PV:
-//     tcgen05 MMAs of one thread execute in issue order, so the PV has read P
-//     before S overwrites those columns.
+//     write P as bf16 back into the same TMEM columns, and O += P V runs as a
+//     TS MMA with P taken from TMEM and V from shared memory (MN-major).  The
+//     next S of a slot is queued behind that slot's PV: tcgen05 MMAs of one
+//     thread execute in issue order, so the PV has read P before S overwrites
+//     those columns.
+//   * TMEM (512 columns): slot X uses S/P at X*256 and O at X*256 + 128.
 //   * O (fp32) stays in TMEM for the whole item; the epilogue divides by l,
 //     converts to bf16 and stores; LSE = (m + log2 l) ln 2.
 //   * Every mbarrier wait is bounded; a timeout raises the CTA abort flag and
@@ -46,43 +54,96 @@ namespace {
 using namespace ptx;
 
 constexpr int kRowsM = 128;           // query rows per tile (tcgen05 M)
-constexpr int kSoftmaxWarps = 8;      // two per 32-row lane group
-constexpr int kThreads = 320;         // 8 softmax warps + TMA warp + MMA warp
+constexpr int kSlots = 2;             // query blocks per work item
+constexpr int kThreads = 320;         // 2 softmax warpgroups + TMA warp + MMA warp
 constexpr int kTmaWarp = 8;
 constexpr int kMmaWarp = 9;
-constexpr uint32_t kTmemCols = 256;   // per CTA; two CTAs share an SM's 512 columns
-constexpr uint32_t kTmemS = 0;        // S (fp32, block columns) / P (bf16 pairs, block/2 columns)
-constexpr uint32_t kTmemO = 128;      // O (fp32, d columns)
-// S_{j+1} is written into the TMEM columns that hold P_j.  tcgen05 MMAs issued by
-// one thread run in issue order, so S_{j+1} may be queued right behind PV_j; with
-// this set the MMA warp instead waits for PV_j to complete first.
-constexpr bool kWaitPvBeforeS = false;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTmemSlot = 256;   // TMEM columns per slot
+constexpr uint32_t kTmemO = 128;      // O offset inside a slot (S/P at offset 0)
+constexpr int kMinSmem = 120 * 1024;  // more than half an SM's shared memory: one CTA per SM
 
 template <int D, int BS>
 struct Cfg {
-    static constexpr int KBLK = D / 64;                 // 128-byte (64 x bf16) column blocks along d
-    static constexpr int Q_BYTES = KBLK * kRowsM * 128;
-    static constexpr int KV_BYTES = KBLK * BS * 128;
+    static constexpr int KBLK = D / 64;                   // 128-byte (64 x bf16) column blocks along d
+    static constexpr int Q_BYTES = KBLK * kRowsM * 128;   // one Q tile buffer
     static constexpr int Q_LOAD_BYTES = KBLK * BS * 128;  // only the block's rows are loaded
-    static constexpr int OFF_Q = 0;
-    static constexpr int OFF_K = Q_BYTES;
-    static constexpr int OFF_V = Q_BYTES + KV_BYTES;
-    static constexpr int TILE_BYTES = Q_BYTES + 2 * KV_BYTES;
-    // row-max exchange between the two warps of a lane group: buffers 0/1 alternate
-    // by tile, buffers 2/3 by item (row sums at the epilogue); each [2 halves][rows]
-    static constexpr int XCHG_BYTES = 4 * 2 * kRowsM * 4;
-    static constexpr int SMEM_BYTES = TILE_BYTES + 1024 /*align slack*/ + 256 /*barriers etc*/ + XCHG_BYTES;
+    static constexpr int STAGE_BYTES = KBLK * BS * 128;   // one K or V tile
+    static constexpr int NST = STAGE_BYTES >= 32768 ? 4 : 8;
+    static constexpr int OFF_RING = kSlots * Q_BYTES;
+    static constexpr int TILE_BYTES = OFF_RING + NST * STAGE_BYTES;
+    static constexpr int NEED = TILE_BYTES + 1024 /*alignment slack*/ + 512 /*barriers*/;
+    static constexpr int SMEM_BYTES = NEED > kMinSmem ? NEED : kMinSmem;
     static constexpr uint32_t IDESC_S = idesc_bf16_f32(kRowsM, BS, 0, 0);
     static constexpr uint32_t IDESC_PV = idesc_bf16_f32(kRowsM, D, 0, 1);
 };
 
 struct Barriers {
-    uint64_t q_full, q_empty, k_full, k_empty, v_full, v_empty, s_full, p_full, o_full, o_empty, pv_done;
+    uint64_t ring_full[8], ring_empty[8];
+    uint64_t q_full[kSlots], q_empty[kSlots], s_full[kSlots], p_full[kSlots], o_full[kSlots], o_empty[kSlots];
     uint64_t sched_full[2], sched_empty[2];
     uint64_t drain;
-    int4 sched_item[2];   // {row, col start, count, valid}
+    int4 sched_item[2][kSlots];  // per slot: {row or -1, col start, count, valid item}
     uint32_t tmem_base;
     int abort_flag;
+};
+
+// One step of the merge of the two rows' key-block lists.
+struct Step {
+    int kblk;   // key block to load (0 for a skipped index)
+    bool pa, pb;
+};
+
+// Walks the union of two strictly ascending key-block lists in order.  An entry
+// that is out of range or not ascending is processed alone (its tile is loaded
+// from block 0 and masked out by that row's softmax), so the producer, the MMA
+// warp and the softmax warps all see each row's tiles in CSR order.
+struct Merge {
+    const int32_t *a, *b;
+    int na, nbl, ia, ib, prev_a, prev_b, nkb;
+    bool bad;  // the last step was a skipped index
+    __device__ void init(const int32_t *col_idx, int4 sa, int4 sb, int nkb_) {
+        a = col_idx + sa.y;
+        na = sa.x >= 0 ? sa.z : 0;
+        b = col_idx + sb.y;
+        nbl = sb.x >= 0 ? sb.z : 0;
+        ia = ib = 0;
+        prev_a = prev_b = -1;
+        nkb = nkb_;
+        bad = false;
+    }
+    __device__ bool done() const { return ia >= na && ib >= nbl; }
+    __device__ Step next() {
+        const bool ha = ia < na, hb = ib < nbl;
+        const int xa = ha ? a[ia] : 0, xb = hb ? b[ib] : 0;
+        const bool va = ha && xa >= 0 && xa < nkb && xa > prev_a;
+        const bool vb = hb && xb >= 0 && xb < nkb && xb > prev_b;
+        Step s;
+        bad = false;
+        if (ha && !va) {
+            s = {0, true, false};
+            bad = true;
+            ++ia;
+        } else if (hb && !vb) {
+            s = {0, false, true};
+            bad = true;
+            ++ib;
+        } else if (ha && hb && xa == xb) {
+            s = {xa, true, true};
+            prev_a = prev_b = xa;
+            ++ia;
+            ++ib;
+        } else if (ha && (!hb || xa < xb)) {
+            s = {xa, true, false};
+            prev_a = xa;
+            ++ia;
+        } else {
+            s = {xb, false, true};
+            prev_b = xb;
+            ++ib;
+        }
+        return s;
+    }
 };
 
 constexpr float kRescaleLog2 = 8.0f;  // rescale O only when the row max grows by more than 2^8
@@ -113,8 +174,7 @@ __device__ __forceinline__ float ex2_poly(float x) {
 }
 
 // Of every 8 exponentials of a full (unmasked) block, this many run as ex2_poly on
-// the FMA pipe instead of the MUFU unit, whose throughput otherwise equals the MMA
-// time per tile.
+// the FMA pipe instead of the MUFU unit.
 constexpr int kPolyOf8 = 0;
 
 __device__ __forceinline__ float max3f(float a, float b, float c) {
@@ -123,18 +183,13 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
     return r;
 }
 
-// Named barrier for the two warps that share a lane group (ids 1..4; 0 is __syncthreads).
-__device__ __forceinline__ void pair_sync(int group) {
-    asm volatile("bar.sync %0, 64;" ::"r"(group + 1) : "memory");
-}
-
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
 template <int D, int BS>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, 1)
     sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                            const __grid_constant__ CUtensorMap tmap_v, const int32_t *__restrict__ row_ptr,
                            const int32_t *__restrict__ col_idx, const int32_t *__restrict__ order, int n_items,
@@ -146,30 +201,31 @@ __global__ void __launch_bounds__(kThreads, 2)
     // 1024-byte alignment for the 128-byte-swizzled tiles
     const uint32_t base_addr = smem_addr(smem_raw);
     unsigned char *smem = smem_raw + ((1024 - (base_addr & 1023)) & 1023);
-    unsigned char *sQ = smem + C::OFF_Q;
-    unsigned char *sK = smem + C::OFF_K;
-    unsigned char *sV = smem + C::OFF_V;
+    unsigned char *sQ = smem;                    // slot X at X * Q_BYTES
+    unsigned char *ring = smem + C::OFF_RING;    // stage s at s * STAGE_BYTES
     Barriers *bar = reinterpret_cast<Barriers *>(smem + C::TILE_BYTES);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     volatile int *abort_flag = &bar->abort_flag;
+    const int npair = (nb + 1) / 2;              // items per head
 
     if (threadIdx.x == 0) {
-        mbar_init(&bar->q_full, 1);
-        mbar_init(&bar->q_empty, 1);
-        mbar_init(&bar->k_full, 1);
-        mbar_init(&bar->k_empty, 1);
-        mbar_init(&bar->v_full, 1);
-        mbar_init(&bar->v_empty, 1);
-        mbar_init(&bar->s_full, 1);
-        mbar_init(&bar->p_full, kSoftmaxWarps);
-        mbar_init(&bar->o_full, 1);
-        mbar_init(&bar->o_empty, kSoftmaxWarps);
-        mbar_init(&bar->pv_done, 1);
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&bar->sched_full[i], 1);
-            mbar_init(&bar->sched_empty[i], 1 + kSoftmaxWarps);
+        for (int s = 0; s < C::NST; ++s) {
+            mbar_init(&bar->ring_full[s], 1);
+            mbar_init(&bar->ring_empty[s], 1);
+        }
+        for (int x = 0; x < kSlots; ++x) {
+            mbar_init(&bar->q_full[x], 1);
+            mbar_init(&bar->q_empty[x], 1);
+            mbar_init(&bar->s_full[x], 1);
+            mbar_init(&bar->p_full[x], 4);
+            mbar_init(&bar->o_full[x], 1);
+            mbar_init(&bar->o_empty[x], 4);
+        }
+        for (int k = 0; k < 2; ++k) {
+            mbar_init(&bar->sched_full[k], 1);
+            mbar_init(&bar->sched_empty[k], 1 + 8);
         }
         mbar_init(&bar->drain, 1);
         bar->abort_flag = 0;
@@ -177,10 +233,11 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     // Q rows beyond the block (block size 64) are never loaded: keep them zero.
     if (BS < kRowsM) {
-        for (int kb = 0; kb < C::KBLK; ++kb) {
-            uint4 *z = reinterpret_cast<uint4 *>(sQ + kb * kRowsM * 128 + BS * 128);
-            for (int i = threadIdx.x; i < (kRowsM - BS) * 128 / 16; i += kThreads) z[i] = make_uint4(0, 0, 0, 0);
-        }
+        for (int x = 0; x < kSlots; ++x)
+            for (int kb = 0; kb < C::KBLK; ++kb) {
+                uint4 *z = reinterpret_cast<uint4 *>(sQ + x * C::Q_BYTES + kb * kRowsM * 128 + BS * 128);
+                for (int i = threadIdx.x; i < (kRowsM - BS) * 128 / 16; i += kThreads) z[i] = make_uint4(0, 0, 0, 0);
+            }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
     if (warp == kMmaWarp) {
@@ -198,127 +255,203 @@ __global__ void __launch_bounds__(kThreads, 2)
             prefetch_tensormap(&tmap_q);
             prefetch_tensormap(&tmap_k);
             prefetch_tensormap(&tmap_v);
-            uint32_t it = 0, kc = 0, vc = 0;
-            uint32_t q_armed = 0;
+            uint32_t it = 0, rc = 0;                  // items published, ring loads issued
+            uint32_t q_armed[kSlots] = {0, 0};        // Q loads issued per slot
+            uint32_t q_items[kSlots] = {0, 0};        // items with a Q tile per slot
             bool ok = true;
             while (ok) {
                 const int idx = atomicAdd(work_counter, 1);
-                const int row = (idx < n_items) ? order[idx] : -1;
-                int start = 0, count = 0;
-                if (row >= 0) {
-                    start = row_ptr[row];
-                    count = row_ptr[row + 1] - start;
-                    if (count < 0) {
-                        record_error(dev_status, FVATTN_ERR_BAD_CSR);
-                        count = 0;
+                const int p = (idx < n_items) ? order[idx] : -1;
+                int4 sx[kSlots] = {make_int4(-1, 0, 0, 0), make_int4(-1, 0, 0, 0)};
+                if (p >= 0) {
+                    const int bh = p / npair, i2 = p % npair;
+                    for (int x = 0; x < kSlots; ++x) {
+                        if (2 * i2 + x >= nb) continue;  // an odd last block has no partner
+                        const int rw = bh * nb + 2 * i2 + x;
+                        int c = row_ptr[rw + 1] - row_ptr[rw];
+                        if (c < 0) {
+                            record_error(dev_status, FVATTN_ERR_BAD_CSR);
+                            c = 0;
+                        }
+                        sx[x] = make_int4(rw, row_ptr[rw], c, 1);
                     }
                 }
-                const uint32_t slot = it & 1;
-                if (!mbar_wait(&bar->sched_empty[slot], ((it >> 1) & 1) ^ 1, abort_flag, dev_status)) break;
-                bar->sched_item[slot] = make_int4(row, start, count, row >= 0);
-                mbar_arrive(&bar->sched_full[slot]);
-                if (row < 0) break;
-                const int bh = row / nb;
-                const int qb = row % nb;
-                if (!mbar_wait(&bar->q_empty, (it & 1) ^ 1, abort_flag, dev_status)) break;
-                // Test hook: CTA 0 leaves the Q tile of its first item unloaded, so the
-                // MMA warp's bounded wait for it runs out (exercises the timeout path).
-                if (!(test_stall && blockIdx.x == 0 && it == 0)) {
-                    mbar_arrive_expect_tx(&bar->q_full, C::Q_LOAD_BYTES);
-                    for (int kb = 0; kb < C::KBLK; ++kb)
-                        tma_load_3d(sQ + kb * kRowsM * 128, &tmap_q, &bar->q_full, kb * 64, qb * BS, bh);
-                    q_armed = it + 1;
-                }
-                int prev = -1;
-                for (int j = 0; j < count && ok; ++j) {
-                    int kblk = col_idx[start + j];
-                    if (kblk < 0 || kblk >= nb || kblk <= prev) {
-                        record_error(dev_status, FVATTN_ERR_BAD_CSR);
-                        kblk = 0;  // load a valid tile; the softmax masks it out
-                    } else {
-                        prev = kblk;
+                const uint32_t k = it & 1;
+                if (!mbar_wait(&bar->sched_empty[k], ((it >> 1) & 1) ^ 1, abort_flag, dev_status)) break;
+                bar->sched_item[k][0] = sx[0];
+                bar->sched_item[k][1] = sx[1];
+                mbar_arrive(&bar->sched_full[k]);
+                if (p < 0) break;
+                const int bh = sx[0].x / nb;
+                // Q tiles of the rows that have key blocks
+                for (int x = 0; x < kSlots && ok; ++x) {
+                    if (sx[x].x < 0 || sx[x].z == 0) continue;
+                    if (!mbar_wait(&bar->q_empty[x], (q_items[x] & 1) ^ 1, abort_flag, dev_status)) {
+                        ok = false;
+                        break;
                     }
-                    if (!mbar_wait(&bar->k_empty, (kc & 1) ^ 1, abort_flag, dev_status)) { ok = false; break; }
-                    mbar_arrive_expect_tx(&bar->k_full, C::KV_BYTES);
+                    ++q_items[x];
+                    // Test hook: CTA 0 leaves its first Q tile unloaded, so the MMA warp's
+                    // bounded wait for it runs out (exercises the timeout path).
+                    if (test_stall && blockIdx.x == 0 && it == 0) continue;
+                    const int qb = sx[x].x % nb;
+                    mbar_arrive_expect_tx(&bar->q_full[x], C::Q_LOAD_BYTES);
                     for (int kb = 0; kb < C::KBLK; ++kb)
-                        tma_load_3d(sK + kb * BS * 128, &tmap_k, &bar->k_full, kb * 64, kblk * BS, bh);
-                    ++kc;
-                    if (!mbar_wait(&bar->v_empty, (vc & 1) ^ 1, abort_flag, dev_status)) { ok = false; break; }
-                    mbar_arrive_expect_tx(&bar->v_full, C::KV_BYTES);
-                    for (int kb = 0; kb < C::KBLK; ++kb)
-                        tma_load_3d(sV + kb * BS * 128, &tmap_v, &bar->v_full, kb * 64, kblk * BS, bh);
-                    ++vc;
+                        tma_load_3d(sQ + x * C::Q_BYTES + kb * kRowsM * 128, &tmap_q, &bar->q_full[x], kb * 64,
+                                    qb * BS, bh);
+                    q_armed[x] = q_items[x];
+                }
+                // K and V of every block of the union, in merge order
+                Merge mg;
+                mg.init(col_idx, sx[0], sx[1], nb);
+                while (ok && !mg.done()) {
+                    const Step s = mg.next();
+                    if (mg.bad) record_error(dev_status, FVATTN_ERR_BAD_CSR);
+                    for (int kv = 0; kv < 2 && ok; ++kv) {
+                        const uint32_t st = rc % C::NST;
+                        if (!mbar_wait(&bar->ring_empty[st], ((rc / C::NST) & 1) ^ 1, abort_flag, dev_status)) {
+                            ok = false;
+                            break;
+                        }
+                        mbar_arrive_expect_tx(&bar->ring_full[st], C::STAGE_BYTES);
+                        for (int kb = 0; kb < C::KBLK; ++kb)
+                            tma_load_3d(ring + st * C::STAGE_BYTES + kb * BS * 128, kv == 0 ? &tmap_k : &tmap_v,
+                                        &bar->ring_full[st], kb * 64, s.kblk * BS, bh);
+                        ++rc;
+                    }
                 }
                 ++it;
             }
-            // wait for every load this thread issued to land before the CTA exits
-            if (q_armed > 0) mbar_wait_teardown(&bar->q_full, (q_armed - 1) & 1);
-            if (kc > 0) mbar_wait_teardown(&bar->k_full, (kc - 1) & 1);
-            if (vc > 0) mbar_wait_teardown(&bar->v_full, (vc - 1) & 1);
+            // every load this thread issued lands before the CTA exits
+            for (uint32_t st = 0; st < static_cast<uint32_t>(C::NST); ++st) {
+                if (rc > st) {
+                    const uint32_t times = (rc - st + C::NST - 1) / C::NST;
+                    mbar_wait_teardown(&bar->ring_full[st], (times - 1) & 1);
+                }
+            }
+            for (int x = 0; x < kSlots; ++x)
+                if (q_armed[x] > 0) mbar_wait_teardown(&bar->q_full[x], (q_armed[x] - 1) & 1);
         }
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            const uint32_t tS = tmem + kTmemS;
-            const uint32_t tO = tmem + kTmemO;
-            const uint32_t q0 = smem_addr(sQ), k0 = smem_addr(sK), v0 = smem_addr(sV);
-            uint32_t it = 0, kc = 0, vc = 0, pc = 0;
-            uint32_t pv_issued = 0, pv_seen = 0;  // P lives in S's columns: S_{j+1} waits for PV_j
+            const uint32_t q0 = smem_addr(sQ), r0 = smem_addr(ring);
+            uint32_t it = 0, rc = 0;
+            uint32_t qn[kSlots] = {0, 0}, on[kSlots] = {0, 0}, pc[kSlots] = {0, 0};
             bool ok = true;
+            auto wait = [&](uint64_t *b, uint32_t parity) {
+                if (ok && !mbar_wait(b, parity, abort_flag, dev_status)) ok = false;
+                return ok;
+            };
+            // S_X = Q_X K^T from ring stage st
+            auto issue_s = [&](int x, uint32_t st) {
+                const uint32_t qa = q0 + x * C::Q_BYTES, kbase = r0 + st * C::STAGE_BYTES;
+                const uint32_t tS = tmem + x * kTmemSlot;
+#pragma unroll
+                for (int k = 0; k < D / 16; ++k) {
+                    const uint32_t kb = k >> 2, ko = (k & 3) * 32;
+                    const uint64_t da = smem_desc_sw128(qa + kb * kRowsM * 128 + ko, 16, 1024);
+                    const uint64_t db = smem_desc_sw128(kbase + kb * BS * 128 + ko, 16, 1024);
+                    mma_ss(tS, da, db, C::IDESC_S, k > 0 ? 1u : 0u);
+                }
+                mma_commit(&bar->s_full[x]);
+            };
+            // O_X (+)= P_X V from ring stage st
+            auto issue_pv = [&](int x, uint32_t st, bool first) {
+                const uint32_t vbase = r0 + st * C::STAGE_BYTES;
+                const uint32_t tS = tmem + x * kTmemSlot, tO = tS + kTmemO;
+#pragma unroll
+                for (int k = 0; k < BS / 16; ++k) {
+                    const uint64_t dv = smem_desc_sw128(vbase + k * 16 * 128, BS * 128, 1024);
+                    mma_ts(tO, tS + k * 8, dv, C::IDESC_PV, (!first || k > 0) ? 1u : 0u);
+                }
+            };
             while (ok) {
-                const uint32_t slot = it & 1;
-                if (!mbar_wait(&bar->sched_full[slot], (it >> 1) & 1, abort_flag, dev_status)) break;
-                const int4 item = bar->sched_item[slot];
-                mbar_arrive(&bar->sched_empty[slot]);
-                if (!item.w) break;
-                const int count = item.z;
-                if (!mbar_wait(&bar->q_full, it & 1, abort_flag, dev_status)) break;
-                for (int j = 0; j < count; ++j) {
-                    // S = Q K_j^T
-                    if (!mbar_wait(&bar->k_full, kc & 1, abort_flag, dev_status)) { ok = false; break; }
-                    if (kWaitPvBeforeS && pv_issued > pv_seen) {
-                        if (!mbar_wait(&bar->pv_done, pv_seen & 1, abort_flag, dev_status)) { ok = false; break; }
-                        pv_seen = pv_issued;
+                const uint32_t k = it & 1;
+                if (!wait(&bar->sched_full[k], (it >> 1) & 1)) break;
+                const int4 sx[kSlots] = {bar->sched_item[k][0], bar->sched_item[k][1]};
+                mbar_arrive(&bar->sched_empty[k]);
+                if (!sx[0].w) break;
+                bool q_wait[kSlots], first_pv[kSlots];
+                for (int x = 0; x < kSlots; ++x) {
+                    q_wait[x] = sx[x].x >= 0 && sx[x].z > 0;
+                    first_pv[x] = true;
+                    // a row without key blocks: only the O handshake with its warpgroup
+                    if (sx[x].x >= 0 && sx[x].z == 0 && wait(&bar->o_empty[x], (on[x] & 1) ^ 1)) {
+                        mma_commit(&bar->o_full[x]);
+                        ++on[x];
                     }
-                    tc_fence_after();
-#pragma unroll
-                    for (int k = 0; k < D / 16; ++k) {
-                        const uint32_t kb = k >> 2, ko = (k & 3) * 32;
-                        const uint64_t da = smem_desc_sw128(q0 + kb * kRowsM * 128 + ko, 16, 1024);
-                        const uint64_t db = smem_desc_sw128(k0 + kb * BS * 128 + ko, 16, 1024);
-                        mma_ss(tS, da, db, C::IDESC_S, k > 0 ? 1u : 0u);
+                }
+                Merge mg;
+                mg.init(col_idx, sx[0], sx[1], nb);
+                int b_pending = -1;  // ring stage of V for the B tile whose PV is still to issue
+                while (ok && !mg.done()) {
+                    const Step s = mg.next();
+                    const uint32_t kst = rc % C::NST, vst = (rc + 1) % C::NST;
+                    const uint32_t kph = (rc / C::NST) & 1, vph = ((rc + 1) / C::NST) & 1;
+                    rc += 2;
+                    if (!wait(&bar->ring_full[kst], kph)) break;
+                    if (s.pa) {
+                        if (q_wait[0]) {
+                            if (!wait(&bar->q_full[0], qn[0] & 1)) break;
+                            ++qn[0];
+                            q_wait[0] = false;
+                        }
+                        tc_fence_after();
+                        issue_s(0, kst);
                     }
-                    mma_commit(&bar->k_empty);
-                    if (j == count - 1) mma_commit(&bar->q_empty);
-                    mma_commit(&bar->s_full);
-                    ++kc;
-                    // O += P_j V_j once the softmax has written P_j (and rescaled O)
-                    if (!mbar_wait(&bar->p_full, pc & 1, abort_flag, dev_status)) { ok = false; break; }
-                    ++pc;
-                    if (j == 0 && !mbar_wait(&bar->o_empty, (it & 1) ^ 1, abort_flag, dev_status)) {
-                        ok = false;
-                        break;
+                    if (b_pending >= 0) {
+                        if (!wait(&bar->p_full[1], pc[1] & 1)) break;
+                        ++pc[1];
+                        if (first_pv[1] && !wait(&bar->o_empty[1], (on[1] & 1) ^ 1)) break;
+                        tc_fence_after();
+                        issue_pv(1, b_pending, first_pv[1]);
+                        first_pv[1] = false;
+                        mma_commit(&bar->ring_empty[b_pending]);
+                        b_pending = -1;
                     }
-                    if (!mbar_wait(&bar->v_full, vc & 1, abort_flag, dev_status)) { ok = false; break; }
-                    tc_fence_after();
-#pragma unroll
-                    for (int k = 0; k < BS / 16; ++k) {
-                        // keys [16k, 16k+16): P of column half h sits at h*BS/2, packed in pairs
-                        const uint32_t pcol = 8 * k + (k / (BS / 32)) * (BS / 4);
-                        const uint64_t dv = smem_desc_sw128(v0 + k * 16 * 128, BS * 128, 1024);
-                        mma_ts(tO, tS + pcol, dv, C::IDESC_PV, (j > 0 || k > 0) ? 1u : 0u);
+                    if (s.pb) {
+                        if (q_wait[1]) {
+                            if (!wait(&bar->q_full[1], qn[1] & 1)) break;
+                            ++qn[1];
+                            q_wait[1] = false;
+                        }
+                        tc_fence_after();
+                        issue_s(1, kst);
                     }
-                    mma_commit(&bar->v_empty);
-                    mma_commit(&bar->pv_done);
-                    ++pv_issued;
-                    ++vc;
+                    mma_commit(&bar->ring_empty[kst]);  // K read by every S above
+                    if (!wait(&bar->ring_full[vst], vph)) break;
+                    if (s.pa) {
+                        if (!wait(&bar->p_full[0], pc[0] & 1)) break;
+                        ++pc[0];
+                        if (first_pv[0] && !wait(&bar->o_empty[0], (on[0] & 1) ^ 1)) break;
+                        tc_fence_after();
+                        issue_pv(0, vst, first_pv[0]);
+                        first_pv[0] = false;
+                    }
+                    if (s.pb) {
+                        b_pending = static_cast<int>(vst);
+                    } else {
+                        mma_commit(&bar->ring_empty[vst]);
+                    }
+                }
+                if (ok && b_pending >= 0 && wait(&bar->p_full[1], pc[1] & 1)) {
+                    ++pc[1];
+                    if (!first_pv[1] || wait(&bar->o_empty[1], (on[1] & 1) ^ 1)) {
+                        tc_fence_after();
+                        issue_pv(1, b_pending, first_pv[1]);
+                        first_pv[1] = false;
+                        mma_commit(&bar->ring_empty[b_pending]);
+                    }
                 }
                 if (!ok) break;
-                if (count == 0) {
-                    mma_commit(&bar->q_empty);
-                    if (!mbar_wait(&bar->o_empty, (it & 1) ^ 1, abort_flag, dev_status)) break;
+                for (int x = 0; x < kSlots; ++x) {
+                    if (sx[x].x >= 0 && sx[x].z > 0) {
+                        mma_commit(&bar->q_empty[x]);
+                        mma_commit(&bar->o_full[x]);
+                        ++on[x];
+                    }
                 }
-                mma_commit(&bar->o_full);
                 ++it;
             }
             // every MMA issued by this thread completes before TMEM is released
@@ -327,30 +460,27 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
     } else {
         // ------------------------------------------------ softmax / epilogue
-        // warp w: rows 32*(w%4) .. +31 (its TMEM lane quarter), key columns of half
-        // h = w/4; the two warps of a lane group exchange their row maxima.
-        constexpr int HALF = BS / 2;               // S columns per warp
-        constexpr int OHALF = D / 2;               // O columns per warp
-        const int g = warp & 3, h = warp >> 2;
-        const int r = g * 32 + lane;                               // tile row = TMEM lane
-        const uint32_t lane_base = static_cast<uint32_t>(g * 32) << 16;
-        const uint32_t tS = tmem + kTmemS + lane_base + h * HALF;  // this warp's S columns; P goes
-                                                                   // to the first HALF/2 of them
-        const uint32_t tO = tmem + kTmemO + lane_base + h * OHALF;
-        float *xchg = reinterpret_cast<float *>(smem + C::TILE_BYTES + 256);  // [4][2][kRowsM]
-        uint32_t it = 0, sc = 0;
+        const int X = warp >> 2;                                   // slot of this warpgroup
+        const int r = threadIdx.x & (kRowsM - 1);                  // tile row = TMEM lane
+        const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        const uint32_t tS = tmem + X * kTmemSlot + lane_base;
+        const uint32_t tO = tS + kTmemO;
+        uint32_t it = 0, sc = 0, on = 0;
         while (true) {
-            const uint32_t slot = it & 1;
-            if (!mbar_wait(&bar->sched_full[slot], (it >> 1) & 1, abort_flag, dev_status)) break;
-            const int4 item = bar->sched_item[slot];
+            const uint32_t k = it & 1;
+            if (!mbar_wait(&bar->sched_full[k], (it >> 1) & 1, abort_flag, dev_status)) break;
+            const int4 item = bar->sched_item[k][X];
+            const bool valid_item = bar->sched_item[k][0].w != 0;
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bar->sched_empty[slot]);
-            if (!item.w) break;
+            if (lane == 0) mbar_arrive(&bar->sched_empty[k]);
+            ++it;
+            if (!valid_item) break;
+            if (item.x < 0) continue;                              // slot B of an odd last block
             const int row = item.x, start = item.y, count = item.z;
             const int64_t bh = row / nb;
             const int qb = row % nb;
             const int t_row = qb * BS + r;                         // token index of this thread's row
-            float m = -CUDART_INF_F, l = 0.0f;                     // l: this half's share of the row sum
+            float m = -CUDART_INF_F, l = 0.0f;
             int prev = -1;
             bool ok = true;
             for (int j = 0; j < count; ++j) {
@@ -358,49 +488,42 @@ __global__ void __launch_bounds__(kThreads, 2)
                 const bool valid = kblk >= 0 && kblk < nb && kblk > prev;
                 if (valid) prev = kblk;
                 const int key0 = kblk * BS;
-                // keys of this block that exist and are allowed for this row, counted
-                // from the start of this warp's column half
+                // keys of this block that exist and are allowed for this row
                 int lim = valid ? min(BS, N - key0) : 0;
                 if (causal) lim = min(lim, t_row - key0 + 1);
-                lim -= h * HALF;
-                if (!mbar_wait(&bar->s_full, sc & 1, abort_flag, dev_status)) { ok = false; break; }
+                if (!mbar_wait(&bar->s_full[X], sc & 1, abort_flag, dev_status)) { ok = false; break; }
                 ++sc;
                 tc_fence_after();
-                uint32_t v[HALF];
+                // the whole S row of this thread: BS fp32 values
+                uint32_t v[BS];
 #pragma unroll
-                for (int c0 = 0; c0 < HALF; c0 += 32)
-                    tmem_ld32(tS + c0, *reinterpret_cast<uint32_t(*)[32]>(&v[c0]));
+                for (int c0 = 0; c0 < BS; c0 += 32) tmem_ld32(tS + c0, *reinterpret_cast<uint32_t(*)[32]>(&v[c0]));
                 tmem_wait_ld();
-                if (lim < HALF) {  // ragged last block, causal diagonal, or a skipped index
+                if (lim < BS) {  // ragged last block, causal diagonal, or a skipped index
 #pragma unroll
-                    for (int c = 0; c < HALF; ++c)
+                    for (int c = 0; c < BS; ++c)
                         if (c >= lim) v[c] = __float_as_uint(-CUDART_INF_F);
                 }
                 float mq[4] = {-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F};
 #pragma unroll
-                for (int c = 0; c < HALF; c += 8) {
+                for (int c = 0; c < BS; c += 8) {
 #pragma unroll
                     for (int q = 0; q < 4; ++q)
                         mq[q] = max3f(mq[q], __uint_as_float(v[c + 2 * q]), __uint_as_float(v[c + 2 * q + 1]));
                 }
-                const float mine = max3f(mq[0], mq[1], fmaxf(mq[2], mq[3]));
-                float *xb = xchg + (j & 1) * 2 * kRowsM;
-                xb[h * kRowsM + r] = mine;
-                pair_sync(g);
-                const float mxs = fmaxf(mine, xb[(1 - h) * kRowsM + r]) * scale_log2;
+                const float mxs = max3f(mq[0], mq[1], fmaxf(mq[2], mq[3])) * scale_log2;
                 // The reference maximum only moves when the row maximum exceeds it by
                 // more than 2^8: P stays below 256 and the rescale of O is rare.  O and
-                // l always share the same reference, so the final O / l is exact.  Both
-                // warps of a row take the same decision from the same values.
+                // l always share the same reference, so the final O / l is exact.
                 const bool need = mxs > m + kRescaleLog2;
                 const float m_new = need ? mxs : m;
                 const float alpha = need ? ex2_approx(m - m_new) : 1.0f;
                 const float neg_m = (m_new == -CUDART_INF_F) ? 0.0f : -m_new;
                 float rs[4] = {0.0f, 0.0f, 0.0f, 0.0f};
                 // P packed as bf16 pairs in place: v[c/2] <- (p[c], p[c+1])
-                if (lim >= HALF) {
+                if (lim >= BS) {
 #pragma unroll
-                    for (int c = 0; c < HALF; c += 2) {
+                    for (int c = 0; c < BS; c += 2) {
                         const float x0 = fmaf(__uint_as_float(v[c]), scale_log2, neg_m);
                         const float x1 = fmaf(__uint_as_float(v[c + 1]), scale_log2, neg_m);
                         const float p0 = ((c & 7) >= 8 - kPolyOf8) ? ex2_poly(x0) : ex2_approx(x0);
@@ -410,26 +533,22 @@ __global__ void __launch_bounds__(kThreads, 2)
                     }
                 } else {
 #pragma unroll
-                    for (int c = 0; c < HALF; c += 2) {
+                    for (int c = 0; c < BS; c += 2) {
                         const float p0 = ex2_approx(fmaf(__uint_as_float(v[c]), scale_log2, neg_m));
                         const float p1 = ex2_approx(fmaf(__uint_as_float(v[c + 1]), scale_log2, neg_m));
                         rs[(c >> 1) & 3] += p0 + p1;
                         v[c >> 1] = pack_bf16(p0, p1);
                     }
                 }
-                if constexpr (HALF / 2 >= 32) {
 #pragma unroll
-                    for (int c0 = 0; c0 < HALF / 2; c0 += 32)
-                        tmem_st32(tS + c0, *reinterpret_cast<const uint32_t(*)[32]>(&v[c0]));
-                } else {
-                    tmem_st16(tS, *reinterpret_cast<const uint32_t(*)[16]>(&v[0]));
-                }
+                for (int c0 = 0; c0 < BS / 2; c0 += 32)
+                    tmem_st32(tS + c0, *reinterpret_cast<const uint32_t(*)[32]>(&v[c0]));
                 l = l * alpha + ((rs[0] + rs[1]) + (rs[2] + rs[3]));
-                // rescale this warp's half of the running output (PV_{j-1} has completed:
-                // the S_j commit tracks every earlier MMA of this CTA)
+                // rescale the running output (this slot's previous PV has completed: it
+                // was issued before this S, and the S commit tracks every earlier MMA)
                 if (__any_sync(0xffffffffu, need && j > 0)) {
 #pragma unroll
-                    for (int c0 = 0; c0 < OHALF; c0 += 32) {
+                    for (int c0 = 0; c0 < D; c0 += 32) {
                         uint32_t o[32];
                         tmem_ld32(tO + c0, o);
                         tmem_wait_ld();
@@ -441,22 +560,19 @@ __global__ void __launch_bounds__(kThreads, 2)
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&bar->p_full);
+                if (lane == 0) mbar_arrive(&bar->p_full[X]);
                 m = m_new;
             }
             if (!ok) break;
-            // epilogue: row sum = both halves' shares
-            float *xl = xchg + (2 + (it & 1)) * 2 * kRowsM;
-            xl[h * kRowsM + r] = l;
-            pair_sync(g);
-            const float lsum = l + xl[(1 - h) * kRowsM + r];
-            if (!mbar_wait(&bar->o_full, it & 1, abort_flag, dev_status)) break;
+            // epilogue
+            if (!mbar_wait(&bar->o_full[X], on & 1, abort_flag, dev_status)) break;
+            ++on;
             tc_fence_after();
             const bool row_ok = r < BS && t_row < N;
-            const float inv_l = (lsum > 0.0f) ? 1.0f / lsum : 0.0f;
-            __nv_bfloat16 *orow = O + (bh * N + t_row) * D + h * OHALF;
+            const float inv_l = (l > 0.0f) ? 1.0f / l : 0.0f;
+            __nv_bfloat16 *orow = O + (bh * N + t_row) * D;
 #pragma unroll
-            for (int c0 = 0; c0 < OHALF; c0 += 32) {
+            for (int c0 = 0; c0 < D; c0 += 32) {
                 uint32_t v[32];
                 if (count > 0) {
                     tmem_ld32(tO + c0, v);
@@ -475,12 +591,10 @@ __global__ void __launch_bounds__(kThreads, 2)
                     for (int q = 0; q < 4; ++q) dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
                 }
             }
-            if (row_ok && h == 0)
-                LSE[bh * N + t_row] = (lsum > 0.0f) ? (m + __log2f(lsum)) * 0.69314718055994531f : -CUDART_INF_F;
+            if (row_ok) LSE[bh * N + t_row] = (l > 0.0f) ? (m + __log2f(l)) * 0.69314718055994531f : -CUDART_INF_F;
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bar->o_empty);
-            ++it;
+            if (lane == 0) mbar_arrive(&bar->o_empty[X]);
         }
     }
 
@@ -488,6 +602,17 @@ __global__ void __launch_bounds__(kThreads, 2)
     __syncthreads();
     tc_fence_after();
     if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
+}
+
+// pair_row_ptr[p] = row_ptr[first row of pair p]; the last entry closes the list.
+__global__ void pair_row_ptr_kernel(const int32_t *__restrict__ row_ptr, int64_t BH, int nb,
+                                    int32_t *__restrict__ pair_row_ptr) {
+    const int npair = (nb + 1) / 2;
+    const int64_t n = BH * npair;
+    for (int64_t p = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; p <= n;
+         p += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        pair_row_ptr[p] = (p == n) ? row_ptr[BH * nb] : row_ptr[(p / npair) * nb + 2 * (p % npair)];
+    }
 }
 
 }  // namespace
@@ -499,6 +624,18 @@ int attn_smem_bytes(int d, int bs) {
     if (d == 128 && bs == 64) return Cfg<128, 64>::SMEM_BYTES;
     if (d == 64 && bs == 128) return Cfg<64, 128>::SMEM_BYTES;
     return Cfg<64, 64>::SMEM_BYTES;
+}
+
+int attn_ctas_per_sm() { return 1; }
+
+int64_t attn_num_items(int64_t BH, int nb) { return BH * ((nb + 1) / 2); }
+
+cudaError_t launch_pair_row_ptr(const int32_t *row_ptr, int64_t BH, int nb, int32_t *pair_row_ptr,
+                                cudaStream_t stream) {
+    const int64_t n = attn_num_items(BH, nb) + 1;
+    const int grid = static_cast<int>(n / 256 + 1 < 1024 ? n / 256 + 1 : 1024);
+    pair_row_ptr_kernel<<<grid, 256, 0, stream>>>(row_ptr, BH, nb, pair_row_ptr);
+    return cudaGetLastError();
 }
 
 template <int D, int BS>
@@ -520,4 +657,3 @@ cudaError_t launch_sparse_attn(const AttnLaunch &a, int d, int bs, cudaStream_t 
 }
 
 }  // namespace fvattn
-namespace fvattn { int attn_ctas_per_sm() { return 2; } }

@@ -9,7 +9,7 @@ namespace fvattn {
 
 struct AttnLaunch {
     const CUtensorMap *tmap_q, *tmap_k, *tmap_v;  // host copies, passed by value as kernel parameters
-    const int32_t *row_ptr, *col_idx, *order;
+    const int32_t *row_ptr, *col_idx, *order;  // order: work items (query-block pairs), longest first
     int n_items;
     int *work_counter;  // zeroed before the launch
     int N, nb, causal;
@@ -22,6 +22,11 @@ struct AttnLaunch {
 };
 
 int attn_smem_bytes(int d, int bs);
+// Work items of the attention kernel: pairs of neighbouring query blocks per head.
+int64_t attn_num_items(int64_t BH, int nb);
+// pair_row_ptr[p] = row_ptr[first row of item p], plus the closing entry.
+cudaError_t launch_pair_row_ptr(const int32_t *row_ptr, int64_t BH, int nb, int32_t *pair_row_ptr,
+                                cudaStream_t stream);
 int attn_ctas_per_sm();  // resident CTAs per SM the launch grid is sized for
 cudaError_t launch_sparse_attn(const AttnLaunch &a, int d, int bs, cudaStream_t stream);
 
