@@ -34,7 +34,7 @@ METRIC = "effective TFLOP/s & tensor-pipe % of peak (sparse attn fwd, p=0.9); ro
 UNIT = "TFLOP/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 ROUTE_KERNELS_PER_CALL = 4      # pool, select, CSR scan, CSR scatter
-FWD_KERNELS_PER_CALL = 4        # LPT rank, LPT offsets, LPT scatter, attention
+FWD_KERNELS_PER_CALL = 5        # item list, LPT rank, LPT offsets, LPT scatter, attention
 
 
 def load_peaks():
