@@ -46,6 +46,40 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+KERNEL_SOURCES = ("top_routed_block_b200/csrc/attn_fwd.cu", "top_routed_block_b200/csrc/ptx_sm100.cuh",
+                  "top_routed_block_b200/csrc/common.cuh")
+TRAFFIC_SUMMARY = "profiles/dram_traffic_video_dit.md"
+
+
+def kernel_source_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per attention launch from the committed ncu summary, if it was
+    taken on this workload with the current kernel source; else None."""
+    p = os.path.join(ROOT, TRAFFIC_SUMMARY)
+    if not os.path.exists(p):
+        return None
+    fields = {}
+    with open(p) as f:
+        for line in f:
+            if ":" in line and line.strip().startswith("- "):
+                k, v = line.strip()[2:].split(":", 1)
+                fields[k.strip()] = v.strip().strip("`")
+    if fields.get("workload") != workload or fields.get("kernel_source_sha256") != kernel_source_hash():
+        return None
+    try:
+        return float(fields["traffic_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
 def eff_flops(nnz: int, w: W.Workload) -> float:
     return 4.0 * w.bs * w.bs * w.d * float(nnz)
 
@@ -329,7 +363,7 @@ def run_ours(args, w, rank, world, local):
         "route_frac": r_ms / (r_ms + attn_ms),
         "tensor_frac_of_burst_peak": attn_tflops / burst,
         "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peak, "unit": "TFLOP/s",
-                     "frac": attn_tflops / peak, "traffic": None,
+                     "frac": attn_tflops / peak, "traffic": recorded_traffic(w.name),
                      "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside back-to-back steps)",
                      "note": "achieved = 4*block^2*d*nnz / mean CUDA-event time of the fvattn_sparse_fwd call "
                              "(its 3 small ordering kernels included)"},

@@ -147,9 +147,13 @@ FVATTN_API int fvattn_lpt_order(const int32_t *row_ptr, int64_t rows, int max_co
  *   O           out, bf16 [B,H,N,d].   LSE  out, fp32 [B,H,N].
  *   workspace   >= fvattn_fwd_workspace_bytes(B,H,N,block).
  * Matmuls run on the tensor cores in bf16 with fp32 accumulation; softmax in
- * fp32.  Rows are processed longest-first (fvattn_lpt_order) by a persistent
- * grid.  Out-of-range or non-ascending column indices are skipped and set
- * *dev_status = FVATTN_ERR_BAD_CSR.
+ * fp32.  A persistent grid takes work items (pairs of neighbouring query
+ * blocks of one head) from a queue ordered head-major and longest-first: heads
+ * by total selected blocks descending, the items of a head by block count
+ * descending (ties by lower index), so that the SMs share one head's K and V
+ * in L2 at a time and finish on the shortest items.  B*H <= 4096, else
+ * FVATTN_ERR_UNSUPPORTED.  Out-of-range or non-ascending column indices are
+ * skipped and set *dev_status = FVATTN_ERR_BAD_CSR.
  */
 FVATTN_API int fvattn_sparse_fwd(const void *Q, const void *K, const void *V, const int32_t *row_ptr,
                       const int32_t *col_idx, int B, int H, int N, int d, int block, int causal, void *O,
@@ -164,8 +168,13 @@ FVATTN_API int fvattn_sparse_fwd(const void *Q, const void *K, const void *V, co
  *   hQ, hK, hV    host bf16 [B,H,N,d];  hO host bf16 [B,H,N,d];  hLSE host fp32 [B,H,N].
  *   dQ, dK, dV, dO, dLSE, row_ptr, col_idx (capacity col_capacity), head_counts,
  *   route_ws (route_ws_bytes), fwd_ws (fwd_ws_bytes): device buffers as for
- *   fvattn_route / fvattn_sparse_fwd.  dev_status: device int32[2] (routing
- *   status, then attention status).
+ *   fvattn_route / fvattn_sparse_fwd.  dev_status: device int32[3] (scratch for
+ *   routing and attention, then the first error over the whole call).
+ * The heads are processed in chunks of about 64 MB per tensor: the copies in of
+ * one chunk, the compute of the previous one (on `stream`) and the copies out of
+ * the one before run concurrently, on two streams the call creates and destroys
+ * (host buffers must be pinned for the copies to overlap).  Work already queued
+ * on `stream` completes before the first copy starts.
  * Returns the first host error, else the first nonzero device status read
  * after the sync.
  */
@@ -192,7 +201,7 @@ FVATTN_API int fvattn_attention_host(const void *hQ, const void *hK, const void 
  * file-scope device array of FVATTN_NOALLOC_SCRATCH_BYTES (4 MiB) inside the
  * library, which every device that loads the library keeps until the process
  * exits.  Shapes that need more return FVATTN_ERR_CAPACITY without launching
- * anything (about 500k rows B*H*ceil(N/block) at most).
+ * anything (about 2M rows B*H*ceil(N/block) at most).
  *
  * The first call on each device looks up the array's device address
  * (cudaGetSymbolAddress, with that device current) and caches it; make that first

@@ -164,3 +164,27 @@ def test_bad_csr_is_reported_and_the_rest_is_computed(oracle_mod):
     # the context is still healthy
     O2, LSE2 = run_fwd(dQ, dK, dV, good_rp, good_ci, w.bs, False)
     compare_attention(O2, LSE2, Oref, Lref, tokens, w.d, "after-badcsr")
+
+
+def test_host_buffer_path_matches_device_path():
+    """fvattn_attention_host (chunked copies in, routing, attention, copies out)
+    returns exactly what the device entry points return: heads are independent."""
+    import top_routed_block_b200 as fv
+    w = W.Workload("host_path", B=2, H=12, N=2000, d=128, bs=128, p=0.8, dist="structured", grid=(5, 20, 20),
+                   head_scale=("uniform", 0.5, 4.0), seed=44)
+    Q, K, V = W.generate(w)
+    dQ, dK, dV = to_dev(Q), to_dev(K), to_dev(V)
+    plan = fv.FvattnPlan(w.B, w.H, w.N, w.d, w.bs)
+    O_dev, L_dev, _ = plan(dQ, dK, dV, w.p)
+    plan.check()
+    O_dev, L_dev = O_dev.clone(), L_dev.clone()
+    pin = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory()
+    hQ, hK, hV = pin(Q), pin(K), pin(V)
+    hO = torch.empty((w.B, w.H, w.N, w.d), dtype=torch.bfloat16).pin_memory()
+    hL = torch.empty((w.B, w.H, w.N), dtype=torch.float32).pin_memory()
+    for _ in range(2):
+        hO.fill_(float("nan"))
+        fv.fvattn_attention_host(hQ, hK, hV, w.p, w.bs, False, plan=plan, dQ=torch.empty_like(dQ),
+                                 dK=torch.empty_like(dK), dV=torch.empty_like(dV), hO=hO, hLSE=hL)
+        assert torch.equal(hO, O_dev.cpu())
+        assert torch.equal(hL, L_dev.cpu())

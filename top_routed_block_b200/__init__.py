@@ -247,7 +247,7 @@ class FvattnPlan:
         self.fwd_ws = _empty_bytes(fvattn_fwd_workspace_bytes(B, H, N, block), dev)
         self.O = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev)
         self.LSE = torch.empty((B, H, N), dtype=torch.float32, device=dev)
-        self.status = torch.zeros(2, dtype=torch.int32, device=dev)
+        self.status = torch.zeros(3, dtype=torch.int32, device=dev)   # route, attention, first error (host path)
 
     def run_route(self, Q, K, p, stream=None) -> RouteResult:
         return fvattn_route(Q, K, p, self.block, stream=stream, out=self.route, workspace=self.route_ws)
@@ -264,7 +264,7 @@ class FvattnPlan:
 
     def check(self):
         self.status[0:1].copy_(self.route.dev_status)
-        check_status(self.status, "fvattn")
+        check_status(self.status[:2], "fvattn")
 
 
 def fvattn_attention_host(hQ: torch.Tensor, hK: torch.Tensor, hV: torch.Tensor, p: float, block: int,

@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -96,22 +97,26 @@ bool make_map(CUtensorMap *m, const void *base, int64_t BH, int N, int d, int ro
 }
 
 struct FwdWorkspace {
-    size_t order, item_ptr, counter, lpt, total;
+    size_t order, head_rank, counter, total;
 };
 
-// items: work items of the attention kernel; max_count: largest blocks per item.
-FwdWorkspace fwd_layout(int64_t items, int max_count) {
+// items: work items of the attention kernel; BH: heads.
+FwdWorkspace fwd_layout(int64_t items, int64_t BH) {
     FwdWorkspace w{};
     Carver c;
     w.order = c.take<int32_t>(static_cast<size_t>(items));
-    w.item_ptr = c.take<int32_t>(static_cast<size_t>(items) + 1);
+    w.head_rank = c.take<int32_t>(static_cast<size_t>(BH));
     w.counter = c.take<int32_t>(64);
-    w.lpt = align_up(c.off, 256);
-    w.total = w.lpt + lpt_workspace_layout(items, max_count).total;
+    w.total = align_up(c.off, 256);
     return w;
 }
 
 int from_cuda(cudaError_t e) { return e == cudaSuccess ? FVATTN_OK : FVATTN_ERR_CUDA; }
+
+// st[2] keeps the first error of st[0] (routing) and st[1] (attention) over successive calls.
+__global__ void status_merge_kernel(int32_t *st) {
+    if (st[2] == 0) st[2] = st[0] != 0 ? st[0] : st[1];
+}
 
 }  // namespace
 
@@ -159,8 +164,9 @@ size_t fvattn_fwd_workspace_bytes(int B, int H, int N, int block) {
     if (B < 1 || H < 1 || N < 1 || (block != 64 && block != 128)) return 0;
     const int64_t nb = ceil_div(N, block);
     if (nb > kMaxCount) return 0;
-    return fwd_layout(attn_num_items(static_cast<int64_t>(B) * H, static_cast<int>(nb)), 2 * static_cast<int>(nb))
-        .total;
+    const int64_t BH = static_cast<int64_t>(B) * H;
+    if (BH > kMaxHeads) return 0;
+    return fwd_layout(attn_num_items(BH, static_cast<int>(nb)), BH).total;
 }
 
 int fvattn_route(const void *Q, const void *K, int B, int H, int N, int d, int block, double p, int32_t *row_ptr,
@@ -220,11 +226,12 @@ static int sparse_fwd_impl(const void *Q, const void *K, const void *V, const in
     const int64_t BH = static_cast<int64_t>(B) * H;
     const int nb = static_cast<int>(ceil_div(N, block));
     const int64_t rows = BH * nb;
+    if (BH > kMaxHeads) return FVATTN_ERR_UNSUPPORTED;
     const int64_t items = attn_num_items(BH, nb);
-    const FwdWorkspace w = fwd_layout(items, 2 * nb);
+    const FwdWorkspace w = fwd_layout(items, BH);
     char *ws = static_cast<char *>(workspace);
     int32_t *order = reinterpret_cast<int32_t *>(ws + w.order);
-    int32_t *item_ptr = reinterpret_cast<int32_t *>(ws + w.item_ptr);
+    int32_t *head_rank = reinterpret_cast<int32_t *>(ws + w.head_rank);
     int *counter = reinterpret_cast<int *>(ws + w.counter);
 
     CUtensorMap mq, mk, mv;
@@ -234,11 +241,8 @@ static int sparse_fwd_impl(const void *Q, const void *K, const void *V, const in
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if ((rc = from_cuda(cudaMemsetAsync(dev_status, 0, sizeof(int32_t), s))) != FVATTN_OK) return rc;
-    // work items (pairs of neighbouring query blocks) longest first
-    if ((rc = from_cuda(launch_pair_row_ptr(row_ptr, BH, nb, item_ptr, s))) != FVATTN_OK) return rc;
-    if ((rc = from_cuda(launch_lpt_order(item_ptr, items, 2 * nb, order, ws + w.lpt, dev_status, s))) !=
-        FVATTN_OK)
-        return rc;
+    // work items (pairs of neighbouring query blocks): head-major, longest first
+    if ((rc = from_cuda(launch_item_order(row_ptr, BH, nb, head_rank, order, s))) != FVATTN_OK) return rc;
     if ((rc = from_cuda(cudaMemsetAsync(counter, 0, sizeof(int), s))) != FVATTN_OK) return rc;
 
     AttnLaunch a{};
@@ -285,30 +289,74 @@ int fvattn_attention_host(const void *hQ, const void *hK, const void *hV, int B,
                           size_t fwd_ws_bytes, int32_t *dev_status, fvattn_stream_t stream) {
     int rc = check_shape(B, H, N, d, block);
     if (rc != FVATTN_OK) return rc;
-    if (!hQ || !hK || !hV || !hO || !hLSE) return FVATTN_ERR_INVALID_ARG;
+    if (!hQ || !hK || !hV || !hO || !hLSE || !dQ || !dK || !dV || !dO || !dLSE || !dev_status)
+        return FVATTN_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(dev_status) & 3u) return FVATTN_ERR_ALIGNMENT;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    const size_t bytes = static_cast<size_t>(B) * H * N * d * 2;
-    const size_t lse_bytes = static_cast<size_t>(B) * H * N * sizeof(float);
-    if (!dQ || !dK || !dV || !dO || !dLSE) return FVATTN_ERR_INVALID_ARG;
-    if ((rc = from_cuda(cudaMemcpyAsync(dQ, hQ, bytes, cudaMemcpyHostToDevice, s))) != FVATTN_OK) return rc;
-    if ((rc = from_cuda(cudaMemcpyAsync(dK, hK, bytes, cudaMemcpyHostToDevice, s))) != FVATTN_OK) return rc;
-    if ((rc = from_cuda(cudaMemcpyAsync(dV, hV, bytes, cudaMemcpyHostToDevice, s))) != FVATTN_OK) return rc;
-    rc = fvattn_route(dQ, dK, B, H, N, d, block, p, row_ptr, col_idx, col_capacity, head_counts, route_ws,
-                      route_ws_bytes, dev_status, stream);
+    const int64_t BH = static_cast<int64_t>(B) * H;
+    const size_t head_bytes = static_cast<size_t>(N) * d * 2;
+    // Heads are independent for routing and attention: split B*H into chunks of about
+    // 64 MB per tensor so that copies in, compute and copies out of different chunks
+    // overlap (two extra streams for the copies, the caller's stream for compute).
+    const int64_t hc = std::max<int64_t>(1, std::min<int64_t>(BH, (64ll << 20) / static_cast<int64_t>(head_bytes)));
+    cudaStream_t s_in = nullptr, s_out = nullptr;
+    cudaEvent_t ev_in = nullptr, ev_out = nullptr;
+    auto cleanup = [&]() {
+        if (ev_in) cudaEventDestroy(ev_in);
+        if (ev_out) cudaEventDestroy(ev_out);
+        if (s_in) cudaStreamDestroy(s_in);
+        if (s_out) cudaStreamDestroy(s_out);
+    };
+    if (cudaStreamCreateWithFlags(&s_in, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&s_out, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ev_in, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ev_out, cudaEventDisableTiming) != cudaSuccess) {
+        cleanup();
+        return FVATTN_ERR_CUDA;
+    }
+    // dev_status: [0] routing of the current chunk, [1] attention of the current chunk,
+    // [2] first error over all chunks.  The copy streams start after everything already
+    // queued on the caller's stream.
+    rc = from_cuda(cudaMemsetAsync(dev_status + 2, 0, sizeof(int32_t), s));
+    if (rc == FVATTN_OK) rc = from_cuda(cudaEventRecord(ev_out, s));
+    if (rc == FVATTN_OK) rc = from_cuda(cudaStreamWaitEvent(s_in, ev_out, 0));
+    for (int64_t off = 0; off < BH && rc == FVATTN_OK; off += hc) {
+        const int hn = static_cast<int>(std::min<int64_t>(hc, BH - off));
+        const size_t o = static_cast<size_t>(off) * head_bytes, nbytes = static_cast<size_t>(hn) * head_bytes;
+        const size_t lo = static_cast<size_t>(off) * N * sizeof(float), lbytes = static_cast<size_t>(hn) * N * sizeof(float);
+        auto dptr = [&](void *base) { return static_cast<char *>(base) + o; };
+        auto hptr = [&](const void *base) { return static_cast<const char *>(base) + o; };
+        if ((rc = from_cuda(cudaMemcpyAsync(dptr(dQ), hptr(hQ), nbytes, cudaMemcpyHostToDevice, s_in))) ||
+            (rc = from_cuda(cudaMemcpyAsync(dptr(dK), hptr(hK), nbytes, cudaMemcpyHostToDevice, s_in))) ||
+            (rc = from_cuda(cudaMemcpyAsync(dptr(dV), hptr(hV), nbytes, cudaMemcpyHostToDevice, s_in))) ||
+            (rc = from_cuda(cudaEventRecord(ev_in, s_in))) || (rc = from_cuda(cudaStreamWaitEvent(s, ev_in, 0))))
+            break;
+        rc = fvattn_route(dptr(dQ), dptr(dK), 1, hn, N, d, block, p, row_ptr, col_idx, col_capacity,
+                          head_counts + off, route_ws, route_ws_bytes, dev_status, stream);
+        if (rc != FVATTN_OK) break;
+        rc = fvattn_sparse_fwd(dptr(dQ), dptr(dK), dptr(dV), row_ptr, col_idx, 1, hn, N, d, block, causal,
+                               dptr(dO), reinterpret_cast<float *>(reinterpret_cast<char *>(dLSE) + lo), fwd_ws,
+                               fwd_ws_bytes, dev_status + 1, stream);
+        if (rc != FVATTN_OK) break;
+        status_merge_kernel<<<1, 1, 0, s>>>(dev_status);
+        if ((rc = from_cuda(cudaGetLastError())) || (rc = from_cuda(cudaEventRecord(ev_out, s))) ||
+            (rc = from_cuda(cudaStreamWaitEvent(s_out, ev_out, 0))) ||
+            (rc = from_cuda(cudaMemcpyAsync(static_cast<char *>(hO) + o, dptr(dO), nbytes, cudaMemcpyDeviceToHost,
+                                            s_out))) ||
+            (rc = from_cuda(cudaMemcpyAsync(reinterpret_cast<char *>(hLSE) + lo,
+                                            reinterpret_cast<char *>(dLSE) + lo, lbytes, cudaMemcpyDeviceToHost,
+                                            s_out))))
+            break;
+    }
+    int32_t st = 0;
+    if (rc == FVATTN_OK) rc = from_cuda(cudaMemcpyAsync(&st, dev_status + 2, sizeof(st), cudaMemcpyDeviceToHost, s));
+    const int rs1 = from_cuda(cudaStreamSynchronize(s_in));
+    const int rs2 = from_cuda(cudaStreamSynchronize(s_out));
+    const int rs3 = from_cuda(cudaStreamSynchronize(s));
+    cleanup();
     if (rc != FVATTN_OK) return rc;
-    // the routing status is kept: fvattn_sparse_fwd must not clear a routing error
-    int32_t *fwd_status = dev_status + 1;
-    if ((reinterpret_cast<uintptr_t>(fwd_status) & 3u) != 0) return FVATTN_ERR_ALIGNMENT;
-    rc = fvattn_sparse_fwd(dQ, dK, dV, row_ptr, col_idx, B, H, N, d, block, causal, dO, dLSE, fwd_ws, fwd_ws_bytes,
-                           fwd_status, stream);
-    if (rc != FVATTN_OK) return rc;
-    if ((rc = from_cuda(cudaMemcpyAsync(hO, dO, bytes, cudaMemcpyDeviceToHost, s))) != FVATTN_OK) return rc;
-    if ((rc = from_cuda(cudaMemcpyAsync(hLSE, dLSE, lse_bytes, cudaMemcpyDeviceToHost, s))) != FVATTN_OK) return rc;
-    int32_t st[2] = {0, 0};
-    if ((rc = from_cuda(cudaMemcpyAsync(st, dev_status, sizeof(st), cudaMemcpyDeviceToHost, s))) != FVATTN_OK)
-        return rc;
-    if ((rc = from_cuda(cudaStreamSynchronize(s))) != FVATTN_OK) return rc;
-    return st[0] != 0 ? st[0] : st[1];
+    if (rs1 != FVATTN_OK || rs2 != FVATTN_OK || rs3 != FVATTN_OK) return FVATTN_ERR_CUDA;
+    return st;
 }
 
 }  // extern "C"

@@ -604,15 +604,77 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
 }
 
-// pair_row_ptr[p] = row_ptr[first row of pair p]; the last entry closes the list.
-__global__ void pair_row_ptr_kernel(const int32_t *__restrict__ row_ptr, int64_t BH, int nb,
-                                    int32_t *__restrict__ pair_row_ptr) {
-    const int npair = (nb + 1) / 2;
-    const int64_t n = BH * npair;
-    for (int64_t p = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; p <= n;
-         p += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        pair_row_ptr[p] = (p == n) ? row_ptr[BH * nb] : row_ptr[(p / npair) * nb + 2 * (p % npair)];
+// ------------------------------------------------------------- work order
+// Items are ordered head-major, longest first: heads by their total selected
+// blocks (descending, equal totals by head index), and inside a head the items
+// by their block count (descending, equal counts by item index).  All SMs then
+// work on about one head at a time, whose K and V stay in L2, and the grid ends
+// on the lightest head's shortest items.
+
+constexpr int kOrderThreads = 1024;
+
+// "x comes after y": key descending, index ascending.
+__device__ __forceinline__ bool later(int kx, int ix, int ky, int iy) { return kx < ky || (kx == ky && ix > iy); }
+
+// Sorts n <= 2 * kOrderThreads * reps (key, index) pairs in shared memory, padded to np2.
+__device__ void bitonic_sort(int *key, int *idx, int np2) {
+    for (int k = 2; k <= np2; k <<= 1) {
+        for (int jj = k >> 1; jj > 0; jj >>= 1) {
+            for (int e = threadIdx.x; e < (np2 >> 1); e += blockDim.x) {
+                const int a = (e / jj) * 2 * jj + (e % jj), b = a + jj;
+                const bool up = (a & k) == 0;
+                const bool swap = up ? later(key[a], idx[a], key[b], idx[b]) : later(key[b], idx[b], key[a], idx[a]);
+                if (swap) {
+                    const int tk = key[a], ti = idx[a];
+                    key[a] = key[b];
+                    idx[a] = idx[b];
+                    key[b] = tk;
+                    idx[b] = ti;
+                }
+            }
+            __syncthreads();
+        }
     }
+}
+
+// One CTA: head_rank[h] = position of head h in the order of head totals.
+__global__ void __launch_bounds__(kOrderThreads) head_rank_kernel(const int32_t *__restrict__ row_ptr, int BH, int nb,
+                                                                  int np2, int32_t *__restrict__ head_rank) {
+    extern __shared__ int sm_order[];
+    int *key = sm_order, *idx = sm_order + np2;
+    for (int e = threadIdx.x; e < np2; e += blockDim.x) {
+        key[e] = e < BH ? row_ptr[static_cast<int64_t>(e + 1) * nb] - row_ptr[static_cast<int64_t>(e) * nb] : -1;
+        idx[e] = e < BH ? e : 0x7fffffff;
+    }
+    __syncthreads();
+    bitonic_sort(key, idx, np2);
+    for (int e = threadIdx.x; e < BH; e += blockDim.x) head_rank[idx[e]] = e;
+}
+
+// One CTA per head: its items sorted by block count, written at head_rank[h] * npair.
+__global__ void __launch_bounds__(kOrderThreads) item_order_kernel(const int32_t *__restrict__ row_ptr, int nb,
+                                                                   int np2, const int32_t *__restrict__ head_rank,
+                                                                   int32_t *__restrict__ order) {
+    extern __shared__ int sm_order[];
+    int *key = sm_order, *idx = sm_order + np2;
+    const int npair = (nb + 1) / 2;
+    const int64_t bh = blockIdx.x;
+    for (int e = threadIdx.x; e < np2; e += blockDim.x) {
+        if (e < npair) {
+            const int64_t r = bh * nb + 2 * e;
+            const int64_t r_end = (2 * e + 2 <= nb) ? r + 2 : r + 1;
+            key[e] = row_ptr[r_end] - row_ptr[r];
+            idx[e] = e;
+        } else {
+            key[e] = -1;
+            idx[e] = 0x7fffffff;
+        }
+    }
+    __syncthreads();
+    bitonic_sort(key, idx, np2);
+    const int64_t base = static_cast<int64_t>(head_rank[bh]) * npair;
+    for (int e = threadIdx.x; e < npair; e += blockDim.x)
+        order[base + e] = static_cast<int32_t>(bh * npair + idx[e]);
 }
 
 }  // namespace
@@ -630,11 +692,20 @@ int attn_ctas_per_sm() { return 1; }
 
 int64_t attn_num_items(int64_t BH, int nb) { return BH * ((nb + 1) / 2); }
 
-cudaError_t launch_pair_row_ptr(const int32_t *row_ptr, int64_t BH, int nb, int32_t *pair_row_ptr,
-                                cudaStream_t stream) {
-    const int64_t n = attn_num_items(BH, nb) + 1;
-    const int grid = static_cast<int>(n / 256 + 1 < 1024 ? n / 256 + 1 : 1024);
-    pair_row_ptr_kernel<<<grid, 256, 0, stream>>>(row_ptr, BH, nb, pair_row_ptr);
+static int pow2_at_least(int n) {
+    int p = 1;
+    while (p < n) p <<= 1;
+    return p;
+}
+
+cudaError_t launch_item_order(const int32_t *row_ptr, int64_t BH, int nb, int32_t *head_rank, int32_t *order,
+                              cudaStream_t stream) {
+    const int hp2 = pow2_at_least(static_cast<int>(BH));
+    const int ip2 = pow2_at_least((nb + 1) / 2);
+    head_rank_kernel<<<1, kOrderThreads, 2 * hp2 * sizeof(int), stream>>>(row_ptr, static_cast<int>(BH), nb, hp2,
+                                                                           head_rank);
+    item_order_kernel<<<static_cast<unsigned>(BH), kOrderThreads, 2 * ip2 * sizeof(int), stream>>>(
+        row_ptr, nb, ip2, head_rank, order);
     return cudaGetLastError();
 }
 

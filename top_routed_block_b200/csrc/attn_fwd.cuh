@@ -24,9 +24,10 @@ struct AttnLaunch {
 int attn_smem_bytes(int d, int bs);
 // Work items of the attention kernel: pairs of neighbouring query blocks per head.
 int64_t attn_num_items(int64_t BH, int nb);
-// pair_row_ptr[p] = row_ptr[first row of item p], plus the closing entry.
-cudaError_t launch_pair_row_ptr(const int32_t *row_ptr, int64_t BH, int nb, int32_t *pair_row_ptr,
-                                cudaStream_t stream);
+// order[] = work items head-major, longest first (heads by total selected blocks,
+// items of a head by block count); head_rank[BH] is scratch.  B*H <= 4096.
+cudaError_t launch_item_order(const int32_t *row_ptr, int64_t BH, int nb, int32_t *head_rank, int32_t *order,
+                              cudaStream_t stream);
 int attn_ctas_per_sm();  // resident CTAs per SM the launch grid is sized for
 cudaError_t launch_sparse_attn(const AttnLaunch &a, int d, int bs, cudaStream_t stream);
 

@@ -31,5 +31,6 @@ struct Carver {
 
 constexpr int kMaxRouteBlocks = 1024;   // routing keeps one row's scores in shared memory
 constexpr int kMaxCount = 4096;         // largest key-block count a row may hold
+constexpr int kMaxHeads = 4096;         // largest B*H of the attention call (head ordering in one CTA)
 
 }  // namespace fvattn
