@@ -21,6 +21,13 @@ SMALL = [
                grid=(1, 1, 1024 * 64 - 5), head_scale=("uniform", 0.5, 4.0), seed=34),
     W.Workload("single_block", B=1, H=2, N=50, d=64, bs=64, p=0.9, seed=35),
     W.Workload("p_one_small", B=2, H=2, N=700, d=128, bs=128, p=1.0, seed=36),
+    # key-block counts that land in each register-sort width of the selection kernel
+    W.Workload("nb47_d64", B=1, H=3, N=3000, d=64, bs=64, p=0.8, dist="structured", grid=(3, 10, 100),
+               head_scale=("uniform", 0.5, 4.0), seed=37),
+    W.Workload("nb313_d64", B=1, H=2, N=20000, d=64, bs=64, p=0.9, dist="structured", grid=(5, 40, 100),
+               head_scale=("uniform", 0.5, 4.0), seed=38),
+    W.Workload("nb600_d128", B=1, H=2, N=600 * 64 - 17, d=128, bs=64, p=0.7, dist="structured",
+               grid=(1, 1, 600 * 64 - 17), head_scale=("uniform", 0.5, 8.0), seed=39),
 ]
 
 
@@ -67,3 +74,23 @@ def test_route_capacity_overflow_reported(oracle_mod):
     torch.cuda.synchronize()
     assert int(out.dev_status.item()) == fv.FVATTN_ERR_CAPACITY
     assert int(out.row_ptr[-1].item()) == int(ora.row_ptr[-1])
+
+
+@pytest.mark.parametrize("nb", [1, 8, 47, 128, 256, 313, 929])
+def test_route_all_ties_keep_lowest_indices(nb):
+    """K = 0 makes every score 0 and every probability exactly 1/nb, so the
+    selection is decided by the tie-break alone: the first ceil(p*nb) blocks by
+    index (FVAttn review, §1 "Top-p routing"; ties by lower index)."""
+    p = 0.3
+    bs, d = 64, 64
+    N = nb * bs - (5 if nb > 1 else 0)
+    rng = np.random.default_rng(nb)
+    Q = rng.standard_normal((1, 2, N, d)).astype(np.float32)
+    Qb = (Q.view(np.uint32) >> 16).astype(np.uint16)       # bf16 by truncation: any values will do
+    Kb = np.zeros_like(Qb)
+    rp, ci, hc = gpu_route(to_dev(Qb), to_dev(Kb), p, bs)
+    k = int(np.ceil(p * nb))
+    assert np.all(np.diff(rp) == k)
+    for row in range(2 * nb):
+        assert np.array_equal(ci[rp[row]:rp[row + 1]], np.arange(k))
+    assert np.all(hc == k * nb)

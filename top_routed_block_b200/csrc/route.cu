@@ -14,8 +14,9 @@
 // Kernels:
 //   pool_kernel           HBM-bound: reads Q and K once, writes fp64 block means
 //                         (Q means row-major [BH,nb,d], K means transposed [BH,d,nb]).
-//   route_select_kernel   per (head, 8 query blocks): fp64 scores, softmax, a bitonic
-//                         sort of (score, index), prefix sum to p, a row bitmap.
+//   route_select_kernel   per (head, 8 query blocks): fp64 scores for the 8 rows, then
+//                         one warp per row: softmax, a bitonic sort of (score, index) in
+//                         registers, prefix sum to p, a row bitmap.
 //   csr_scan_kernel       row_ptr = exclusive scan of the row counts; head counts.
 //   csr_scatter_kernel    col_idx from the row bitmaps, ascending.
 #include <cstdint>
@@ -85,9 +86,16 @@ __global__ void __launch_bounds__(256) pool_kernel(const uint16_t *__restrict__ 
 }
 
 // ------------------------------------------------------ scores and selection
+//
+// One CTA per (head, kSelRows consecutive query blocks), one warp per query
+// block.  The score phase is shared by the CTA: thread t owns key blocks
+// j = t + m*kSelThreads and accumulates all kSelRows rows for them, so every K
+// mean is loaded once per CTA.  After one block barrier each warp finishes its
+// row alone (softmax, a bitonic sort held in registers, the prefix sum to p,
+// the row bitmap), with warp shuffles and no further block barrier.
 
-constexpr int kSelThreads = 256;
-constexpr int kSelRows = 8;  // query blocks per CTA (they share the K-mean loads)
+constexpr int kSelRows = 8;                  // query blocks (and warps) per CTA
+constexpr int kSelThreads = 32 * kSelRows;
 
 __device__ __forceinline__ double warp_max(double v) {
 #pragma unroll
@@ -100,184 +108,183 @@ __device__ __forceinline__ double warp_sum(double v) {
     return v;
 }
 
-// Block-wide reductions over kSelThreads threads; `red` holds 32 doubles.
-__device__ __forceinline__ double block_max(double v, double *red) {
-    v = warp_max(v);
-    const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
-    __syncthreads();
-    if (l == 0) red[w] = v;
-    __syncthreads();
-    double r = (l < kSelThreads / 32) ? red[l] : -CUDART_INF;
-    return warp_max(r);
-}
-__device__ __forceinline__ double block_sum(double v, double *red) {
-    v = warp_sum(v);
-    const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
-    __syncthreads();
-    if (l == 0) red[w] = v;
-    __syncthreads();
-    double r = (l < kSelThreads / 32) ? red[l] : 0.0;
-    return warp_sum(r);
+// x precedes y in the selection order: score descending, then index ascending.
+__device__ __forceinline__ bool precedes(double sx, int ix, double sy, int iy) {
+    return (sx > sy) || (sx == sy && ix < iy);
 }
 
-// "x comes after y" in the selection order: score descending, index ascending.
-__device__ __forceinline__ bool after(double kx, int ix, double ky, int iy) {
-    return (kx < ky) || (kx == ky && ix > iy);
-}
-
-template <int D>
+// MJ: key blocks per thread in the score phase (nb <= MJ * kSelThreads).
+// EPL: sorted positions per lane (nb <= 32 * EPL); lane l holds positions
+// l*EPL .. l*EPL+EPL-1, so a bitonic stage of partner distance j < EPL stays in
+// one lane's registers and a stage of distance j >= EPL pairs lane l with lane
+// l ^ (j / EPL).
+template <int D, int MJ, int EPL>
 __global__ void __launch_bounds__(kSelThreads) route_select_kernel(const double *__restrict__ qbar,
-                                                                   const double *__restrict__ kbarT, int nb, int np2,
-                                                                   double p, double scale,
-                                                                   int32_t *__restrict__ counts,
+                                                                   const double *__restrict__ kbarT, int nb, double p,
+                                                                   double scale, int32_t *__restrict__ counts,
                                                                    uint32_t *__restrict__ bitmap, int W) {
+    constexpr int NP2 = 32 * EPL;
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    double *sq = reinterpret_cast<double *>(smem_raw);          // [kSelRows][D]
-    double *ss = sq + kSelRows * D;                             // [kSelRows][nb] scores
-    double *pe = ss + kSelRows * nb;                            // [nb] probabilities by index
-    double *sk = pe + nb;                                       // [np2] sort keys, then cumulative mass
-    double *red = sk + np2;                                     // [32]
-    int *si = reinterpret_cast<int *>(red + 32);                // [np2] sort indices
-    uint32_t *bm = reinterpret_cast<uint32_t *>(si + np2);      // [32] row bitmap
-    int *kfirst = reinterpret_cast<int *>(bm + 32);             // [1]
+    double *sq = reinterpret_cast<double *>(smem_raw);                 // [kSelRows][D] query means
+    double *ss = sq + kSelRows * D;                                    // [kSelRows][nb] scores, then probabilities
+    uint32_t *bm = reinterpret_cast<uint32_t *>(ss + kSelRows * nb);   // [kSelRows][32] row bitmaps
 
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t bh = blockIdx.y;
     const int i0 = blockIdx.x * kSelRows;
     const int nrows = min(kSelRows, nb - i0);
 
-    for (int e = tid; e < kSelRows * D; e += kSelThreads) {
-        const int r = e / D;
-        sq[e] = (r < nrows) ? qbar[(bh * nb + i0) * D + e] : 0.0;
-    }
+    for (int e = tid; e < kSelRows * D; e += kSelThreads) sq[e] = (e / D < nrows) ? qbar[(bh * nb + i0) * D + e] : 0.0;
     __syncthreads();
 
     // s_ij = (sum_c qbar_i[c] * kbar_j[c]) * scale, c in index order, no fused multiply-add
-    constexpr int MJ = kMaxRouteBlocks / kSelThreads;
-    double acc[kSelRows][MJ];
+    {
+        double acc[kSelRows][MJ];
 #pragma unroll
-    for (int r = 0; r < kSelRows; ++r)
+        for (int r = 0; r < kSelRows; ++r)
 #pragma unroll
-        for (int m = 0; m < MJ; ++m) acc[r][m] = 0.0;
-    const double *kt = kbarT + bh * D * nb;
-    for (int c = 0; c < D; ++c) {
-        double kv[MJ];
+            for (int m = 0; m < MJ; ++m) acc[r][m] = 0.0;
+        const double *kt = kbarT + bh * D * nb;
+#pragma unroll 4
+        for (int c = 0; c < D; ++c) {
+            double kv[MJ];
 #pragma unroll
-        for (int m = 0; m < MJ; ++m) {
-            const int j = tid + m * kSelThreads;
-            kv[m] = (j < nb) ? __ldg(kt + static_cast<int64_t>(c) * nb + j) : 0.0;
-        }
-#pragma unroll
-        for (int r = 0; r < kSelRows; ++r) {
-            const double qv = sq[r * D + c];
-#pragma unroll
-            for (int m = 0; m < MJ; ++m) acc[r][m] = __dadd_rn(acc[r][m], __dmul_rn(qv, kv[m]));
-        }
-    }
-#pragma unroll
-    for (int r = 0; r < kSelRows; ++r)
-#pragma unroll
-        for (int m = 0; m < MJ; ++m) {
-            const int j = tid + m * kSelThreads;
-            if (j < nb && r < nrows) ss[r * nb + j] = __dmul_rn(acc[r][m], scale);
-        }
-    __syncthreads();
-
-    const int ept = (np2 >= kSelThreads) ? np2 / kSelThreads : 1;  // scan items per thread
-    for (int r = 0; r < nrows; ++r) {
-        const double *s = ss + r * nb;
-        const int64_t row = bh * nb + i0 + r;
-        // softmax over key blocks
-        double mx = -CUDART_INF;
-        for (int j = tid; j < nb; j += kSelThreads) mx = fmax(mx, s[j]);
-        mx = block_max(mx, red);
-        double z = 0.0;
-        for (int j = tid; j < nb; j += kSelThreads) {
-            const double e = exp(__dsub_rn(s[j], mx));
-            pe[j] = e;
-            z = __dadd_rn(z, e);
-        }
-        z = block_sum(z, red);
-        for (int j = tid; j < nb; j += kSelThreads) pe[j] = __ddiv_rn(pe[j], z);
-        if (tid < 32) bm[tid] = 0u;
-        if (tid == 0) *kfirst = np2;
-        __syncthreads();
-
-        int count;
-        if (p >= 1.0) {
-            count = nb;
-            for (int j = tid; j < nb; j += kSelThreads) atomicOr(&bm[j >> 5], 1u << (j & 31));
-        } else {
-            for (int e = tid; e < np2; e += kSelThreads) {
-                sk[e] = (e < nb) ? s[e] : -CUDART_INF;
-                si[e] = (e < nb) ? e : 0x7fffffff;
+            for (int m = 0; m < MJ; ++m) {
+                const int j = tid + m * kSelThreads;
+                kv[m] = (j < nb) ? __ldg(kt + static_cast<int64_t>(c) * nb + j) : 0.0;
             }
-            __syncthreads();
-            // bitonic network: ascending in the "after" relation
-            for (int k = 2; k <= np2; k <<= 1) {
-                for (int jj = k >> 1; jj > 0; jj >>= 1) {
-                    for (int e = tid; e < (np2 >> 1); e += kSelThreads) {
-                        const int a = (e / jj) * 2 * jj + (e % jj);
-                        const int b = a + jj;
-                        const double ka = sk[a], kb = sk[b];
-                        const int ia = si[a], ib = si[b];
-                        const bool up = (a & k) == 0;
-                        const bool swap = up ? after(ka, ia, kb, ib) : after(kb, ib, ka, ia);
-                        if (swap) {
-                            sk[a] = kb;
-                            sk[b] = ka;
-                            si[a] = ib;
-                            si[b] = ia;
+#pragma unroll
+            for (int r = 0; r < kSelRows; ++r) {
+                const double qv = sq[r * D + c];
+#pragma unroll
+                for (int m = 0; m < MJ; ++m) acc[r][m] = __dadd_rn(acc[r][m], __dmul_rn(qv, kv[m]));
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < kSelRows; ++r)
+#pragma unroll
+            for (int m = 0; m < MJ; ++m) {
+                const int j = tid + m * kSelThreads;
+                if (j < nb && r < nrows) ss[r * nb + j] = __dmul_rn(acc[r][m], scale);
+            }
+    }
+    __syncthreads();
+    if (warp >= nrows) return;  // only warp-level synchronisation from here on
+
+    double *s = ss + warp * nb;
+    uint32_t *bmw = bm + warp * 32;
+    const int64_t row = bh * nb + i0 + warp;
+    int count;
+    if (p >= 1.0) {
+        count = nb;
+        if (lane < W) {
+            const int nbits = min(32, nb - lane * 32);
+            bmw[lane] = (nbits == 32) ? 0xffffffffu : ((1u << nbits) - 1u);
+        }
+    } else {
+        bmw[lane] = 0u;
+        double key[EPL];
+        int idx[EPL];
+        double mx = -CUDART_INF;
+#pragma unroll
+        for (int q = 0; q < EPL; ++q) {
+            const int e = lane * EPL + q;
+            idx[q] = e;  // padding positions keep their own index and sort last
+            key[q] = (e < nb) ? s[e] : -CUDART_INF;
+            mx = fmax(mx, key[q]);
+        }
+        mx = warp_max(mx);
+        // softmax over key blocks; the probabilities replace the scores in s[] (by index)
+        double z = 0.0;
+#pragma unroll
+        for (int q = 0; q < EPL; ++q) {
+            const int e = lane * EPL + q;
+            if (e < nb) {
+                const double v = exp(__dsub_rn(key[q], mx));
+                s[e] = v;
+                z = __dadd_rn(z, v);
+            }
+        }
+        z = warp_sum(z);
+#pragma unroll
+        for (int q = 0; q < EPL; ++q) {
+            const int e = lane * EPL + q;
+            if (e < nb) s[e] = __ddiv_rn(s[e], z);
+        }
+        // bitonic sort of (score, index) into selection order
+#pragma unroll
+        for (int k = 2; k <= NP2; k <<= 1) {
+#pragma unroll
+            for (int j = k >> 1; j > 0; j >>= 1) {
+                if (j >= EPL) {
+                    const int lm = j / EPL;
+                    const bool lower = ((lane * EPL) & j) == 0;
+#pragma unroll
+                    for (int q = 0; q < EPL; ++q) {
+                        const bool up = (((lane * EPL + q) & k) == 0);
+                        const double ok = __shfl_xor_sync(0xffffffffu, key[q], lm);
+                        const int oi = __shfl_xor_sync(0xffffffffu, idx[q], lm);
+                        // the lower position of an ascending pair keeps the preceding element
+                        const bool take = (lower == up) ? precedes(ok, oi, key[q], idx[q])
+                                                        : precedes(key[q], idx[q], ok, oi);
+                        if (take) {
+                            key[q] = ok;
+                            idx[q] = oi;
                         }
                     }
-                    __syncthreads();
+                } else {
+#pragma unroll
+                    for (int q = 0; q < EPL; ++q) {
+                        const int q2 = q ^ j;
+                        if (q2 > q) {
+                            const bool up = (((lane * EPL + q) & k) == 0);
+                            const bool sw = up ? precedes(key[q2], idx[q2], key[q], idx[q])
+                                               : precedes(key[q], idx[q], key[q2], idx[q2]);
+                            if (sw) {
+                                const double tk = key[q];
+                                key[q] = key[q2];
+                                key[q2] = tk;
+                                const int ti = idx[q];
+                                idx[q] = idx[q2];
+                                idx[q2] = ti;
+                            }
+                        }
+                    }
                 }
             }
-            // inclusive prefix sum of the probabilities in sorted order
-            const int e0 = tid * ept;
-            double loc[kMaxRouteBlocks / kSelThreads];
-            double run = 0.0;
-#pragma unroll
-            for (int q = 0; q < kMaxRouteBlocks / kSelThreads; ++q) {
-                const int e = e0 + q;
-                const double v = (q < ept && e < nb) ? pe[si[e]] : 0.0;
-                run = __dadd_rn(run, v);
-                loc[q] = run;
-            }
-            // exclusive scan of the per-thread totals
-            const int lane = tid & 31, warp = tid >> 5;
-            double inc = run;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const double t = __shfl_up_sync(0xffffffffu, inc, o);
-                if (lane >= o) inc = __dadd_rn(inc, t);
-            }
-            double exc = __shfl_up_sync(0xffffffffu, inc, 1);
-            if (lane == 0) exc = 0.0;
-            __syncthreads();
-            if (lane == 31) red[warp] = inc;
-            __syncthreads();
-            double wpre = 0.0;
-            for (int w = 0; w < warp; ++w) wpre = __dadd_rn(wpre, red[w]);
-            const double pre = __dadd_rn(wpre, exc);
-#pragma unroll
-            for (int q = 0; q < kMaxRouteBlocks / kSelThreads; ++q) {
-                const int e = e0 + q;
-                if (q < ept && e < nb && __dadd_rn(pre, loc[q]) >= p) {
-                    atomicMin(kfirst, e);
-                    break;
-                }
-            }
-            __syncthreads();
-            const int kcut = (*kfirst < nb) ? *kfirst : nb - 1;
-            count = kcut + 1;
-            for (int e = tid; e <= kcut; e += kSelThreads) atomicOr(&bm[si[e] >> 5], 1u << (si[e] & 31));
         }
-        __syncthreads();
-        if (tid < W) bitmap[row * W + tid] = bm[tid];
-        if (tid == 0) counts[row] = count;
-        __syncthreads();
+        __syncwarp();
+        // cumulative mass in sorted order: per-lane running sums plus the lanes before
+        double loc[EPL];
+        double run = 0.0;
+#pragma unroll
+        for (int q = 0; q < EPL; ++q) {
+            run = __dadd_rn(run, (idx[q] < nb) ? s[idx[q]] : 0.0);
+            loc[q] = run;
+        }
+        double inc = run;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const double t = __shfl_up_sync(0xffffffffu, inc, o);
+            if (lane >= o) inc = __dadd_rn(t, inc);
+        }
+        double pre = __shfl_up_sync(0xffffffffu, inc, 1);
+        if (lane == 0) pre = 0.0;
+        int first = NP2;
+#pragma unroll
+        for (int q = EPL - 1; q >= 0; --q)
+            if (__dadd_rn(pre, loc[q]) >= p) first = lane * EPL + q;
+        first = __reduce_min_sync(0xffffffffu, first);
+        const int kcut = (first < nb) ? first : nb - 1;  // the mass never reached p: keep every block
+        count = kcut + 1;
+        __syncwarp();
+#pragma unroll
+        for (int q = 0; q < EPL; ++q)
+            if (lane * EPL + q <= kcut) atomicOr(&bmw[idx[q] >> 5], 1u << (idx[q] & 31));
     }
+    __syncwarp();
+    if (lane < W) bitmap[row * W + lane] = bmw[lane];
+    if (lane == 0) counts[row] = count;
 }
 
 // -------------------------------------------------------------------- CSR
@@ -367,11 +374,46 @@ __global__ void __launch_bounds__(256) csr_scatter_kernel(const uint32_t *__rest
 // ---------------------------------------------------------------- launcher
 
 size_t route_select_smem_bytes(int d, int nb) {
-    int np2 = 1;
-    while (np2 < nb) np2 <<= 1;
-    return sizeof(double) * (kSelRows * d + kSelRows * nb + nb + np2 + 32) + sizeof(int) * np2 +
-           sizeof(uint32_t) * 32 + sizeof(int) * 4;
+    return sizeof(double) * (kSelRows * d + kSelRows * nb) + sizeof(uint32_t) * kSelRows * 32;
 }
+
+namespace {
+
+struct SelectArgs {
+    const double *qbar, *kbarT;
+    int nb;
+    double p, scale;
+    int32_t *counts;
+    uint32_t *bitmap;
+    int W;
+    int64_t BH;
+};
+
+template <int D, int MJ, int EPL>
+cudaError_t launch_select(const SelectArgs &a, cudaStream_t stream) {
+    const size_t smem = route_select_smem_bytes(D, a.nb);
+    cudaError_t e = cudaFuncSetAttribute(route_select_kernel<D, MJ, EPL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    const dim3 grid(static_cast<unsigned>(ceil_div(a.nb, kSelRows)), static_cast<unsigned>(a.BH));
+    route_select_kernel<D, MJ, EPL><<<grid, kSelThreads, smem, stream>>>(a.qbar, a.kbarT, a.nb, a.p, a.scale,
+                                                                         a.counts, a.bitmap, a.W);
+    return cudaGetLastError();
+}
+
+// Smallest register sort that holds nb positions (nb <= kMaxRouteBlocks = 1024).
+template <int D>
+cudaError_t dispatch_select(const SelectArgs &a, cudaStream_t stream) {
+    static_assert(kSelThreads == 256 && kMaxRouteBlocks == 1024, "dispatch covers nb <= 1024 with 256 threads");
+    if (a.nb <= 32) return launch_select<D, 1, 1>(a, stream);
+    if (a.nb <= 64) return launch_select<D, 1, 2>(a, stream);
+    if (a.nb <= 128) return launch_select<D, 1, 4>(a, stream);
+    if (a.nb <= 256) return launch_select<D, 1, 8>(a, stream);
+    if (a.nb <= 512) return launch_select<D, 2, 16>(a, stream);
+    return launch_select<D, 4, 32>(a, stream);
+}
+
+}  // namespace
 
 RouteWorkspace route_workspace_layout(int64_t BH, int nb, int d) {
     RouteWorkspace w{};
@@ -397,29 +439,20 @@ cudaError_t launch_route(const void *Q, const void *K, int64_t BH, int N, int d,
     uint32_t *bitmap = reinterpret_cast<uint32_t *>(ws + w.bitmap);
     const int64_t rows = BH * nb;
     const double scale = 1.0 / sqrt(static_cast<double>(d));
-    int np2 = 1;
-    while (np2 < nb) np2 <<= 1;
-    const size_t sel_smem = route_select_smem_bytes(d, nb);
-    const dim3 sel_grid(static_cast<unsigned>(ceil_div(nb, kSelRows)), static_cast<unsigned>(BH));
+    const SelectArgs sel{qbar, kbarT, nb, p, scale, counts, bitmap, w.W, BH};
     const auto *q16 = static_cast<const uint16_t *>(Q);
     const auto *k16 = static_cast<const uint16_t *>(K);
+    cudaError_t e;
     if (d == 128) {
         const dim3 grid(static_cast<unsigned>(ceil_div(rows, 256 / 16)), 2);
         pool_kernel<128><<<grid, 256, 0, stream>>>(q16, k16, BH, N, bs, nb, qbar, kbarT);
-        cudaError_t e = cudaFuncSetAttribute(route_select_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(sel_smem));
-        if (e != cudaSuccess) return e;
-        route_select_kernel<128><<<sel_grid, kSelThreads, sel_smem, stream>>>(qbar, kbarT, nb, np2, p, scale, counts,
-                                                                              bitmap, w.W);
+        e = dispatch_select<128>(sel, stream);
     } else {
         const dim3 grid(static_cast<unsigned>(ceil_div(rows, 256 / 8)), 2);
         pool_kernel<64><<<grid, 256, 0, stream>>>(q16, k16, BH, N, bs, nb, qbar, kbarT);
-        cudaError_t e = cudaFuncSetAttribute(route_select_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(sel_smem));
-        if (e != cudaSuccess) return e;
-        route_select_kernel<64><<<sel_grid, kSelThreads, sel_smem, stream>>>(qbar, kbarT, nb, np2, p, scale, counts,
-                                                                             bitmap, w.W);
+        e = dispatch_select<64>(sel, stream);
     }
+    if (e != cudaSuccess) return e;
     csr_scan_kernel<<<1, kScanThreads, 0, stream>>>(counts, rows, nb, BH, row_ptr, capacity, head_counts,
                                                     dev_status);
     csr_scatter_kernel<<<static_cast<unsigned>(ceil_div(rows, 8)), 256, 0, stream>>>(bitmap, row_ptr, rows, w.W,
