@@ -18,7 +18,10 @@
 //     run time; here the SMs are balanced instead).
 //   * Warps 0-3 run the softmax, rescale and epilogue of slot A, warps 4-7 those
 //     of slot B (thread = query row = TMEM lane); warp 8 issues TMA loads; warp
-//     9 issues tcgen05 MMAs.  Per union block the MMA warp issues
+//     9 issues tcgen05 MMAs; warps 10-11 complete the third warpgroup.  That
+//     warpgroup hands registers to the softmax warpgroups (setmaxnreg), which
+//     keep a whole 128-column S row per thread without spilling.  Per union
+//     block the MMA warp issues
 //     S_A, PV_B(previous B block), S_B, PV_A: while one warpgroup runs the
 //     softmax of its tile, the tensor cores run the other slot's two GEMMs.
 //   * Q tiles (one per slot) and a ring of K/V stages arrive by TMA (3-D tensor
@@ -40,6 +43,7 @@
 //     records FVATTN_ERR_DEVICE_TIMEOUT; all roles then drain and exit.
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <atomic>
 #include <cstdint>
 #include <math_constants.h>
 
@@ -55,9 +59,18 @@ using namespace ptx;
 
 constexpr int kRowsM = 128;           // query rows per tile (tcgen05 M)
 constexpr int kSlots = 2;             // query blocks per work item
-constexpr int kThreads = 320;         // 2 softmax warpgroups + TMA warp + MMA warp
+constexpr int kThreads = 384;         // 2 softmax warpgroups + one warpgroup for TMA and MMA issue
 constexpr int kTmaWarp = 8;
-constexpr int kMmaWarp = 9;
+constexpr int kMmaWarp = 9;           // warps 10 and 11 only take part in the register hand-over
+// Register hand-over (setmaxnreg): the launch gives every thread kLaunchRegs; the
+// TMA/MMA warpgroup drops to kIssueRegs and the two softmax warpgroups, which
+// hold a whole 128-column S row per thread, rise to kSoftmaxRegs.  The split must
+// not exceed the launch pool (checked on the host before every launch).
+constexpr int kLaunchRegs = 168;      // 65536 / 384, rounded down to a multiple of 8
+constexpr int kIssueRegs = 80;
+constexpr int kSoftmaxRegs = 208;
+static_assert(2 * 128 * kSoftmaxRegs + 128 * kIssueRegs <= kThreads * kLaunchRegs, "register split exceeds the pool");
+static_assert(kSoftmaxRegs % 8 == 0 && kIssueRegs % 8 == 0, "setmaxnreg takes multiples of 8");
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemSlot = 256;   // TMEM columns per slot
 constexpr uint32_t kTmemO = 128;      // O offset inside a slot (S/P at offset 0)
@@ -249,6 +262,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tmem = bar->tmem_base;
 
+    if (warp >= kTmaWarp) {
+    // The register hand-over and the code that uses the new count sit in the same
+    // branch, so the compiler allocates each role's registers against its own limit.
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kIssueRegs));
     if (warp == kTmaWarp) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
@@ -458,7 +475,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_commit(&bar->drain);
             mbar_wait_teardown(&bar->drain, 0);
         }
+    }
     } else {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
         // ------------------------------------------------ softmax / epilogue
         const int X = warp >> 2;                                   // slot of this warpgroup
         const int r = threadIdx.x & (kRowsM - 1);                  // tile row = TMEM lane
@@ -712,6 +731,16 @@ cudaError_t launch_item_order(const int32_t *row_ptr, int64_t BH, int nb, int32_
 template <int D, int BS>
 static cudaError_t launch_t(const AttnLaunch &a, cudaStream_t stream) {
     auto kern = sparse_attn_fwd_kernel<D, BS>;
+    // The register hand-over waits until the pool holds the requested registers, so
+    // it must fit in what the launch allocates: checked once per instantiation.
+    static std::atomic<int> regs_ok{0};  // 0 unknown, 1 fits, -1 does not
+    if (regs_ok.load() == 0) {
+        cudaFuncAttributes fa{};
+        cudaError_t e = cudaFuncGetAttributes(&fa, kern);
+        if (e != cudaSuccess) return e;
+        regs_ok.store(2 * 128 * kSoftmaxRegs + 128 * kIssueRegs <= fa.numRegs * kThreads ? 1 : -1);
+    }
+    if (regs_ok.load() < 0) return cudaErrorInvalidConfiguration;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<D, BS>::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     kern<<<a.grid, kThreads, Cfg<D, BS>::SMEM_BYTES, stream>>>(
