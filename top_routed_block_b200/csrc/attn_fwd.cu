@@ -97,9 +97,11 @@ struct Barriers {
     uint64_t sched_full[2], sched_empty[2];
     uint64_t drain;
     int4 sched_item[2][kSlots];  // per slot: {row or -1, col start, count, valid item}
+    int4 ring_step[8];           // per K stage: {key block, row A uses it, row B uses it, last step of item}
     uint32_t tmem_base;
     int abort_flag;
 };
+static_assert(sizeof(Barriers) <= 512, "barrier block exceeds its shared-memory reservation");
 
 // One step of the merge of the two rows' key-block lists.
 struct Step {
@@ -324,12 +326,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 while (ok && !mg.done()) {
                     const Step s = mg.next();
                     if (mg.bad) record_error(dev_status, FVATTN_ERR_BAD_CSR);
+                    const bool last = mg.done();
                     for (int kv = 0; kv < 2 && ok; ++kv) {
                         const uint32_t st = rc % C::NST;
                         if (!mbar_wait(&bar->ring_empty[st], ((rc / C::NST) & 1) ^ 1, abort_flag, dev_status)) {
                             ok = false;
                             break;
                         }
+                        // the MMA warp reads the step from its K stage once the stage is full
+                        if (kv == 0) bar->ring_step[st] = make_int4(s.kblk, s.pa ? 1 : 0, s.pb ? 1 : 0, last ? 1 : 0);
                         mbar_arrive_expect_tx(&bar->ring_full[st], C::STAGE_BYTES);
                         for (int kb = 0; kb < C::KBLK; ++kb)
                             tma_load_3d(ring + st * C::STAGE_BYTES + kb * BS * 128, kv == 0 ? &tmap_k : &tmap_v,
@@ -399,15 +404,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ++on[x];
                     }
                 }
-                Merge mg;
-                mg.init(col_idx, sx[0], sx[1], nb);
+                // the producer walks the merge of the two rows' block lists and leaves
+                // each step in its K stage, so this thread never reads col_idx
+                bool more = (sx[0].x >= 0 && sx[0].z > 0) || (sx[1].x >= 0 && sx[1].z > 0);
                 int b_pending = -1;  // ring stage of V for the B tile whose PV is still to issue
-                while (ok && !mg.done()) {
-                    const Step s = mg.next();
+                while (ok && more) {
                     const uint32_t kst = rc % C::NST, vst = (rc + 1) % C::NST;
                     const uint32_t kph = (rc / C::NST) & 1, vph = ((rc + 1) / C::NST) & 1;
                     rc += 2;
                     if (!wait(&bar->ring_full[kst], kph)) break;
+                    const int4 step = bar->ring_step[kst];
+                    const Step s = {step.x, step.y != 0, step.z != 0};
+                    more = step.w == 0;
                     if (s.pa) {
                         if (q_wait[0]) {
                             if (!wait(&bar->q_full[0], qn[0] & 1)) break;
