@@ -170,28 +170,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
     return y;
 }
 
-// 2^x on the FMA pipe, for finite x: x = n + f with n = round(x) and f in [-1/2, 1/2];
-// 2^f by a cubic fitted here for least maximum relative error on [-1/2, 1/2]
-// (iteratively reweighted least squares on Chebyshev nodes; max relative error
-// 7.5e-5, far below the 2^-9 rounding of the bf16 P it feeds); 2^n is added to
-// the exponent field.  x is clamped at -126, so results below 2^-126 are not
-// exact (they are then under 1.2e-38).  Adding 1.5*2^23 rounds x to an integer
-// held in the low mantissa bits of t, whose bit pattern shifted left by 23 is
-// n in the exponent field.
-constexpr float kExp2C0 = 0.99992806f, kExp2C1 = 0.69326097f, kExp2C2 = 0.24261114f, kExp2C3 = 0.05517167f;
-
-__device__ __forceinline__ float ex2_poly(float x) {
-    x = fmaxf(x, -126.0f);
-    const float t = __fadd_rn(x, 12582912.0f);
-    const float f = __fsub_rn(x, __fsub_rn(t, 12582912.0f));
-    const float p = fmaf(fmaf(fmaf(kExp2C3, f, kExp2C2), f, kExp2C1), f, kExp2C0);
-    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
-
-// Of every 8 exponentials of a full (unmasked) block, this many run as ex2_poly on
-// the FMA pipe instead of the MUFU unit.
-constexpr int kPolyOf8 = 0;
-
 __device__ __forceinline__ float max3f(float a, float b, float c) {
     float r;
     asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
@@ -548,24 +526,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float neg_m = (m_new == -CUDART_INF_F) ? 0.0f : -m_new;
                 float rs[4] = {0.0f, 0.0f, 0.0f, 0.0f};
                 // P packed as bf16 pairs in place: v[c/2] <- (p[c], p[c+1])
-                if (lim >= BS) {
+                // one loop for full and masked tiles (masked scores are -inf, and 2^-inf = 0),
+                // which keeps the kernel's code small enough for the instruction caches
 #pragma unroll
-                    for (int c = 0; c < BS; c += 2) {
-                        const float x0 = fmaf(__uint_as_float(v[c]), scale_log2, neg_m);
-                        const float x1 = fmaf(__uint_as_float(v[c + 1]), scale_log2, neg_m);
-                        const float p0 = ((c & 7) >= 8 - kPolyOf8) ? ex2_poly(x0) : ex2_approx(x0);
-                        const float p1 = ((c & 7) + 1 >= 8 - kPolyOf8) ? ex2_poly(x1) : ex2_approx(x1);
-                        rs[(c >> 1) & 3] += p0 + p1;
-                        v[c >> 1] = pack_bf16(p0, p1);
-                    }
-                } else {
-#pragma unroll
-                    for (int c = 0; c < BS; c += 2) {
-                        const float p0 = ex2_approx(fmaf(__uint_as_float(v[c]), scale_log2, neg_m));
-                        const float p1 = ex2_approx(fmaf(__uint_as_float(v[c + 1]), scale_log2, neg_m));
-                        rs[(c >> 1) & 3] += p0 + p1;
-                        v[c >> 1] = pack_bf16(p0, p1);
-                    }
+                for (int c = 0; c < BS; c += 2) {
+                    const float p0 = ex2_approx(fmaf(__uint_as_float(v[c]), scale_log2, neg_m));
+                    const float p1 = ex2_approx(fmaf(__uint_as_float(v[c + 1]), scale_log2, neg_m));
+                    rs[(c >> 1) & 3] += p0 + p1;
+                    v[c >> 1] = pack_bf16(p0, p1);
                 }
 #pragma unroll
                 for (int c0 = 0; c0 < BS / 2; c0 += 32)
