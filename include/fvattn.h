@@ -147,11 +147,11 @@ FVATTN_API int fvattn_lpt_order(const int32_t *row_ptr, int64_t rows, int max_co
  *   O           out, bf16 [B,H,N,d].   LSE  out, fp32 [B,H,N].
  *   workspace   >= fvattn_fwd_workspace_bytes(B,H,N,block).
  * Matmuls run on the tensor cores in bf16 with fp32 accumulation; softmax in
- * fp32.  A persistent grid takes work items (pairs of neighbouring query
- * blocks of one head) from a queue ordered head-major and longest-first: heads
- * by total selected blocks descending, the items of a head by block count
- * descending (ties by lower index), so that the SMs share one head's K and V
- * in L2 at a time and finish on the shortest items.  B*H <= 4096, else
+ * fp32.  A persistent grid takes work items (the CSR rows) from a queue
+ * ordered head-major and longest-first: heads by total selected blocks
+ * descending, the rows of a head by block count descending (ties by lower
+ * index), so that the SMs share one head's K and V in L2 at a time and finish
+ * on the shortest rows.  B*H <= 4096, else
  * FVATTN_ERR_UNSUPPORTED.  Out-of-range or non-ascending column indices are
  * skipped and set *dev_status = FVATTN_ERR_BAD_CSR.
  */
@@ -201,7 +201,7 @@ FVATTN_API int fvattn_attention_host(const void *hQ, const void *hK, const void 
  * file-scope device array of FVATTN_NOALLOC_SCRATCH_BYTES (4 MiB) inside the
  * library, which every device that loads the library keeps until the process
  * exits.  Shapes that need more return FVATTN_ERR_CAPACITY without launching
- * anything (about 2M rows B*H*ceil(N/block) at most).
+ * anything (about 1M rows B*H*ceil(N/block) at most).
  *
  * The first call on each device looks up the array's device address
  * (cudaGetSymbolAddress, with that device current) and caches it; make that first

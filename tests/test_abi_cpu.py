@@ -66,8 +66,8 @@ def test_size_helpers(lib):
     assert fv.fvattn_route_workspace_bytes(1, 1, 100, 96, 128) == 0      # d unsupported
     assert fv.fvattn_route_workspace_bytes(1, 1, 100, 64, 32) == 0       # block unsupported
     fw = fv.fvattn_fwd_workspace_bytes(1, 40, 32760, 128)
-    # the work order: one int32 per pair of neighbouring query blocks, plus one rank per head
-    assert fw >= 40 * 128 * 4 + 40 * 4
+    # the work order: one int32 per CSR row, plus one rank per head
+    assert fw >= 40 * 256 * 4 + 40 * 4
     assert fv.fvattn_fwd_workspace_bytes(1, 4097, 128, 128) == 0           # head limit 4096
     assert fv.fvattn_lpt_workspace_bytes(10, 5000) == 0                  # count limit 4096
 

@@ -61,7 +61,7 @@ def test_noalloc_matches_workspace_entry_point_twice(w):
 def test_noalloc_rejects_shapes_beyond_its_scratch():
     import top_routed_block_b200 as fv
     lib = fv.load_library()
-    B, H, N, block = 16, 256, 131072, 128   # 4194304 rows (2097152 query-block pairs): more than the scratch holds
+    B, H, N, block = 16, 256, 65536, 128    # 2097152 rows: more than the scratch holds
     assert fv.fvattn_fwd_workspace_bytes(B, H, N, block) > 4 << 20
     fake = 256  # never dereferenced: the size check fails first
     rc = lib.fvattn_sparse_fwd_noalloc(fake, fake, fake, fake, fake, B, H, N, 128, block, 0, fake, fake, fake, None)

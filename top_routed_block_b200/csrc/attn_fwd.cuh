@@ -8,8 +8,9 @@
 namespace fvattn {
 
 struct AttnLaunch {
-    const CUtensorMap *tmap_q, *tmap_k, *tmap_v;  // host copies, passed by value as kernel parameters
-    const int32_t *row_ptr, *col_idx, *order;  // order: work items (query-block pairs), longest first
+    const CUtensorMap *tmap_k, *tmap_v;  // host copies, passed by value as kernel parameters
+    const void *Q;                       // bf16 [B,H,N,d], read row by row into tensor memory
+    const int32_t *row_ptr, *col_idx, *order;  // order: work items (CSR rows), head-major, longest first
     int n_items;
     int *work_counter;  // zeroed before the launch
     int N, nb, causal;
@@ -22,10 +23,10 @@ struct AttnLaunch {
 };
 
 int attn_smem_bytes(int d, int bs);
-// Work items of the attention kernel: pairs of neighbouring query blocks per head.
+// Work items of the attention kernel: the CSR rows (query blocks of every head).
 int64_t attn_num_items(int64_t BH, int nb);
-// order[] = work items head-major, longest first (heads by total selected blocks,
-// items of a head by block count); head_rank[BH] is scratch.  B*H <= 4096.
+// order[] = rows head-major, longest first (heads by total selected blocks, rows of
+// a head by block count); head_rank[BH] is scratch.  B*H <= 4096, nb <= 4096.
 cudaError_t launch_item_order(const int32_t *row_ptr, int64_t BH, int nb, int32_t *head_rank, int32_t *order,
                               cudaStream_t stream);
 int attn_ctas_per_sm();  // resident CTAs per SM the launch grid is sized for
