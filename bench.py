@@ -341,6 +341,27 @@ def run_ours(args, w, rank, world, local):
     h2d = 3 * elem * 2
     d2h = elem * 2 + w.B * w.H * w.N * 4 + 8
 
+    # Load balance over the SMs (outside the timed region): busy time of every CTA of the
+    # persistent grid, with the head-major longest-first queue and with rows in index order.
+    # The host-buffer path above routed chunk by chunk into the plan: route the whole batch again.
+    plan.run_route(dQ, dK, w.p, stream=stream)
+    balance = {}
+    for name, natural in (("lpt", False), ("natural", True)):
+        runs = []
+        for _ in range(3):
+            a.record(stream)
+            _, _, st, busy = fv.fvattn_sparse_fwd_profiled(dQ, dK, dV, plan.route.row_ptr, plan.route.col_idx, w.bs,
+                                                           w.causal, natural_order=natural, stream=stream, O=plan.O,
+                                                           LSE=plan.LSE, workspace=plan.fwd_ws,
+                                                           dev_status=plan.status[1:2])
+            b.record(stream)
+            torch.cuda.synchronize(dev)
+            fv.check_status(st, "fvattn_sparse_fwd_profiled")
+            t = busy.double().cpu().numpy()
+            runs.append((a.elapsed_time(b), float(t.max() / t.mean()), float(t.max() * 1e-6), int(t.size)))
+        ms_, lif, mx, g = sorted(runs)[1]  # the median run by time
+        balance[name] = {"lif": lif, "call_ms": ms_, "max_cta_busy_ms": mx, "ctas": g}
+
     if rank != 0:
         return
     peaks, peak_src = load_peaks()
@@ -351,6 +372,7 @@ def run_ours(args, w, rank, world, local):
         cpu = oracle_sample(w, Qh, Kh, Vh, budget_s=args.cpu_budget)
         cpu.pop("route_s_full", None)
     counts = plan.route.head_counts.cpu().numpy()
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": max(3, args.warmup), "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
@@ -370,7 +392,18 @@ def run_ours(args, w, rank, world, local):
         "route_roofline": {"bound": "hbm", "pool_bytes": 2 * elem * 2,
                            "achieved_gbs_whole_route": 2 * elem * 2 / (r_ms * 1e-3) / 1e9,
                            "peak": float(peaks["hbm_gbs"]), "unit": "GB/s"},
-        "head_counts": {"min": int(counts.min()), "max": int(counts.max()), "mean": float(counts.mean())},
+        "head_counts": {"min": int(counts.min()), "max": int(counts.max()), "mean": float(counts.mean()),
+                        "density_histogram": {"edges": [round(x, 1) for x in np.linspace(0.0, 1.0, 11)],
+                                              "heads": np.histogram(counts / float(w.nb * w.nb), bins=10,
+                                                                    range=(0.0, 1.0))[0].tolist()}},
+        "load_balance": dict(balance, note="LIF = max / mean busy time over the CTAs of the persistent grid "
+                                           "(global timer, one call each); lpt = the head-major longest-first "
+                                           "queue fvattn_sparse_fwd uses, natural = rows in index order"),
+        "mufu": {"exp_per_s": float(nnz) * w.bs * w.bs / (attn_ms * 1e-3),
+                 "ceiling_at_max_clock": 16.0 * sms * float(peaks.get("sm_max_mhz", 1965.0)) * 1e6,
+                 "frac": float(nnz) * w.bs * w.bs / (attn_ms * 1e-3)
+                         / (16.0 * sms * float(peaks.get("sm_max_mhz", 1965.0)) * 1e6),
+                 "note": "one exp2 per selected score (full tiles); ceiling = 16 per clock per SM"},
         "e2e": {"value": flops / (e2e_ms * 1e-3) / 1e12 * world, "unit": UNIT, "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": args.steps * (ROUTE_KERNELS_PER_CALL + FWD_KERNELS_PER_CALL),

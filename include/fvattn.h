@@ -229,6 +229,26 @@ FVATTN_API int fvattn_test_sparse_fwd_stall(const void *Q, const void *K, const 
                                             int causal, void *O, float *LSE, void *workspace, size_t ws_bytes,
                                             int32_t *dev_status, fvattn_stream_t stream);
 
+/*
+ * fvattn_sparse_fwd_profiled -- fvattn_sparse_fwd that also reports how busy
+ * each CTA of its persistent grid was, for the load-imbalance factor
+ * LIF = max / mean busy time over the SMs (FVAttn review §3 reports the LIF of
+ * its run-time balancing, 1.34 -> 1.08 across GPUs; here the SMs of one GPU).
+ * A diagnostic entry point: results equal those of fvattn_sparse_fwd.
+ *   order_mode   0: the head-major longest-first work queue fvattn_sparse_fwd uses;
+ *                1: rows in index order, the comparison point.
+ *   cta_busy_ns  device int64[number of SMs], 8-byte aligned: entry c receives the
+ *                global-timer nanoseconds from CTA c's start to the end of its last
+ *                work item (entries past *grid are left untouched).
+ *   grid         out (host): number of CTAs launched (at most the number of SMs).
+ * Other arguments, layouts and errors as fvattn_sparse_fwd; order_mode outside
+ * {0,1} or a null cta_busy_ns / grid is FVATTN_ERR_INVALID_ARG.
+ */
+FVATTN_API int fvattn_sparse_fwd_profiled(const void *Q, const void *K, const void *V, const int32_t *row_ptr,
+                                          const int32_t *col_idx, int B, int H, int N, int d, int block, int causal,
+                                          void *O, float *LSE, void *workspace, size_t ws_bytes, int32_t *dev_status,
+                                          int order_mode, int64_t *cta_busy_ns, int *grid, fvattn_stream_t stream);
+
 /* Compiled-in build description (architecture, version), static string. */
 FVATTN_API const char *fvattn_build_info(void);
 

@@ -188,3 +188,26 @@ def test_host_buffer_path_matches_device_path():
                                  dK=torch.empty_like(dK), dV=torch.empty_like(dV), hO=hO, hLSE=hL)
         assert torch.equal(hO, O_dev.cpu())
         assert torch.equal(hL, L_dev.cpu())
+
+
+def test_profiled_forward_reports_busy_time_and_matches():
+    """fvattn_sparse_fwd_profiled returns exactly what fvattn_sparse_fwd returns, in
+    either work order (rows are independent), plus a positive busy time per CTA."""
+    import top_routed_block_b200 as fv
+    w = W.Workload("profiled", B=1, H=6, N=3000, d=128, bs=128, p=0.8, dist="structured", grid=(5, 20, 30),
+                   head_scale=("uniform", 0.5, 4.0), seed=45)
+    Q, K, V = W.generate(w)
+    dQ, dK, dV = to_dev(Q), to_dev(K), to_dev(V)
+    r = fv.fvattn_route(dQ, dK, w.p, w.bs)
+    fv.check_status(r.dev_status, "route")
+    O_ref, L_ref, st = fv.fvattn_sparse_fwd(dQ, dK, dV, r.row_ptr, r.col_idx, w.bs, False)
+    fv.check_status(st, "fwd")
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    for natural in (False, True):
+        O, L, st, busy = fv.fvattn_sparse_fwd_profiled(dQ, dK, dV, r.row_ptr, r.col_idx, w.bs, False,
+                                                       natural_order=natural)
+        fv.check_status(st, "profiled")
+        assert torch.equal(O, O_ref) and torch.equal(L, L_ref)
+        b = busy.cpu().numpy()
+        assert 1 <= b.size <= min(sms, w.rows)
+        assert np.all(b > 0)

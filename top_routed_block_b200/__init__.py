@@ -68,6 +68,7 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         "fvattn_sparse_fwd": (I, [P, P, P, P, P, I, I, I, I, I, I, P, P, P, SZ, P, P]),
         "fvattn_sparse_fwd_noalloc": (I, [P, P, P, P, P, I, I, I, I, I, I, P, P, P, P]),
         "fvattn_test_sparse_fwd_stall": (I, [P, P, P, P, P, I, I, I, I, I, I, P, P, P, SZ, P, P]),
+        "fvattn_sparse_fwd_profiled": (I, [P, P, P, P, P, I, I, I, I, I, I, P, P, P, SZ, P, I, P, P, P]),
         "fvattn_attention_host": (I, [P, P, P, I, I, I, I, I, D, I, P, P, P, P, P, P, P, P, P, I64, P, P, SZ, P, SZ,
                                       P, P]),
     }
@@ -208,6 +209,37 @@ def fvattn_sparse_fwd(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, row_ptr
                                _ptr(dev_status), _stream_ptr(stream))
     _check(rc, "fvattn_sparse_fwd")
     return O, LSE, dev_status
+
+
+def fvattn_sparse_fwd_profiled(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, row_ptr: torch.Tensor,
+                               col_idx: torch.Tensor, block: int, causal: bool = False, *, natural_order: bool = False,
+                               stream=None, O: torch.Tensor | None = None, LSE: torch.Tensor | None = None,
+                               workspace: torch.Tensor | None = None, dev_status: torch.Tensor | None = None):
+    """fvattn_sparse_fwd plus the per-CTA busy time (ns) of its persistent grid.
+
+    Returns (O, LSE, dev_status, busy_ns) with busy_ns an int64 device tensor of one
+    entry per launched CTA; ``natural_order`` takes the rows in index order instead
+    of the head-major longest-first queue."""
+    lib = load_library()
+    B, H, N, d = _shape(Q)
+    dev = Q.device
+    if O is None:
+        O = torch.empty_like(Q)
+    if LSE is None:
+        LSE = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    if dev_status is None:
+        dev_status = torch.zeros(1, dtype=torch.int32, device=dev)
+    if workspace is None:
+        workspace = _empty_bytes(fvattn_fwd_workspace_bytes(B, H, N, block), dev)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    busy = torch.zeros(sms, dtype=torch.int64, device=dev)
+    grid = ctypes.c_int(0)
+    rc = lib.fvattn_sparse_fwd_profiled(_ptr(Q), _ptr(K), _ptr(V), _ptr(row_ptr), _ptr(col_idx), B, H, N, d, block,
+                                        1 if causal else 0, _ptr(O), _ptr(LSE), _ptr(workspace), workspace.numel(),
+                                        _ptr(dev_status), 1 if natural_order else 0, _ptr(busy), ctypes.byref(grid),
+                                        _stream_ptr(stream))
+    _check(rc, "fvattn_sparse_fwd_profiled")
+    return O, LSE, dev_status, busy[: grid.value]
 
 
 def fvattn_sparse_fwd_noalloc(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, row_ptr: torch.Tensor,

@@ -208,7 +208,8 @@ int fvattn_lpt_order(const int32_t *row_ptr, int64_t rows, int max_count, int32_
 static int sparse_fwd_impl(const void *Q, const void *K, const void *V, const int32_t *row_ptr,
                            const int32_t *col_idx, int B, int H, int N, int d, int block, int causal, void *O,
                            float *LSE, void *workspace, size_t ws_bytes, int32_t *dev_status, fvattn_stream_t stream,
-                           int test_stall) {
+                           int test_stall, int order_mode = 0, int64_t *cta_busy_ns = nullptr,
+                           int *grid_out = nullptr) {
     int rc = check_shape(B, H, N, d, block);
     if (rc != FVATTN_OK) return rc;
     if (!Q || !K || !V || !row_ptr || !col_idx || !O || !LSE || !workspace || !dev_status)
@@ -239,8 +240,10 @@ static int sparse_fwd_impl(const void *Q, const void *K, const void *V, const in
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if ((rc = from_cuda(cudaMemsetAsync(dev_status, 0, sizeof(int32_t), s))) != FVATTN_OK) return rc;
-    // work items (CSR rows): head-major, longest first
-    if ((rc = from_cuda(launch_item_order(row_ptr, BH, nb, head_rank, order, s))) != FVATTN_OK) return rc;
+    // work items (CSR rows): head-major, longest first (or rows by index, for comparison)
+    rc = from_cuda(order_mode == 1 ? launch_natural_order(items, order, s)
+                                   : launch_item_order(row_ptr, BH, nb, head_rank, order, s));
+    if (rc != FVATTN_OK) return rc;
     if ((rc = from_cuda(cudaMemsetAsync(counter, 0, sizeof(int), s))) != FVATTN_OK) return rc;
 
     AttnLaunch a{};
@@ -262,6 +265,8 @@ static int sparse_fwd_impl(const void *Q, const void *K, const void *V, const in
     const int64_t max_grid = static_cast<int64_t>(attn_ctas_per_sm()) * info.sms;
     a.grid = static_cast<int>(items < max_grid ? items : max_grid);
     a.test_stall = test_stall;
+    a.cta_busy_ns = reinterpret_cast<long long *>(cta_busy_ns);
+    if (grid_out) *grid_out = a.grid;
     return from_cuda(launch_sparse_attn(a, d, block, s));
 }
 
@@ -278,6 +283,17 @@ int fvattn_test_sparse_fwd_stall(const void *Q, const void *K, const void *V, co
                                  fvattn_stream_t stream) {
     return sparse_fwd_impl(Q, K, V, row_ptr, col_idx, B, H, N, d, block, causal, O, LSE, workspace, ws_bytes,
                            dev_status, stream, 1);
+}
+
+int fvattn_sparse_fwd_profiled(const void *Q, const void *K, const void *V, const int32_t *row_ptr,
+                               const int32_t *col_idx, int B, int H, int N, int d, int block, int causal, void *O,
+                               float *LSE, void *workspace, size_t ws_bytes, int32_t *dev_status, int order_mode,
+                               int64_t *cta_busy_ns, int *grid, fvattn_stream_t stream) {
+    if (order_mode != 0 && order_mode != 1) return FVATTN_ERR_INVALID_ARG;
+    if (!cta_busy_ns || !grid) return FVATTN_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(cta_busy_ns) & 7u) return FVATTN_ERR_ALIGNMENT;
+    return sparse_fwd_impl(Q, K, V, row_ptr, col_idx, B, H, N, d, block, causal, O, LSE, workspace, ws_bytes,
+                           dev_status, stream, 0, order_mode, cta_busy_ns, grid);
 }
 
 int fvattn_attention_host(const void *hQ, const void *hK, const void *hV, int B, int H, int N, int d, int block,

@@ -108,7 +108,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                            const int32_t *__restrict__ col_idx, const int32_t *__restrict__ order, int n_items,
                            int *__restrict__ work_counter, int N, int nb, int causal, float scale_log2,
                            __nv_bfloat16 *__restrict__ O, float *__restrict__ LSE, int32_t *dev_status,
-                           int test_stall) {
+                           int test_stall, long long *__restrict__ cta_busy_ns) {
     using C = Cfg<D, BS>;
     constexpr int NST = C::NST;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -148,6 +148,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = bar->tmem_base;
+    long long t_start = 0;  // global timer (ns) when this CTA starts its items, if busy times are asked for
+    if (cta_busy_ns && threadIdx.x == 0) asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_start));
 
     if (warp == kTmaWarp) {
         // ------------------------------------------------------------ producer
@@ -477,7 +479,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    if (cta_busy_ns && threadIdx.x == 0) {
+        long long t_end;
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_end));
+        cta_busy_ns[blockIdx.x] = t_end - t_start;
+    }
     if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
+}
+
+// Natural order (rows by index), the comparison point for the load-imbalance factor.
+__global__ void natural_order_kernel(int64_t n, int32_t *__restrict__ order) {
+    for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+        order[i] = static_cast<int32_t>(i);
 }
 
 // ------------------------------------------------------------- work order
@@ -582,6 +596,12 @@ cudaError_t launch_item_order(const int32_t *row_ptr, int64_t BH, int nb, int32_
     return cudaGetLastError();
 }
 
+cudaError_t launch_natural_order(int64_t n, int32_t *order, cudaStream_t stream) {
+    const int grid = static_cast<int>(n / 256 + 1 < 1024 ? n / 256 + 1 : 1024);
+    natural_order_kernel<<<grid, 256, 0, stream>>>(n, order);
+    return cudaGetLastError();
+}
+
 template <int D, int BS>
 static cudaError_t launch_t(const AttnLaunch &a, cudaStream_t stream) {
     auto kern = sparse_attn_fwd_kernel<D, BS>;
@@ -590,7 +610,7 @@ static cudaError_t launch_t(const AttnLaunch &a, cudaStream_t stream) {
     kern<<<a.grid, kThreads, Cfg<D, BS>::SMEM_BYTES, stream>>>(
         *a.tmap_k, *a.tmap_v, static_cast<const __nv_bfloat16 *>(a.Q), a.row_ptr, a.col_idx, a.order, a.n_items,
         a.work_counter, a.N, a.nb, a.causal, a.scale_log2, static_cast<__nv_bfloat16 *>(a.O), a.LSE, a.dev_status,
-        a.test_stall);
+        a.test_stall, a.cta_busy_ns);
     return cudaGetLastError();
 }
 

@@ -20,6 +20,7 @@ struct AttnLaunch {
     int32_t *dev_status;
     int grid;
     int test_stall;     // nonzero only from the test hook: one bounded wait runs out
+    long long *cta_busy_ns;  // per-CTA busy time (global timer, ns), or null
 };
 
 int attn_smem_bytes(int d, int bs);
@@ -29,6 +30,8 @@ int64_t attn_num_items(int64_t BH, int nb);
 // a head by block count); head_rank[BH] is scratch.  B*H <= 4096, nb <= 4096.
 cudaError_t launch_item_order(const int32_t *row_ptr, int64_t BH, int nb, int32_t *head_rank, int32_t *order,
                               cudaStream_t stream);
+// order[i] = i: rows in index order (the comparison point for the load balance).
+cudaError_t launch_natural_order(int64_t n, int32_t *order, cudaStream_t stream);
 int attn_ctas_per_sm();  // resident CTAs per SM the launch grid is sized for
 cudaError_t launch_sparse_attn(const AttnLaunch &a, int d, int bs, cudaStream_t stream);
 
