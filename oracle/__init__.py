@@ -48,7 +48,9 @@ def _load():
         lib.oracle_attn_rows.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, P, P, P, i64, P, P, i32]
         lib.oracle_attn_tiled.argtypes = lib.oracle_attn_rows.argtypes
         lib.oracle_lpt_order.argtypes = [P, i64, P]
-        for f in ("oracle_pool", "oracle_route", "oracle_attn_rows", "oracle_attn_tiled", "oracle_lpt_order"):
+        lib.oracle_attn_bwd.argtypes = [P, P, P, P, i32, i32, i32, i32, i32, i32, P, P, P, P, P, i32]
+        for f in ("oracle_pool", "oracle_route", "oracle_attn_rows", "oracle_attn_tiled", "oracle_lpt_order",
+                  "oracle_attn_bwd"):
             getattr(lib, f).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -141,6 +143,26 @@ def attn_rows(Q, K, V, bs, causal, row_ptr, col_idx, tokens, nthreads=None):
 def attn_tiled(Q, K, V, bs, causal, row_ptr, col_idx, tokens, nthreads=None):
     """Block-by-block online softmax; equal to :func:`attn_rows` up to rounding."""
     return _attn(_load().oracle_attn_tiled, Q, K, V, bs, causal, row_ptr, col_idx, tokens, nthreads)
+
+
+def attn_bwd(Q, K, V, dO, bs, causal, row_ptr, col_idx, nthreads=None):
+    """Gradients of sum(dO * O) for the attention of :func:`attn_rows` (all bf16 bit
+    patterns [B,H,N,d]). Returns dQ, dK, dV as fp64 [B,H,N,d]."""
+    Q, K, V, dO = _bits(Q), _bits(K), _bits(V), _bits(dO)
+    B, H, N, d = Q.shape
+    row_ptr = np.ascontiguousarray(row_ptr, dtype=np.int32)
+    col_idx = np.ascontiguousarray(col_idx, dtype=np.int32)
+    if col_idx.size == 0:
+        col_idx = np.zeros(1, dtype=np.int32)
+    dQ = np.empty((B, H, N, d), dtype=np.float64)
+    dK = np.empty_like(dQ)
+    dV = np.empty_like(dQ)
+    rc = _load().oracle_attn_bwd(_ptr(Q), _ptr(K), _ptr(V), _ptr(dO), B, H, N, d, bs, 1 if causal else 0,
+                                 _ptr(row_ptr), _ptr(col_idx), _ptr(dQ), _ptr(dK), _ptr(dV),
+                                 nthreads or default_threads())
+    if rc != 0:
+        raise ValueError("oracle_attn_bwd failed")
+    return dQ, dK, dV
 
 
 def lpt_order(row_ptr: np.ndarray) -> np.ndarray:

@@ -37,6 +37,9 @@
  *   attn_rows   high-precision Decimal brute force on tiny inputs, closed
  *               forms (single key, K = 0 mean of V, constant V)
  *   attn_tiled  equals attn_rows (the "exact" tiling identity of [FA])
+ *   attn_bwd    central finite differences of a numpy fp64 brute-force forward,
+ *               fp64 torch autograd of dense attention, and the dense-case
+ *               identities sum_u dK_u = 0 and sum_u dV_u = sum_t dO_t
  *   lpt_order   brute-force sort on small inputs
  */
 #include <math.h>
@@ -478,5 +481,116 @@ int oracle_lpt_order(const int32_t *row_ptr, int64_t rows, int32_t *order) {
     qsort(w, (size_t)rows, sizeof(work_item), by_count_desc_id_asc);
     for (int64_t r = 0; r < rows; ++r) order[r] = (int32_t)w[r].id;
     free(w);
+    return 0;
+}
+
+/* ---------------------------------------- attention gradients, row by row */
+/*
+ * Gradients of the loss L = sum_t dO_t . O_t for the attention of attn_rows
+ * (the training use the [FA] review measures in §Experiments 1 "Training
+ * Efficiency" needs them; the pages print no formulas, so these are the plain
+ * derivatives of the definition above).  Per query token t with allowed keys
+ * u (its CSR row's blocks, u < N, u <= t if causal), s_u = q_t . k_u / sqrt(d),
+ * P_u = softmax(s)_u, O_t = sum_u P_u v_u:
+ *   dV_u += P_u dO_t
+ *   dP_u  = dO_t . v_u,   D_t = dO_t . O_t,   dS_u = P_u (dP_u - D_t)
+ *   dQ_t  = sum_u dS_u k_u / sqrt(d)
+ *   dK_u += dS_u q_t / sqrt(d)
+ * One thread owns one (batch, head): all its accumulations are private, and
+ * every sum runs over t and u in index order.  A token with no allowed key
+ * contributes nothing (its O is 0).
+ */
+typedef struct {
+    const uint16_t *Q, *K, *V, *dO;
+    int N, d, bs, causal;
+    int64_t nb;
+    const int32_t *row_ptr, *col_idx;
+    double *dQ, *dK, *dV;
+    double scale;
+} bwd_ctx;
+
+static void attn_bwd_range(void *vctx, int64_t begin, int64_t end) {
+    bwd_ctx *c = (bwd_ctx *)vctx;
+    int d = c->d;
+    int64_t cap = c->nb * c->bs;
+    double *q = (double *)malloc(sizeof(double) * d);
+    double *go = (double *)malloc(sizeof(double) * d);
+    double *o = (double *)malloc(sizeof(double) * d);
+    double *p = (double *)malloc(sizeof(double) * cap);
+    int64_t *u_of = (int64_t *)malloc(sizeof(int64_t) * cap);
+    if (!q || !go || !o || !p || !u_of) goto out;
+    for (int64_t bh = begin; bh < end; ++bh) {
+        const int64_t base = bh * c->N * d;
+        for (int64_t i = 0; i < (int64_t)c->N * d; ++i) {
+            c->dQ[base + i] = 0.0;
+            c->dK[base + i] = 0.0;
+            c->dV[base + i] = 0.0;
+        }
+        for (int64_t t = 0; t < c->N; ++t) {
+            int64_t row = bh * c->nb + t / c->bs;
+            for (int ch = 0; ch < d; ++ch) {
+                q[ch] = bf16_bits_to_double(c->Q[base + t * d + ch]);
+                go[ch] = bf16_bits_to_double(c->dO[base + t * d + ch]);
+            }
+            /* scores and softmax over the allowed keys */
+            int64_t n = 0;
+            double m = -INFINITY;
+            for (int32_t e = c->row_ptr[row]; e < c->row_ptr[row + 1]; ++e) {
+                int64_t kb = c->col_idx[e];
+                for (int64_t u = kb * c->bs; u < (kb + 1) * c->bs && u < c->N; ++u) {
+                    if (c->causal && u > t) continue;
+                    double dot = 0.0;
+                    for (int ch = 0; ch < d; ++ch) dot = dot + q[ch] * bf16_bits_to_double(c->K[base + u * d + ch]);
+                    p[n] = dot * c->scale;
+                    u_of[n] = u;
+                    if (p[n] > m) m = p[n];
+                    ++n;
+                }
+            }
+            if (n == 0) continue;
+            double z = 0.0;
+            for (int64_t a = 0; a < n; ++a) {
+                p[a] = exp(p[a] - m);
+                z = z + p[a];
+            }
+            for (int64_t a = 0; a < n; ++a) p[a] = p[a] / z;
+            /* O_t and D_t */
+            for (int ch = 0; ch < d; ++ch) o[ch] = 0.0;
+            for (int64_t a = 0; a < n; ++a)
+                for (int ch = 0; ch < d; ++ch) o[ch] = o[ch] + p[a] * bf16_bits_to_double(c->V[base + u_of[a] * d + ch]);
+            double D = 0.0;
+            for (int ch = 0; ch < d; ++ch) D = D + go[ch] * o[ch];
+            /* the gradients */
+            double *dq = c->dQ + base + t * d;
+            for (int64_t a = 0; a < n; ++a) {
+                const int64_t u = u_of[a];
+                double dp = 0.0;
+                for (int ch = 0; ch < d; ++ch) dp = dp + go[ch] * bf16_bits_to_double(c->V[base + u * d + ch]);
+                const double ds = p[a] * (dp - D);
+                double *dv = c->dV + base + u * d, *dk = c->dK + base + u * d;
+                for (int ch = 0; ch < d; ++ch) {
+                    dv[ch] = dv[ch] + p[a] * go[ch];
+                    dq[ch] = dq[ch] + ds * bf16_bits_to_double(c->K[base + u * d + ch]) * c->scale;
+                    dk[ch] = dk[ch] + ds * q[ch] * c->scale;
+                }
+            }
+        }
+    }
+out:
+    free(q);
+    free(go);
+    free(o);
+    free(p);
+    free(u_of);
+}
+
+int oracle_attn_bwd(const uint16_t *Q, const uint16_t *K, const uint16_t *V, const uint16_t *dO, int B, int H, int N,
+                    int d, int bs, int causal, const int32_t *row_ptr, const int32_t *col_idx, double *dQ, double *dK,
+                    double *dV, int nthreads) {
+    if (!Q || !K || !V || !dO || !row_ptr || !col_idx || !dQ || !dK || !dV) return -1;
+    if (B < 1 || H < 1 || N < 1 || d < 1 || bs < 1) return -1;
+    bwd_ctx c = {Q, K, V, dO, N, d, bs, causal, num_blocks(N, bs), row_ptr, col_idx, dQ, dK, dV,
+                 1.0 / sqrt((double)d)};
+    parallel_for((int64_t)B * H, nthreads, attn_bwd_range, &c);
     return 0;
 }

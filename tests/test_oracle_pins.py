@@ -413,3 +413,86 @@ def test_bf16_rounding_is_nearest_even():
     assert back[0] == 1.0 and back[1] == 1.0          # tie rounds to even
     assert back[2] == 1.0 + 2**-6                       # tie rounds up to even
     assert back[3] == -2.5 and back[4] == 0.0
+
+
+# ------------------------------------------------------- attention gradients
+
+def numpy_forward(Qf, Kf, Vf, bs, causal, row_ptr, col_idx):
+    """Plain fp64 numpy statement of the masked attention forward (brute force)."""
+    B, H, N, d = Qf.shape
+    nb = -(-N // bs)
+    O = np.zeros_like(Qf)
+    for b in range(B):
+        for h in range(H):
+            for t in range(N):
+                row = (b * H + h) * nb + t // bs
+                keys = [u for kb in col_idx[row_ptr[row]:row_ptr[row + 1]]
+                        for u in range(kb * bs, min((kb + 1) * bs, N)) if not (causal and u > t)]
+                if not keys:
+                    continue
+                s = Kf[b, h, keys] @ Qf[b, h, t] / math.sqrt(d)
+                w = np.exp(s - s.max())
+                O[b, h, t] = (w / w.sum()) @ Vf[b, h, keys]
+    return O
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_attn_bwd_matches_finite_differences(oracle_mod, causal):
+    """Directional derivatives of L = sum(dO * O) by central differences of an
+    independent fp64 forward equal the oracle's gradients."""
+    rng = np.random.default_rng(7 + causal)
+    B, H, N, d, bs = 1, 2, 70, 16, 32
+    nb = -(-N // bs)
+    row_ptr, col_idx = random_csr(rng, B * H * nb, nb, p_keep=0.6, allow_empty=True)
+    Q, K, V, dO = (rand_bf16(rng, (B, H, N, d)) for _ in range(4))
+    dQ, dK, dV = oracle_mod.attn_bwd(Q, K, V, dO, bs, causal, row_ptr, col_idx)
+    Qf, Kf, Vf, dOf = fvals(Q), fvals(K), fvals(V), fvals(dO)
+
+    def loss(Qx, Kx, Vx):
+        return float(np.sum(dOf * numpy_forward(Qx, Kx, Vx, bs, causal, row_ptr, col_idx)))
+
+    h = 1e-5
+    for which, grad in (("Q", dQ), ("K", dK), ("V", dV)):
+        for _ in range(3):
+            r = rng.standard_normal((B, H, N, d))
+            args_p = [Qf, Kf, Vf]
+            args_m = [Qf, Kf, Vf]
+            i = "QKV".index(which)
+            args_p[i] = args_p[i] + h * r
+            args_m[i] = args_m[i] - h * r
+            fd = (loss(*args_p) - loss(*args_m)) / (2 * h)
+            an = float(np.sum(grad * r))
+            assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), (which, fd, an)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_attn_bwd_dense_matches_torch_autograd(oracle_mod, causal):
+    """With every block selected the oracle's gradients equal fp64 autograd of
+    softmax(QK^T/sqrt(d))V (lower-triangular mask if causal)."""
+    import torch
+    rng = np.random.default_rng(11 + causal)
+    B, H, N, d, bs = 1, 2, 96, 16, 32
+    nb = N // bs
+    row_ptr, col_idx = oracle_mod.dense_csr(B, H, N, bs, causal)
+    Q, K, V, dO = (rand_bf16(rng, (B, H, N, d)) for _ in range(4))
+    dQ, dK, dV = oracle_mod.attn_bwd(Q, K, V, dO, bs, causal, row_ptr, col_idx)
+    q, k, v = (torch.tensor(fvals(x), dtype=torch.float64, requires_grad=True) for x in (Q, K, V))
+    s = q @ k.transpose(-1, -2) / math.sqrt(d)
+    if causal:
+        s = s.masked_fill(torch.triu(torch.ones(N, N, dtype=torch.bool), 1), float("-inf"))
+    o = torch.softmax(s, dim=-1) @ v
+    (o * torch.tensor(fvals(dO), dtype=torch.float64)).sum().backward()
+    for mine, ref in ((dQ, q.grad), (dK, k.grad), (dV, v.grad)):
+        assert np.max(np.abs(mine - ref.numpy())) < 1e-11
+
+
+def test_attn_bwd_dense_identities(oracle_mod):
+    """Dense, non-causal: every softmax row sums to one and is invariant to a common
+    shift of the keys, so sum_u dV_u = sum_t dO_t and sum_u dK_u = 0 per head."""
+    rng = np.random.default_rng(13)
+    B, H, N, d, bs = 2, 2, 100, 8, 32
+    row_ptr, col_idx = oracle_mod.dense_csr(B, H, N, bs, False)
+    Q, K, V, dO = (rand_bf16(rng, (B, H, N, d)) for _ in range(4))
+    dQ, dK, dV = oracle_mod.attn_bwd(Q, K, V, dO, bs, False, row_ptr, col_idx)
+    assert np.max(np.abs(dV.sum(axis=2) - fvals(dO).sum(axis=2))) < 1e-10
+    assert np.max(np.abs(dK.sum(axis=2))) < 1e-10
