@@ -229,6 +229,37 @@ FVATTN_API int fvattn_test_sparse_fwd_stall(const void *Q, const void *K, const 
                                             int causal, void *O, float *LSE, void *workspace, size_t ws_bytes,
                                             int32_t *dev_status, fvattn_stream_t stream);
 
+/* Device workspace fvattn_sparse_bwd needs, in bytes (0 on bad arguments). */
+FVATTN_API size_t fvattn_bwd_workspace_bytes(int B, int H, int N, int block);
+
+/*
+ * fvattn_sparse_bwd -- gradients of the block-sparse attention of
+ * fvattn_sparse_fwd.  The FlashAttention review measures training with the
+ * fused kernel (§Experiments 1 "Training Efficiency") without printing the
+ * backward pass; these are the plain derivatives of L = sum(dO * O) with P
+ * recomputed from the LSE the forward returned:
+ *   D_t = dO_t . O_t,  P = exp(S - LSE),  dS = P * (dO V^T - D),
+ *   dQ = dS K / sqrt(d),  dK = dS^T Q / sqrt(d),  dV = P^T dO,
+ * every sum restricted to the key tokens the CSR mask allows (u < N, u <= t if
+ * causal), exactly as in the forward.
+ *
+ *   Q, K, V, O, dO  bf16 [B,H,N,d], read only (O and LSE from fvattn_sparse_fwd).
+ *   LSE             fp32 [B,H,N], read only.
+ *   row_ptr, col_idx  the CSR block mask of the forward (ascending columns).
+ *   dQ, dK, dV      out, bf16 [B,H,N,d] (fp32 accumulation in tensor memory).
+ *   workspace       >= fvattn_bwd_workspace_bytes(B,H,N,block).
+ * block must be 128 and d 64 or 128 (else FVATTN_ERR_UNSUPPORTED); B*H <= 4096.
+ * Work: D; the transpose of the mask (key block -> the query blocks that
+ * selected it); a dQ pass over the CSR rows and a dK/dV pass over the key
+ * blocks, both on tcgen05 with accumulators in tensor memory and longest-first
+ * persistent grids.  A malformed CSR sets *dev_status = FVATTN_ERR_BAD_CSR and
+ * leaves the gradients unspecified.  Asynchronous on `stream`.
+ */
+FVATTN_API int fvattn_sparse_bwd(const void *Q, const void *K, const void *V, const void *O, const float *LSE,
+                                 const void *dO, const int32_t *row_ptr, const int32_t *col_idx, int B, int H, int N,
+                                 int d, int block, int causal, void *dQ, void *dK, void *dV, void *workspace,
+                                 size_t ws_bytes, int32_t *dev_status, fvattn_stream_t stream);
+
 /*
  * fvattn_sparse_fwd_profiled -- fvattn_sparse_fwd that also reports how busy
  * each CTA of its persistent grid was, for the load-imbalance factor

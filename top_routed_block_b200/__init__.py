@@ -69,6 +69,8 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         "fvattn_sparse_fwd_noalloc": (I, [P, P, P, P, P, I, I, I, I, I, I, P, P, P, P]),
         "fvattn_test_sparse_fwd_stall": (I, [P, P, P, P, P, I, I, I, I, I, I, P, P, P, SZ, P, P]),
         "fvattn_sparse_fwd_profiled": (I, [P, P, P, P, P, I, I, I, I, I, I, P, P, P, SZ, P, I, P, P, P]),
+        "fvattn_bwd_workspace_bytes": (SZ, [I, I, I, I]),
+        "fvattn_sparse_bwd": (I, [P, P, P, P, P, P, P, P, I, I, I, I, I, I, P, P, P, P, SZ, P, P]),
         "fvattn_attention_host": (I, [P, P, P, I, I, I, I, I, D, I, P, P, P, P, P, P, P, P, P, I64, P, P, SZ, P, SZ,
                                       P, P]),
     }
@@ -240,6 +242,36 @@ def fvattn_sparse_fwd_profiled(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor
                                         _stream_ptr(stream))
     _check(rc, "fvattn_sparse_fwd_profiled")
     return O, LSE, dev_status, busy[: grid.value]
+
+
+def fvattn_bwd_workspace_bytes(B: int, H: int, N: int, block: int) -> int:
+    return int(load_library().fvattn_bwd_workspace_bytes(B, H, N, block))
+
+
+def fvattn_sparse_bwd(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, O: torch.Tensor, LSE: torch.Tensor,
+                      dO: torch.Tensor, row_ptr: torch.Tensor, col_idx: torch.Tensor, block: int,
+                      causal: bool = False, *, stream=None, dQ: torch.Tensor | None = None,
+                      dK: torch.Tensor | None = None, dV: torch.Tensor | None = None,
+                      workspace: torch.Tensor | None = None, dev_status: torch.Tensor | None = None):
+    """Gradients of the block-sparse attention; returns (dQ, dK, dV bf16, dev_status)."""
+    lib = load_library()
+    B, H, N, d = _shape(Q)
+    for t in (K, V, O, dO):
+        if tuple(t.shape) != (B, H, N, d) or t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError("K, V, O and dO must match Q")
+    dev = Q.device
+    dQ = torch.empty_like(Q) if dQ is None else dQ
+    dK = torch.empty_like(Q) if dK is None else dK
+    dV = torch.empty_like(Q) if dV is None else dV
+    if dev_status is None:
+        dev_status = torch.zeros(1, dtype=torch.int32, device=dev)
+    if workspace is None:
+        workspace = _empty_bytes(fvattn_bwd_workspace_bytes(B, H, N, block), dev)
+    rc = lib.fvattn_sparse_bwd(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(LSE), _ptr(dO), _ptr(row_ptr), _ptr(col_idx),
+                               B, H, N, d, block, 1 if causal else 0, _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(workspace),
+                               workspace.numel(), _ptr(dev_status), _stream_ptr(stream))
+    _check(rc, "fvattn_sparse_bwd")
+    return dQ, dK, dV, dev_status
 
 
 def fvattn_sparse_fwd_noalloc(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, row_ptr: torch.Tensor,

@@ -11,6 +11,7 @@
 #include <mutex>
 
 #include "fvattn.h"
+#include "attn_bwd.cuh"
 #include "attn_fwd.cuh"
 #include "common.cuh"
 #include "lpt.cuh"
@@ -112,6 +113,26 @@ FwdWorkspace fwd_layout(int64_t items, int64_t BH) {
 }
 
 int from_cuda(cudaError_t e) { return e == cudaSuccess ? FVATTN_OK : FVATTN_ERR_CUDA; }
+
+struct BwdWorkspace {
+    size_t D, col_ptr, csc_idx, order_q, order_k, head_rank, counters, total;
+};
+
+// rows = B*H*nb CSR rows (= key-block columns); csc capacity = the worst case B*H*nb^2.
+BwdWorkspace bwd_layout(int64_t BH, int N, int nb) {
+    BwdWorkspace w{};
+    Carver c;
+    const int64_t rows = BH * nb;
+    w.D = c.take<float>(static_cast<size_t>(BH) * N);
+    w.col_ptr = c.take<int32_t>(static_cast<size_t>(rows) + 1);
+    w.csc_idx = c.take<int32_t>(static_cast<size_t>(rows) * nb);
+    w.order_q = c.take<int32_t>(static_cast<size_t>(rows));
+    w.order_k = c.take<int32_t>(static_cast<size_t>(rows));
+    w.head_rank = c.take<int32_t>(static_cast<size_t>(BH));
+    w.counters = c.take<int32_t>(64);
+    w.total = align_up(c.off, 256);
+    return w;
+}
 
 // st[2] keeps the first error of st[0] (routing) and st[1] (attention) over successive calls.
 __global__ void status_merge_kernel(int32_t *st) {
@@ -294,6 +315,93 @@ int fvattn_sparse_fwd_profiled(const void *Q, const void *K, const void *V, cons
     if (reinterpret_cast<uintptr_t>(cta_busy_ns) & 7u) return FVATTN_ERR_ALIGNMENT;
     return sparse_fwd_impl(Q, K, V, row_ptr, col_idx, B, H, N, d, block, causal, O, LSE, workspace, ws_bytes,
                            dev_status, stream, 0, order_mode, cta_busy_ns, grid);
+}
+
+size_t fvattn_bwd_workspace_bytes(int B, int H, int N, int block) {
+    if (B < 1 || H < 1 || N < 1 || block != 128) return 0;
+    const int64_t nb = ceil_div(N, block);
+    const int64_t BH = static_cast<int64_t>(B) * H;
+    if (nb > kMaxCount || BH > kMaxHeads) return 0;
+    return bwd_layout(BH, N, static_cast<int>(nb)).total;
+}
+
+int fvattn_sparse_bwd(const void *Q, const void *K, const void *V, const void *O, const float *LSE, const void *dO,
+                      const int32_t *row_ptr, const int32_t *col_idx, int B, int H, int N, int d, int block,
+                      int causal, void *dQ, void *dK, void *dV, void *workspace, size_t ws_bytes,
+                      int32_t *dev_status, fvattn_stream_t stream) {
+    int rc = check_shape(B, H, N, d, block);
+    if (rc != FVATTN_OK) return rc;
+    if (block != 128) return FVATTN_ERR_UNSUPPORTED;
+    if (!Q || !K || !V || !O || !LSE || !dO || !row_ptr || !col_idx || !dQ || !dK || !dV || !workspace ||
+        !dev_status)
+        return FVATTN_ERR_INVALID_ARG;
+    if (causal != 0 && causal != 1) return FVATTN_ERR_INVALID_ARG;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(dO) || !aligned16(dQ) ||
+        !aligned16(dK) || !aligned16(dV) || !aligned16(workspace))
+        return FVATTN_ERR_ALIGNMENT;
+    if ((reinterpret_cast<uintptr_t>(row_ptr) | reinterpret_cast<uintptr_t>(col_idx) |
+         reinterpret_cast<uintptr_t>(LSE) | reinterpret_cast<uintptr_t>(dev_status)) & 3u)
+        return FVATTN_ERR_ALIGNMENT;
+    const int64_t BH = static_cast<int64_t>(B) * H;
+    if (BH > kMaxHeads) return FVATTN_ERR_UNSUPPORTED;
+    const int nb = static_cast<int>(ceil_div(N, block));
+    if (ws_bytes < fvattn_bwd_workspace_bytes(B, H, N, block)) return FVATTN_ERR_CAPACITY;
+    if ((rc = check_device()) != FVATTN_OK) return rc;
+    DeviceInfo info;
+    if (!device_info(&info)) return FVATTN_ERR_CUDA;
+    const int64_t rows = BH * nb;
+    const BwdWorkspace w = bwd_layout(BH, N, nb);
+    char *ws = static_cast<char *>(workspace);
+    float *Dv = reinterpret_cast<float *>(ws + w.D);
+    int32_t *col_ptr = reinterpret_cast<int32_t *>(ws + w.col_ptr);
+    int32_t *csc_idx = reinterpret_cast<int32_t *>(ws + w.csc_idx);
+    int32_t *order_q = reinterpret_cast<int32_t *>(ws + w.order_q);
+    int32_t *order_k = reinterpret_cast<int32_t *>(ws + w.order_k);
+    int32_t *head_rank = reinterpret_cast<int32_t *>(ws + w.head_rank);
+    int *counters = reinterpret_cast<int *>(ws + w.counters);
+
+    CUtensorMap mq, mk, mv, mdo;
+    if (!make_map(&mq, Q, BH, N, d, block) || !make_map(&mk, K, BH, N, d, block) ||
+        !make_map(&mv, V, BH, N, d, block) || !make_map(&mdo, dO, BH, N, d, block))
+        return FVATTN_ERR_CUDA;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if ((rc = from_cuda(cudaMemsetAsync(dev_status, 0, sizeof(int32_t), s))) != FVATTN_OK) return rc;
+    if ((rc = from_cuda(cudaMemsetAsync(counters, 0, 2 * sizeof(int), s))) != FVATTN_OK) return rc;
+    if ((rc = from_cuda(launch_bwd_rowdot(O, dO, BH * N, d, Dv, s))) != FVATTN_OK) return rc;
+    if ((rc = from_cuda(launch_csc(row_ptr, col_idx, BH, nb, col_ptr, csc_idx, dev_status, s))) != FVATTN_OK)
+        return rc;
+    // both queues head-major, longest first: rows by selected blocks, key blocks by selecting rows
+    if ((rc = from_cuda(launch_item_order(row_ptr, BH, nb, head_rank, order_q, s))) != FVATTN_OK) return rc;
+    if ((rc = from_cuda(launch_item_order(col_ptr, BH, nb, head_rank, order_k, s))) != FVATTN_OK) return rc;
+
+    BwdLaunch a{};
+    a.tmap_q = &mq;
+    a.tmap_k = &mk;
+    a.tmap_v = &mv;
+    a.tmap_do = &mdo;
+    a.Q = Q;
+    a.dO = dO;
+    a.LSE = LSE;
+    a.D = Dv;
+    a.row_ptr = row_ptr;
+    a.col_idx = col_idx;
+    a.col_ptr = col_ptr;
+    a.csc_idx = csc_idx;
+    a.order_q = order_q;
+    a.order_k = order_k;
+    a.n_items = static_cast<int>(rows);
+    a.counters = counters;
+    a.N = N;
+    a.nb = nb;
+    a.causal = causal;
+    a.scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(d)));
+    a.dQ = dQ;
+    a.dK = dK;
+    a.dV = dV;
+    a.dev_status = dev_status;
+    a.grid = static_cast<int>(rows < info.sms ? rows : info.sms);
+    if ((rc = from_cuda(launch_bwd_dq(a, d, s))) != FVATTN_OK) return rc;
+    return from_cuda(launch_bwd_dkdv(a, d, s));
 }
 
 int fvattn_attention_host(const void *hQ, const void *hK, const void *hV, int B, int H, int N, int d, int block,
