@@ -362,6 +362,37 @@ def run_ours(args, w, rank, world, local):
         ms_, lif, mx, g = sorted(runs)[1]  # the median run by time
         balance[name] = {"lif": lif, "call_ms": ms_, "max_cta_busy_ms": mx, "ctas": g}
 
+    # Backward (outside the timed region): gradients of the same attention for a random dO.
+    bwd = None
+    if w.bs == 128:
+        plan.run_fwd(dQ, dK, dV, w.causal, stream=stream)
+        gen = torch.Generator(device=dev).manual_seed(1234)
+        dO = torch.randn(dQ.shape, device=dev, dtype=torch.float32, generator=gen).to(torch.bfloat16)
+        ws_b = torch.empty(fv.fvattn_bwd_workspace_bytes(w.B, w.H, w.N, w.bs), dtype=torch.uint8, device=dev)
+        gQ, gK, gV = torch.empty_like(dQ), torch.empty_like(dQ), torch.empty_like(dQ)
+        st_b = torch.zeros(1, dtype=torch.int32, device=dev)
+
+        def bwd_call():
+            fv.fvattn_sparse_bwd(dQ, dK, dV, plan.O, plan.LSE, dO, plan.route.row_ptr, plan.route.col_idx, w.bs,
+                                 w.causal, stream=stream, dQ=gQ, dK=gK, dV=gV, workspace=ws_b, dev_status=st_b)
+        for _ in range(2):
+            bwd_call()
+        torch.cuda.synchronize(dev)
+        fv.check_status(st_b, "fvattn_sparse_bwd")
+        reps = 5
+        a.record(stream)
+        for _ in range(reps):
+            bwd_call()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        fv.check_status(st_b, "fvattn_sparse_bwd")
+        bwd_ms = a.elapsed_time(b) / reps
+        bwd = {"ms": bwd_ms, "tflops_effective": 2.5 * flops / (bwd_ms * 1e-3) / 1e12,
+               "note": "effective = 2.5 x the forward's 4*block^2*d*nnz (five block GEMMs); the kernels run seven "
+                       "(S and dP are recomputed in both the dQ and the dK/dV pass); mean of 5 calls after 2, "
+                       "outside the timed region"}
+        del gQ, gK, gV, ws_b, dO
+
     if rank != 0:
         return
     peaks, peak_src = load_peaks()
@@ -399,6 +430,7 @@ def run_ours(args, w, rank, world, local):
         "load_balance": dict(balance, note="LIF = max / mean busy time over the CTAs of the persistent grid "
                                            "(global timer, one call each); lpt = the head-major longest-first "
                                            "queue fvattn_sparse_fwd uses, natural = rows in index order"),
+        "bwd": None if bwd is None else dict(bwd, frac_of_sustained=bwd["tflops_effective"] / peak),
         "mufu": {"exp_per_s": float(nnz) * w.bs * w.bs / (attn_ms * 1e-3),
                  "ceiling_at_max_clock": 16.0 * sms * float(peaks.get("sm_max_mhz", 1965.0)) * 1e6,
                  "frac": float(nnz) * w.bs * w.bs / (attn_ms * 1e-3)
