@@ -412,39 +412,43 @@ __global__ void __launch_bounds__(kThreads, 1)
                     break;
                 }
                 tc_fence_after();
-                float p[BS];
-                {
-                    uint32_t v[32];
+                // P = exp(S / sqrt(d) - LSE) in fp32, in place
+                uint32_t v[BS];
 #pragma unroll
-                    for (int c0 = 0; c0 < BS; c0 += 32) {
-                        tmem_ld32(tmem + lane_base + C::T_S + c0, v);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int c = 0; c < 32; ++c)
-                            p[c0 + c] = (c0 + c < lim) ? ex2_approx(fmaf(__uint_as_float(v[c]), scale_log2, -lse2))
-                                                       : 0.0f;
-                    }
-                }
+                for (int c0 = 0; c0 < BS; c0 += 32)
+                    tmem_ld32(tmem + lane_base + C::T_S + c0, *reinterpret_cast<uint32_t(*)[32]>(&v[c0]));
+                tmem_wait_ld();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bar->s_free);  // S may be overwritten by the next block
+                if (__all_sync(0xffffffffu, lim >= BS)) {
+#pragma unroll
+                    for (int c = 0; c < BS; ++c)
+                        v[c] = __float_as_uint(ex2_approx(fmaf(__uint_as_float(v[c]), scale_log2, -lse2)));
+                } else {
+#pragma unroll
+                    for (int c = 0; c < BS; ++c)
+                        v[c] = __float_as_uint(c < lim ? ex2_approx(fmaf(__uint_as_float(v[c]), scale_log2, -lse2))
+                                                       : 0.0f);
+                }
                 if (!mbar_wait(&bar->dp_full, tc & 1, abort_flag, dev_status)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                // dS = P (dP - D), as bf16 pairs into the dP columns
+                // dS = P (dP - D), as bf16 pairs into the dP columns (two halves of 64 columns)
 #pragma unroll
-                for (int c0 = 0; c0 < BS; c0 += 32) {
-                    uint32_t v[32];
-                    tmem_ld32(tmem + lane_base + C::T_DP + c0, v);
+                for (int h0 = 0; h0 < BS; h0 += 64) {
+                    uint32_t g[64];
+                    tmem_ld32(tmem + lane_base + C::T_DP + h0, *reinterpret_cast<uint32_t(*)[32]>(&g[0]));
+                    tmem_ld32(tmem + lane_base + C::T_DP + h0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&g[32]));
                     tmem_wait_ld();
-                    uint32_t w[16];
+                    uint32_t w[32];
 #pragma unroll
-                    for (int c = 0; c < 32; c += 2)
-                        w[c >> 1] = pack_bf16(p[c0 + c] * (__uint_as_float(v[c]) - Dt),
-                                              p[c0 + c + 1] * (__uint_as_float(v[c + 1]) - Dt));
-                    tmem_st16(tmem + lane_base + C::T_DP + c0 / 2, w);
+                    for (int c = 0; c < 64; c += 2)
+                        w[c >> 1] = pack_bf16(__uint_as_float(v[h0 + c]) * (__uint_as_float(g[c]) - Dt),
+                                              __uint_as_float(v[h0 + c + 1]) * (__uint_as_float(g[c + 1]) - Dt));
+                    tmem_st32(tmem + lane_base + C::T_DP + h0 / 2, w);
                 }
                 tmem_wait_st();
                 tc_fence_before();
@@ -505,7 +509,7 @@ struct KvCfg {
     static constexpr int NST = 4;
     static constexpr int OFF_RING = 2 * STAGE_BYTES;         // K, V of the item first
     static constexpr int OFF_META = OFF_RING + NST * STAGE_BYTES;
-    static constexpr int TILE_BYTES = OFF_META + 2 * 2 * kRowsM * 4;
+    static constexpr int TILE_BYTES = OFF_META + 3 * 2 * kRowsM * 4;
     static constexpr int SMEM_BYTES = TILE_BYTES + 1024 + 512;
     static constexpr uint32_t T_S = 0, T_DP = 128, T_DK = 256, T_DV = 384;
     static constexpr uint32_t IDESC_T = idesc_bf16_f32(kRowsM, kRowsM, 0, 0);  // S^T, dP^T: both K-major
@@ -514,7 +518,7 @@ struct KvCfg {
 
 struct KvBarriers {
     uint64_t ring_full[4], ring_empty[4];
-    uint64_t kv_full, kv_empty, st_full, dpt_full, p_full, ds_full, meta[2], acc_full, acc_empty;
+    uint64_t kv_full, kv_empty, st_full, dpt_full, p_full, ds_full, meta[3], acc_full, acc_empty;
     uint64_t sched_full[2], sched_empty[2];
     uint64_t drain;
     int4 sched_item[2];  // {column (bh*nb + j), list start, count, valid item}
@@ -538,7 +542,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t base_addr = smem_addr(smem_raw);
     unsigned char *smem = smem_raw + ((1024 - (base_addr & 1023)) & 1023);
     unsigned char *ring = smem + C::OFF_RING;
-    float *meta = reinterpret_cast<float *>(smem + C::OFF_META);  // [2 copies][LSE 128 | D 128]
+    float *meta = reinterpret_cast<float *>(smem + C::OFF_META);  // [3 copies][LSE 128 | D 128]
     KvBarriers *bar = reinterpret_cast<KvBarriers *>(smem + C::TILE_BYTES);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     volatile int *abort_flag = &bar->abort_flag;
@@ -555,8 +559,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(&bar->dpt_full, 1);
         mbar_init(&bar->p_full, 4);
         mbar_init(&bar->ds_full, 4);
-        mbar_init(&bar->meta[0], 4);
-        mbar_init(&bar->meta[1], 4);
+        for (int x = 0; x < 3; ++x) mbar_init(&bar->meta[x], 4);
         mbar_init(&bar->acc_full, 1);
         mbar_init(&bar->acc_empty, 4);
         for (int k = 0; k < 2; ++k) {
@@ -739,24 +742,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int ku = (cl % nb) * BS + r;  // this thread's key token
             const bool key_in = ku < N;
             bool ok = true;
+            // The LSE (log2 units, +inf past N) and D of the item's query block jj, the
+            // CTA's tile number tt, go into shared copy tt % 3 one tile ahead, shared by
+            // the four warps (three copies: a warp can run one tile ahead of the others).
+            auto stage_meta = [&](int jj, uint32_t tt) {
+                const int qb = __ldg(csc_idx + start + jj);
+                float *mt = meta + (tt % 3) * 2 * BS;
+                const int tq = qb * BS + r;
+                const bool qin = qb >= 0 && qb < nb && tq < N;
+                const float lse = qin ? __ldg(LSE + bh * N + tq) : CUDART_INF_F;
+                mt[r] = (lse == -CUDART_INF_F) ? CUDART_INF_F : lse * kLog2e;
+                mt[BS + r] = qin ? __ldg(Dg + bh * N + tq) : 0.0f;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bar->meta[tt % 3]);
+            };
+            if (count > 0) stage_meta(0, tc);
             for (int j = 0; j < count; ++j) {
                 const int qblk = __ldg(csc_idx + start + j);
                 const int q0 = qblk * BS;
-                // this query block's LSE (log2 units, +inf past N) and D, shared by the warps
-                float *mt = meta + (tc & 1) * 2 * BS;
-                {
-                    const int tq = q0 + r;
-                    const bool qin = qblk >= 0 && qblk < nb && tq < N;
-                    const float lse = qin ? __ldg(LSE + bh * N + tq) : CUDART_INF_F;
-                    mt[r] = (lse == -CUDART_INF_F) ? CUDART_INF_F : lse * kLog2e;
-                    mt[BS + r] = qin ? __ldg(Dg + bh * N + tq) : 0.0f;
-                }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bar->meta[tc & 1]);
-                if (!mbar_wait(&bar->meta[tc & 1], (tc >> 1) & 1, abort_flag, dev_status)) {
-                    ok = false;
-                    break;
-                }
+                const float *mt = meta + (tc % 3) * 2 * BS;
                 // queries of this block that exist (and, causal, come at or after the key)
                 int lo = 0, hi = min(BS, N - q0);  // allowed columns: [lo, hi)
                 if (causal) lo = max(0, ku - q0);
@@ -766,49 +770,71 @@ __global__ void __launch_bounds__(kThreads, 1)
                     break;
                 }
                 tc_fence_after();
-                float p[BS];
+                uint32_t v[BS];
 #pragma unroll
-                for (int c0 = 0; c0 < BS; c0 += 32) {
-                    uint32_t v[32];
-                    tmem_ld32(tmem + lane_base + C::T_S + c0, v);
-                    tmem_wait_ld();
+                for (int c0 = 0; c0 < BS; c0 += 32)
+                    tmem_ld32(tmem + lane_base + C::T_S + c0, *reinterpret_cast<uint32_t(*)[32]>(&v[c0]));
+                if (!mbar_wait(&bar->meta[tc % 3], (tc / 3) & 1, abort_flag, dev_status)) {
+                    ok = false;
+                    break;
+                }
+                tmem_wait_ld();
+                // P^T = exp(S^T / sqrt(d) - LSE), packed in place as bf16 pairs: v[c/2] <- (p[c], p[c+1])
+                if (__all_sync(0xffffffffu, lo == 0 && hi == BS)) {
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) {
-                        const int cc = c0 + c;
-                        p[cc] = (cc >= lo && cc < hi) ? ex2_approx(fmaf(__uint_as_float(v[c]), scale_log2, -mt[cc]))
-                                                      : 0.0f;
+                    for (int c = 0; c < BS; c += 4) {
+                        const float4 l4 = *reinterpret_cast<const float4 *>(mt + c);
+                        const float p0 = ex2_approx(fmaf(__uint_as_float(v[c]), scale_log2, -l4.x));
+                        const float p1 = ex2_approx(fmaf(__uint_as_float(v[c + 1]), scale_log2, -l4.y));
+                        const float p2 = ex2_approx(fmaf(__uint_as_float(v[c + 2]), scale_log2, -l4.z));
+                        const float p3 = ex2_approx(fmaf(__uint_as_float(v[c + 3]), scale_log2, -l4.w));
+                        v[c >> 1] = pack_bf16(p0, p1);
+                        v[(c >> 1) + 1] = pack_bf16(p2, p3);
+                    }
+                } else {
+#pragma unroll
+                    for (int c = 0; c < BS; c += 2) {
+                        const float p0 = (c >= lo && c < hi)
+                                             ? ex2_approx(fmaf(__uint_as_float(v[c]), scale_log2, -mt[c])) : 0.0f;
+                        const float p1 = (c + 1 >= lo && c + 1 < hi)
+                                             ? ex2_approx(fmaf(__uint_as_float(v[c + 1]), scale_log2, -mt[c + 1]))
+                                             : 0.0f;
+                        v[c >> 1] = pack_bf16(p0, p1);
                     }
                 }
-                // P^T as bf16 pairs into the S^T columns, for dV += P^T dO
+                // P^T into the S^T columns, for dV += P^T dO
 #pragma unroll
-                for (int c0 = 0; c0 < BS; c0 += 32) {
-                    uint32_t w[16];
-#pragma unroll
-                    for (int c = 0; c < 32; c += 2) w[c >> 1] = pack_bf16(p[c0 + c], p[c0 + c + 1]);
-                    tmem_st16(tmem + lane_base + C::T_S + c0 / 2, w);
-                }
+                for (int c0 = 0; c0 < BS / 2; c0 += 32)
+                    tmem_st32(tmem + lane_base + C::T_S + c0, *reinterpret_cast<const uint32_t(*)[32]>(&v[c0]));
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bar->p_full);
+                // the next block's LSE and D while the tensor cores work
+                if (j + 1 < count) stage_meta(j + 1, tc + 1);
                 if (!mbar_wait(&bar->dpt_full, tc & 1, abort_flag, dev_status)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                // dS^T = P^T (dP^T - D), as bf16 pairs into the dP^T columns
+                // dS^T = P^T (dP^T - D) with P^T in bf16, packed into the dP^T columns
+                uint32_t g[BS];
 #pragma unroll
-                for (int c0 = 0; c0 < BS; c0 += 32) {
-                    uint32_t v[32];
-                    tmem_ld32(tmem + lane_base + C::T_DP + c0, v);
-                    tmem_wait_ld();
-                    uint32_t w[16];
+                for (int c0 = 0; c0 < BS; c0 += 32)
+                    tmem_ld32(tmem + lane_base + C::T_DP + c0, *reinterpret_cast<uint32_t(*)[32]>(&g[c0]));
+                tmem_wait_ld();
 #pragma unroll
-                    for (int c = 0; c < 32; c += 2)
-                        w[c >> 1] = pack_bf16(p[c0 + c] * (__uint_as_float(v[c]) - mt[BS + c0 + c]),
-                                              p[c0 + c + 1] * (__uint_as_float(v[c + 1]) - mt[BS + c0 + c + 1]));
-                    tmem_st16(tmem + lane_base + C::T_DP + c0 / 2, w);
+                for (int c = 0; c < BS; c += 4) {
+                    const float4 d4 = *reinterpret_cast<const float4 *>(mt + BS + c);
+                    const uint32_t pa = v[c >> 1], pb = v[(c >> 1) + 1];
+                    g[c >> 1] = pack_bf16(__uint_as_float(pa << 16) * (__uint_as_float(g[c]) - d4.x),
+                                          __uint_as_float(pa & 0xFFFF0000u) * (__uint_as_float(g[c + 1]) - d4.y));
+                    g[(c >> 1) + 1] = pack_bf16(__uint_as_float(pb << 16) * (__uint_as_float(g[c + 2]) - d4.z),
+                                                __uint_as_float(pb & 0xFFFF0000u) * (__uint_as_float(g[c + 3]) - d4.w));
                 }
+#pragma unroll
+                for (int c0 = 0; c0 < BS / 2; c0 += 32)
+                    tmem_st32(tmem + lane_base + C::T_DP + c0, *reinterpret_cast<const uint32_t(*)[32]>(&g[c0]));
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
