@@ -95,3 +95,9 @@ def test_bwd_user_mask_with_empty_rows_and_unselected_keys(oracle_mod):
             rp.append(len(ci))
     csr = (np.asarray(rp, np.int32), np.asarray(ci, np.int32))
     run_case(oracle_mod, B=1, H=2, N=600, d=64, seed=54, csr=csr)
+
+
+def test_bwd_routed_more_blocks_and_heads(oracle_mod):
+    """32 key blocks per head and 8 heads, routed at p = 0.9: long CSR rows and
+    columns, several items per CTA."""
+    run_case(oracle_mod, B=1, H=8, N=4096, d=128, p=0.9, seed=55)
