@@ -247,7 +247,6 @@ static int sparse_fwd_impl(const void *Q, const void *K, const void *V, const in
     if (!device_info(&info)) return FVATTN_ERR_CUDA;
     const int64_t BH = static_cast<int64_t>(B) * H;
     const int nb = static_cast<int>(ceil_div(N, block));
-    const int64_t rows = BH * nb;
     if (BH > kMaxHeads) return FVATTN_ERR_UNSUPPORTED;
     const int64_t items = attn_num_items(BH, nb);
     const FwdWorkspace w = fwd_layout(items, BH);

@@ -275,21 +275,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             };
             // D[dcol] = A[acol] (TMEM, 128 x d) * B^T, B a K-major tile of ring stage st
             auto issue_nt = [&](uint32_t dcol, uint32_t acol, uint32_t st) {
-                const uint32_t b = r0 + st * C::STAGE_BYTES;
+                const uint64_t d0 = smem_desc_sw128(r0 + st * C::STAGE_BYTES, 16, 1024);
 #pragma unroll
-                for (int k = 0; k < D / 16; ++k) {
-                    const uint64_t db = smem_desc_sw128(b + (k >> 2) * BS * 128 + (k & 3) * 32, 16, 1024);
-                    mma_ts(tmem + dcol, tmem + acol + k * 8, db, C::IDESC_S, k > 0 ? 1u : 0u);
-                }
+                for (int k = 0; k < D / 16; ++k)
+                    mma_ts_nc(tmem + dcol, tmem + acol + k * 8, d0 + (((k >> 2) * BS * 128 + (k & 3) * 32) >> 4),
+                              C::IDESC_S, k > 0 ? 1u : 0u);
             };
             // dQ (+)= dS K, K of ring stage st read MN-major
             auto issue_dq = [&](uint32_t st, bool first) {
-                const uint32_t b = r0 + st * C::STAGE_BYTES;
+                const uint64_t d0 = smem_desc_sw128(r0 + st * C::STAGE_BYTES, BS * 128, 1024);
+                const uint32_t acc0 = first ? 0u : 1u;
 #pragma unroll
-                for (int k = 0; k < BS / 16; ++k) {
-                    const uint64_t db = smem_desc_sw128(b + k * 16 * 128, BS * 128, 1024);
-                    mma_ts(tmem + C::T_DQ, tmem + C::T_DP + k * 8, db, C::IDESC_Q, (!first || k > 0) ? 1u : 0u);
-                }
+                for (int k = 0; k < BS / 16; ++k)
+                    mma_ts_nc(tmem + C::T_DQ, tmem + C::T_DP + k * 8, d0 + ((k * 16 * 128) >> 4), C::IDESC_Q,
+                              k > 0 ? 1u : acc0);
             };
             while (ok) {
                 const uint32_t k = it & 1;
@@ -650,21 +649,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             };
             // D[dcol] = A B^T with A (the item's K or V) and B (a ring tile) both K-major
             auto issue_t = [&](uint32_t dcol, uint32_t a, uint32_t st) {
-                const uint32_t b = r0 + st * C::STAGE_BYTES;
+                const uint64_t a0 = smem_desc_sw128(a, 16, 1024);
+                const uint64_t b0 = smem_desc_sw128(r0 + st * C::STAGE_BYTES, 16, 1024);
 #pragma unroll
                 for (int k = 0; k < D / 16; ++k) {
-                    const uint32_t off = (k >> 2) * BS * 128 + (k & 3) * 32;
-                    mma_ss(tmem + dcol, smem_desc_sw128(a + off, 16, 1024), smem_desc_sw128(b + off, 16, 1024),
-                           C::IDESC_T, k > 0 ? 1u : 0u);
+                    const uint32_t off = ((k >> 2) * BS * 128 + (k & 3) * 32) >> 4;
+                    mma_ss_nc(tmem + dcol, a0 + off, b0 + off, C::IDESC_T, k > 0 ? 1u : 0u);
                 }
             };
             // acc[dcol] (+)= A[acol] (TMEM, bf16 pairs) B, B a ring tile read MN-major
             auto issue_acc = [&](uint32_t dcol, uint32_t acol, uint32_t st, bool first) {
-                const uint32_t b = r0 + st * C::STAGE_BYTES;
+                const uint64_t b0 = smem_desc_sw128(r0 + st * C::STAGE_BYTES, BS * 128, 1024);
+                const uint32_t acc0 = first ? 0u : 1u;
 #pragma unroll
                 for (int k = 0; k < BS / 16; ++k)
-                    mma_ts(tmem + dcol, tmem + acol + k * 8, smem_desc_sw128(b + k * 16 * 128, BS * 128, 1024),
-                           C::IDESC_A, (!first || k > 0) ? 1u : 0u);
+                    mma_ts_nc(tmem + dcol, tmem + acol + k * 8, b0 + ((k * 16 * 128) >> 4), C::IDESC_A,
+                              k > 0 ? 1u : acc0);
             };
             while (ok) {
                 const uint32_t k = it & 1;
