@@ -418,8 +418,13 @@ int fvattn_attention_host(const void *hQ, const void *hK, const void *hV, int B,
     const size_t head_bytes = static_cast<size_t>(N) * d * 2;
     // Heads are independent for routing and attention: split B*H into chunks of about
     // 64 MB per tensor so that copies in, compute and copies out of different chunks
-    // overlap (two extra streams for the copies, the caller's stream for compute).
+    // overlap (two extra streams for the copies, the caller's stream for compute).  The
+    // copies in are the bottleneck; what follows the last one (that chunk's compute and
+    // copy out) is not hidden, so the last chunks halve in size down to one head.
     const int64_t hc = std::max<int64_t>(1, std::min<int64_t>(BH, (64ll << 20) / static_cast<int64_t>(head_bytes)));
+    auto chunk_heads = [&](int64_t remaining) {
+        return remaining > 2 * hc ? hc : std::max<int64_t>(1, std::min<int64_t>(hc, (remaining + 1) / 2));
+    };
     cudaStream_t s_in = nullptr, s_out = nullptr;
     cudaEvent_t ev_in = nullptr, ev_out = nullptr;
     auto cleanup = [&]() {
@@ -441,8 +446,9 @@ int fvattn_attention_host(const void *hQ, const void *hK, const void *hV, int B,
     rc = from_cuda(cudaMemsetAsync(dev_status + 2, 0, sizeof(int32_t), s));
     if (rc == FVATTN_OK) rc = from_cuda(cudaEventRecord(ev_out, s));
     if (rc == FVATTN_OK) rc = from_cuda(cudaStreamWaitEvent(s_in, ev_out, 0));
-    for (int64_t off = 0; off < BH && rc == FVATTN_OK; off += hc) {
-        const int hn = static_cast<int>(std::min<int64_t>(hc, BH - off));
+    int hn = 0;
+    for (int64_t off = 0; off < BH && rc == FVATTN_OK; off += hn) {
+        hn = static_cast<int>(chunk_heads(BH - off));
         const size_t o = static_cast<size_t>(off) * head_bytes, nbytes = static_cast<size_t>(hn) * head_bytes;
         const size_t lo = static_cast<size_t>(off) * N * sizeof(float), lbytes = static_cast<size_t>(hn) * N * sizeof(float);
         auto dptr = [&](void *base) { return static_cast<char *>(base) + o; };
