@@ -49,8 +49,10 @@ def _load():
         lib.oracle_attn_tiled.argtypes = lib.oracle_attn_rows.argtypes
         lib.oracle_lpt_order.argtypes = [P, i64, P]
         lib.oracle_attn_bwd.argtypes = [P, P, P, P, i32, i32, i32, i32, i32, i32, P, P, P, P, P, i32]
+        lib.oracle_attn_bwd_sampled.argtypes = [P, P, P, P, i32, i32, i32, i32, i32, i32, P, P, P, i64, P, P, P,
+                                                i64, P, P, i32]
         for f in ("oracle_pool", "oracle_route", "oracle_attn_rows", "oracle_attn_tiled", "oracle_lpt_order",
-                  "oracle_attn_bwd"):
+                  "oracle_attn_bwd", "oracle_attn_bwd_sampled"):
             getattr(lib, f).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -163,6 +165,40 @@ def attn_bwd(Q, K, V, dO, bs, causal, row_ptr, col_idx, nthreads=None):
     if rc != 0:
         raise ValueError("oracle_attn_bwd failed")
     return dQ, dK, dV
+
+
+def attn_bwd_sampled(Q, K, V, dO, bs, causal, row_ptr, col_idx, q_tokens, k_tokens, nthreads=None):
+    """The gradients of :func:`attn_bwd` at sampled tokens only (global indices
+    b*H*N + h*N + t): dQ rows of ``q_tokens`` and dK, dV rows of ``k_tokens``, fp64
+    [n, d] each.  Key tokens are grouped by (head, key block) internally so that one
+    query row's softmax serves every sampled key of its block."""
+    Q, K, V, dO = _bits(Q), _bits(K), _bits(V), _bits(dO)
+    B, H, N, d = Q.shape
+    row_ptr = np.ascontiguousarray(row_ptr, dtype=np.int32)
+    col_idx = np.ascontiguousarray(col_idx, dtype=np.int32)
+    if col_idx.size == 0:
+        col_idx = np.zeros(1, dtype=np.int32)
+    q_tokens = np.ascontiguousarray(q_tokens, dtype=np.int64)
+    k_tokens = np.ascontiguousarray(k_tokens, dtype=np.int64)
+    key = (k_tokens // N) * (N // bs + 1) + (k_tokens % N) // bs  # (head, key block)
+    perm = np.argsort(key, kind="stable")
+    ks = np.ascontiguousarray(k_tokens[perm])
+    starts = np.flatnonzero(np.r_[True, np.diff(key[perm]) != 0]) if ks.size else np.zeros(0, np.int64)
+    group_ptr = np.ascontiguousarray(np.r_[starts, ks.size], dtype=np.int64)
+    dQ = np.empty((max(q_tokens.size, 1), d), dtype=np.float64)
+    dKs = np.empty((max(ks.size, 1), d), dtype=np.float64)
+    dVs = np.empty_like(dKs)
+    rc = _load().oracle_attn_bwd_sampled(_ptr(Q), _ptr(K), _ptr(V), _ptr(dO), B, H, N, d, bs, 1 if causal else 0,
+                                         _ptr(row_ptr), _ptr(col_idx), _ptr(q_tokens), q_tokens.size, _ptr(dQ),
+                                         _ptr(ks), _ptr(group_ptr), group_ptr.size - 1, _ptr(dKs), _ptr(dVs),
+                                         nthreads or default_threads())
+    if rc != 0:
+        raise ValueError("oracle_attn_bwd_sampled failed")
+    dK = np.empty((k_tokens.size, d), dtype=np.float64)
+    dV = np.empty_like(dK)
+    dK[perm] = dKs[: ks.size]
+    dV[perm] = dVs[: ks.size]
+    return dQ[: q_tokens.size], dK, dV
 
 
 def lpt_order(row_ptr: np.ndarray) -> np.ndarray:

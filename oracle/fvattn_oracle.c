@@ -594,3 +594,168 @@ int oracle_attn_bwd(const uint16_t *Q, const uint16_t *K, const uint16_t *V, con
     parallel_for((int64_t)B * H, nthreads, attn_bwd_range, &c);
     return 0;
 }
+
+/* ------------------------------ gradients of sampled query and key tokens */
+
+/*
+ * The same derivatives as oracle_attn_bwd, evaluated only where asked, so that
+ * the gradients of full-size problems can be checked on samples:
+ *   dQ_t for the listed query tokens (one row's softmax each), and
+ *   dK_u, dV_u for the listed key tokens, summed over every query token t whose
+ *   CSR row lists u's block (u <= t if causal), t in index order.
+ * Key tokens come grouped by (batch*head, key block) through group_ptr: one
+ * query row's softmax serves every key of its group.  Per row the operations
+ * and their order are those of oracle_attn_bwd, so both give identical values.
+ */
+typedef struct {
+    const uint16_t *Q, *K, *V, *dO;
+    int N, d, bs, causal;
+    int64_t nb;
+    const int32_t *row_ptr, *col_idx;
+    double scale;
+    int64_t nq;
+    const int64_t *q_tok;
+    double *dQ;
+    const int64_t *k_tok, *group_ptr;
+    double *dK, *dV;
+} bwd_sample_ctx;
+
+/* Softmax row of query token t of head bh: fills p (probabilities), u_of, o, and
+ * returns the number of allowed keys and D_t = dO_t . O_t (q and go filled). */
+static int64_t bwd_row(const bwd_sample_ctx *c, int64_t bh, int64_t t, double *q, double *go, double *o,
+                       double *p, int64_t *u_of, double *D_out) {
+    const int d = c->d;
+    const int64_t base = bh * c->N * d;
+    const int64_t row = bh * c->nb + t / c->bs;
+    for (int ch = 0; ch < d; ++ch) {
+        q[ch] = bf16_bits_to_double(c->Q[base + t * d + ch]);
+        go[ch] = bf16_bits_to_double(c->dO[base + t * d + ch]);
+    }
+    int64_t n = 0;
+    double m = -INFINITY;
+    for (int32_t e = c->row_ptr[row]; e < c->row_ptr[row + 1]; ++e) {
+        int64_t kb = c->col_idx[e];
+        for (int64_t u = kb * c->bs; u < (kb + 1) * c->bs && u < c->N; ++u) {
+            if (c->causal && u > t) continue;
+            double dot = 0.0;
+            for (int ch = 0; ch < d; ++ch) dot = dot + q[ch] * bf16_bits_to_double(c->K[base + u * d + ch]);
+            p[n] = dot * c->scale;
+            u_of[n] = u;
+            if (p[n] > m) m = p[n];
+            ++n;
+        }
+    }
+    if (n == 0) return 0;
+    double z = 0.0;
+    for (int64_t a = 0; a < n; ++a) {
+        p[a] = exp(p[a] - m);
+        z = z + p[a];
+    }
+    for (int64_t a = 0; a < n; ++a) p[a] = p[a] / z;
+    for (int ch = 0; ch < d; ++ch) o[ch] = 0.0;
+    for (int64_t a = 0; a < n; ++a)
+        for (int ch = 0; ch < d; ++ch) o[ch] = o[ch] + p[a] * bf16_bits_to_double(c->V[base + u_of[a] * d + ch]);
+    double D = 0.0;
+    for (int ch = 0; ch < d; ++ch) D = D + go[ch] * o[ch];
+    *D_out = D;
+    return n;
+}
+
+static void bwd_sample_range(void *vctx, int64_t begin, int64_t end) {
+    bwd_sample_ctx *c = (bwd_sample_ctx *)vctx;
+    const int d = c->d;
+    const int64_t cap = c->nb * c->bs;
+    double *q = (double *)malloc(sizeof(double) * d);
+    double *go = (double *)malloc(sizeof(double) * d);
+    double *o = (double *)malloc(sizeof(double) * d);
+    double *p = (double *)malloc(sizeof(double) * cap);
+    int64_t *u_of = (int64_t *)malloc(sizeof(int64_t) * cap);
+    if (!q || !go || !o || !p || !u_of) goto out;
+    for (int64_t it = begin; it < end; ++it) {
+        if (it < c->nq) { /* dQ of one query token */
+            const int64_t g = c->q_tok[it], bh = g / c->N, t = g % c->N;
+            const int64_t base = bh * c->N * d;
+            double *dq = c->dQ + it * d;
+            for (int ch = 0; ch < d; ++ch) dq[ch] = 0.0;
+            double D = 0.0;
+            const int64_t n = bwd_row(c, bh, t, q, go, o, p, u_of, &D);
+            for (int64_t a = 0; a < n; ++a) {
+                const int64_t u = u_of[a];
+                double dp = 0.0;
+                for (int ch = 0; ch < d; ++ch) dp = dp + go[ch] * bf16_bits_to_double(c->V[base + u * d + ch]);
+                const double ds = p[a] * (dp - D);
+                for (int ch = 0; ch < d; ++ch)
+                    dq[ch] = dq[ch] + ds * bf16_bits_to_double(c->K[base + u * d + ch]) * c->scale;
+            }
+            continue;
+        }
+        /* dK, dV of one group of key tokens (same head, same key block) */
+        const int64_t gi = it - c->nq;
+        const int64_t k0 = c->group_ptr[gi], k1 = c->group_ptr[gi + 1];
+        if (k1 <= k0) continue;
+        const int64_t bh = c->k_tok[k0] / c->N, kb = (c->k_tok[k0] % c->N) / c->bs;
+        const int64_t base = bh * c->N * d;
+        for (int64_t k = k0; k < k1; ++k)
+            for (int ch = 0; ch < d; ++ch) {
+                c->dK[k * d + ch] = 0.0;
+                c->dV[k * d + ch] = 0.0;
+            }
+        for (int64_t qb = 0; qb < c->nb; ++qb) {
+            const int64_t row = bh * c->nb + qb;
+            int listed = 0;
+            for (int32_t e = c->row_ptr[row]; e < c->row_ptr[row + 1]; ++e)
+                if (c->col_idx[e] == kb) listed = 1;
+            if (!listed) continue;
+            for (int64_t t = qb * c->bs; t < (qb + 1) * c->bs && t < c->N; ++t) {
+                double D = 0.0;
+                const int64_t n = bwd_row(c, bh, t, q, go, o, p, u_of, &D);
+                for (int64_t a = 0; a < n; ++a) {
+                    const int64_t u = u_of[a];
+                    for (int64_t k = k0; k < k1; ++k) {
+                        if (c->k_tok[k] % c->N != u) continue;
+                        double dp = 0.0;
+                        for (int ch = 0; ch < d; ++ch)
+                            dp = dp + go[ch] * bf16_bits_to_double(c->V[base + u * d + ch]);
+                        const double ds = p[a] * (dp - D);
+                        double *dv = c->dV + k * d, *dk = c->dK + k * d;
+                        for (int ch = 0; ch < d; ++ch) {
+                            dv[ch] = dv[ch] + p[a] * go[ch];
+                            dk[ch] = dk[ch] + ds * q[ch] * c->scale;
+                        }
+                    }
+                }
+            }
+        }
+    }
+out:
+    free(q);
+    free(go);
+    free(o);
+    free(p);
+    free(u_of);
+}
+
+int oracle_attn_bwd_sampled(const uint16_t *Q, const uint16_t *K, const uint16_t *V, const uint16_t *dO, int B,
+                            int H, int N, int d, int bs, int causal, const int32_t *row_ptr, const int32_t *col_idx,
+                            const int64_t *q_tok, int64_t nq, double *dQ, const int64_t *k_tok,
+                            const int64_t *group_ptr, int64_t ngroups, double *dK, double *dV, int nthreads) {
+    if (!Q || !K || !V || !dO || !row_ptr || !col_idx) return -1;
+    if (B < 1 || H < 1 || N < 1 || d < 1 || bs < 1 || nq < 0 || ngroups < 0) return -1;
+    if ((nq > 0 && (!q_tok || !dQ)) || (ngroups > 0 && (!k_tok || !group_ptr || !dK || !dV))) return -1;
+    const int64_t total = (int64_t)B * H * N;
+    for (int64_t i = 0; i < nq; ++i)
+        if (q_tok[i] < 0 || q_tok[i] >= total) return -1;
+    for (int64_t gi = 0; gi < ngroups; ++gi) {
+        if (group_ptr[gi + 1] < group_ptr[gi]) return -1;
+        for (int64_t k = group_ptr[gi]; k < group_ptr[gi + 1]; ++k) {
+            if (k_tok[k] < 0 || k_tok[k] >= total) return -1;
+            if (k_tok[k] / N != k_tok[group_ptr[gi]] / N ||
+                (k_tok[k] % N) / bs != (k_tok[group_ptr[gi]] % N) / bs)
+                return -1; /* a group spans one head and one key block */
+        }
+    }
+    bwd_sample_ctx c = {Q, K, V, dO, N, d, bs, causal ? 1 : 0, num_blocks(N, bs), row_ptr, col_idx,
+                        1.0 / sqrt((double)d), nq, q_tok, dQ, k_tok, group_ptr, dK, dV};
+    parallel_for(nq + ngroups, nthreads, bwd_sample_range, &c);
+    return 0;
+}

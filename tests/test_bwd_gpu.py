@@ -101,3 +101,66 @@ def test_bwd_routed_more_blocks_and_heads(oracle_mod):
     """32 key blocks per head and 8 heads, routed at p = 0.9: long CSR rows and
     columns, several items per CTA."""
     run_case(oracle_mod, B=1, H=8, N=4096, d=128, p=0.9, seed=55)
+
+
+def _cheap_key_groups(rp, ci, w, rng, max_groups=10, max_select=2, per_block=4):
+    """Sampled key tokens for dK/dV at full size: key blocks that at most
+    ``max_select`` query blocks select (at least one), one per head in a seeded
+    head order, up to ``max_groups`` heads; four tokens per block, the ragged tail
+    included when it is the block.  The oracle rebuilds every selecting query
+    row's softmax for each block, so this bounds its work."""
+    BH, nb = w.B * w.H, w.nb
+    toks, rows = [], 0
+    for bh in rng.permutation(BH):
+        if len(toks) == max_groups:
+            break
+        cols = ci[rp[bh * nb]:rp[(bh + 1) * nb]]
+        counts = np.bincount(cols, minlength=nb)
+        sel = np.flatnonzero((counts > 0) & (counts <= max_select))
+        if sel.size == 0:
+            continue
+        kb = int(rng.choice(sel))
+        rows += int(counts[kb]) * w.bs
+        t0, t1 = kb * w.bs, min(w.N, (kb + 1) * w.bs)
+        ts = rng.choice(np.arange(t0, t1), size=min(per_block, t1 - t0), replace=False)
+        toks.append(bh * w.N + np.sort(ts))
+    return (np.concatenate(toks).astype(np.int64) if toks else np.zeros(0, np.int64)), rows
+
+
+FULL_BWD = [(W.VIDEO, False), (W.DENSE_CAUSAL, True)]
+
+
+@pytest.mark.parametrize("w,causal", FULL_BWD, ids=lambda x: x.name if hasattr(x, "name") else str(x))
+def test_bwd_full_size_sampled(w, causal, oracle_mod):
+    """Full-size gradients (the configuration the benchmark times for video) on
+    samples: dQ rows of query blocks 0, the ragged last one and two random ones in
+    every head, and dK/dV rows of key blocks selected by one or two query blocks
+    (which bounds the oracle's work) in up to ten heads.  The mask comes from the oracle's own
+    routing (video) or is the dense causal one, so no oracle input comes from the
+    GPU; O and LSE for the backward come from the GPU forward on that mask."""
+    import top_routed_block_b200 as fv
+    rng = np.random.default_rng(61)
+    Q, K, V = W.generate(w)
+    if causal:
+        rp, ci = oracle_mod.dense_csr(w.B, w.H, w.N, w.bs, True)
+    else:
+        r = oracle_mod.route(Q, K, w.p, w.bs)
+        rp, ci = r.row_ptr, r.col_idx
+    dO = W.f32_to_bf16_bits(rng.standard_normal(Q.shape).astype(np.float32))
+    dQ_, dK_, dV_, dO_ = (to_dev(x) for x in (Q, K, V, dO))
+    rp_t = torch.from_numpy(np.ascontiguousarray(rp, np.int32)).cuda()
+    ci_t = torch.from_numpy(np.ascontiguousarray(ci, np.int32)).cuda()
+    O, LSE, st = fv.fvattn_sparse_fwd(dQ_, dK_, dV_, rp_t, ci_t, w.bs, causal)
+    fv.check_status(st, "fwd")
+    gQ, gK, gV, st = fv.fvattn_sparse_bwd(dQ_, dK_, dV_, O, LSE, dO_, rp_t, ci_t, w.bs, causal)
+    fv.check_status(st, "bwd")
+    q_tok = W.sample_tokens(w, per_head_blocks=2, rows_per_block=2)
+    k_tok, rows = _cheap_key_groups(rp, ci, w, rng)
+    assert k_tok.size >= 8, "no affordable key blocks to sample"
+    rq, rk, rv = oracle_mod.attn_bwd_sampled(Q, K, V, dO, w.bs, causal, rp, ci, q_tok, k_tok)
+    d = w.d
+    grads_close("dQ (sampled)", gQ.reshape(-1, d)[torch.from_numpy(q_tok).cuda()], rq)
+    kt = torch.from_numpy(k_tok).cuda()
+    grads_close("dK (sampled)", gK.reshape(-1, d)[kt], rk)
+    grads_close("dV (sampled)", gV.reshape(-1, d)[kt], rv)
+    print(w.name, "query rows", q_tok.size, "key rows", k_tok.size, "oracle query rows rebuilt", rows)

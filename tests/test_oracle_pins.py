@@ -496,3 +496,40 @@ def test_attn_bwd_dense_identities(oracle_mod):
     dQ, dK, dV = oracle_mod.attn_bwd(Q, K, V, dO, bs, False, row_ptr, col_idx)
     assert np.max(np.abs(dV.sum(axis=2) - fvals(dO).sum(axis=2))) < 1e-10
     assert np.max(np.abs(dK.sum(axis=2))) < 1e-10
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_attn_bwd_sampled_equals_full_gradients(oracle_mod, causal):
+    """The sampled-token gradients are the full oracle's rows, value for value: query
+    tokens anywhere (ragged last block, empty CSR rows), key tokens grouped and
+    ungrouped, a key block no row selects (zero gradients), a repeated token."""
+    rng = np.random.default_rng(21 + causal)
+    B, H, N, d, bs = 2, 2, 100, 16, 32
+    nb = -(-N // bs)
+    row_ptr, col_idx = random_csr(rng, B * H * nb, nb, p_keep=0.5, allow_empty=True)
+    Q, K, V, dO = (rand_bf16(rng, (B, H, N, d)) for _ in range(4))
+    dQ, dK, dV = oracle_mod.attn_bwd(Q, K, V, dO, bs, causal, row_ptr, col_idx)
+    total = B * H * N
+    q_tok = np.r_[rng.choice(total, 20, replace=False), total - 1, 0]
+    k_tok = np.r_[rng.choice(total, 24, replace=False), 3, 3, N - 1, total - 1]
+    sq, sk, sv = oracle_mod.attn_bwd_sampled(Q, K, V, dO, bs, causal, row_ptr, col_idx, q_tok, k_tok)
+    flat = lambda a: a.reshape(total, d)
+    assert np.array_equal(sq, flat(dQ)[q_tok])
+    assert np.array_equal(sk, flat(dK)[k_tok])
+    assert np.array_equal(sv, flat(dV)[k_tok])
+
+
+def test_attn_bwd_sampled_dense_matches_torch_autograd(oracle_mod):
+    """Dense non-causal: the sampled rows equal fp64 autograd of softmax(QK^T/sqrt(d))V."""
+    import torch
+    rng = np.random.default_rng(23)
+    B, H, N, d, bs = 1, 2, 80, 16, 32
+    row_ptr, col_idx = oracle_mod.dense_csr(B, H, N, bs, False)
+    Q, K, V, dO = (rand_bf16(rng, (B, H, N, d)) for _ in range(4))
+    q, k, v = (torch.tensor(fvals(x), dtype=torch.float64, requires_grad=True) for x in (Q, K, V))
+    o = torch.softmax(q @ k.transpose(-1, -2) / math.sqrt(d), dim=-1) @ v
+    (o * torch.tensor(fvals(dO), dtype=torch.float64)).sum().backward()
+    toks = np.array([0, 31, 32, 79, N + 5, 2 * N - 1])
+    sq, sk, sv = oracle_mod.attn_bwd_sampled(Q, K, V, dO, bs, False, row_ptr, col_idx, toks, toks)
+    for mine, ref in ((sq, q.grad), (sk, k.grad), (sv, v.grad)):
+        assert np.max(np.abs(mine - ref.numpy().reshape(-1, d)[toks])) < 1e-11
