@@ -40,6 +40,8 @@
  *   attn_bwd    central finite differences of a numpy fp64 brute-force forward,
  *               fp64 torch autograd of dense attention, and the dense-case
  *               identities sum_u dK_u = 0 and sum_u dV_u = sum_t dO_t
+ *   attn_bwd_sampled  equal, value for value, to attn_bwd at the sampled
+ *               tokens, and to fp64 torch autograd of dense attention
  *   lpt_order   brute-force sort on small inputs
  */
 #include <math.h>
