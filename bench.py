@@ -319,6 +319,11 @@ def run_ours(args, w, rank, world, local):
     attn_ms = statistics.mean(fwd_ms)
     attn_tflops = flops / (attn_ms * 1e-3) / 1e12
     r_ms = statistics.mean(route_ms)
+    step_ms = [a + b for a, b in zip(route_ms, fwd_ms)]
+    timing = {"step_ms_mean": statistics.mean(step_ms), "step_ms_median": statistics.median(step_ms),
+              "attn_ms_median": statistics.median(fwd_ms), "route_ms_median": statistics.median(route_ms),
+              "note": "per-step CUDA events on the launching stream (routing call, attention call); the line's "
+                      "ms_per_step is the whole timed region / steps, max over ranks"}
 
     # end to end through the host-buffer entry point
     hO = torch.empty((w.B, w.H, w.N, w.d), dtype=torch.bfloat16).pin_memory()
@@ -412,7 +417,7 @@ def run_ours(args, w, rank, world, local):
                    "causal": w.causal, "nnz_blocks": nnz, "density": nnz / (w.B * w.H * w.nb * w.nb),
                    "l2": "inputs larger than L2 (each of Q, K, V is %d MB)" % (elem * 2 // 10**6),
                    "parallelism": f"replicas x{world}"},
-        "attn_tflops": attn_tflops, "attn_ms": attn_ms, "route_ms": r_ms,
+        "attn_tflops": attn_tflops, "attn_ms": attn_ms, "route_ms": r_ms, "timing": timing,
         "route_frac": r_ms / (r_ms + attn_ms),
         "tensor_frac_of_burst_peak": attn_tflops / burst,
         "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peak, "unit": "TFLOP/s",
