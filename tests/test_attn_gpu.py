@@ -166,12 +166,21 @@ def test_bad_csr_is_reported_and_the_rest_is_computed(oracle_mod):
     compare_attention(O2, LSE2, Oref, Lref, tokens, w.d, "after-badcsr")
 
 
-def test_host_buffer_path_matches_device_path():
+HOST_CASES = [
+    # 24 heads of 0.5 MB: under two chunks of 64 MB, so the chunks halve at once (12, 6, 3, 2, 1)
+    W.Workload("host_path", B=2, H=12, N=2000, d=128, bs=128, p=0.8, dist="structured", grid=(5, 20, 20),
+               head_scale=("uniform", 0.5, 4.0), seed=44),
+    # 20 heads of 8 MB: a full 8-head chunk first, then the halving tail (8, 6, 3, 2, 1)
+    W.Workload("host_path_chunks", B=1, H=20, N=32768, d=128, bs=128, p=0.9, dist="structured",
+               grid=(8, 64, 64), head_scale=("uniform", 0.5, 4.0), seed=46),
+]
+
+
+@pytest.mark.parametrize("w", HOST_CASES, ids=lambda w: w.name)
+def test_host_buffer_path_matches_device_path(w):
     """fvattn_attention_host (chunked copies in, routing, attention, copies out)
     returns exactly what the device entry points return: heads are independent."""
     import top_routed_block_b200 as fv
-    w = W.Workload("host_path", B=2, H=12, N=2000, d=128, bs=128, p=0.8, dist="structured", grid=(5, 20, 20),
-                   head_scale=("uniform", 0.5, 4.0), seed=44)
     Q, K, V = W.generate(w)
     dQ, dK, dV = to_dev(Q), to_dev(K), to_dev(V)
     plan = fv.FvattnPlan(w.B, w.H, w.N, w.d, w.bs)
