@@ -173,8 +173,10 @@ FVATTN_API int fvattn_sparse_fwd(const void *Q, const void *K, const void *V, co
  * The heads are processed in chunks of about 64 MB per tensor: the copies in of
  * one chunk, the compute of the previous one (on `stream`) and the copies out of
  * the one before run concurrently, on two streams the call creates and destroys
- * (host buffers must be pinned for the copies to overlap).  Work already queued
- * on `stream` completes before the first copy starts.
+ * (host buffers must be pinned for the copies to overlap).  Once two chunks or
+ * fewer remain, the chunks halve in size down to one head, so that little
+ * compute and copying out follows the last copy in.  Work already queued on
+ * `stream` completes before the first copy starts.
  * Returns the first host error, else the first nonzero device status read
  * after the sync.
  */
