@@ -127,17 +127,18 @@ def _cheap_key_groups(rp, ci, w, rng, max_groups=10, max_select=2, per_block=4):
     return (np.concatenate(toks).astype(np.int64) if toks else np.zeros(0, np.int64)), rows
 
 
-FULL_BWD = [(W.VIDEO, False), (W.DENSE_CAUSAL, True)]
+FULL_BWD = [(W.VIDEO, False), (W.DENSE_CAUSAL, True), (W.LONG, False)]
 
 
 @pytest.mark.parametrize("w,causal", FULL_BWD, ids=lambda x: x.name if hasattr(x, "name") else str(x))
 def test_bwd_full_size_sampled(w, causal, oracle_mod):
-    """Full-size gradients (the configuration the benchmark times for video) on
+    """Full-size gradients (video: the configuration the benchmark times; long video:
+    118,800 tokens with a 16-token last block) on
     samples: dQ rows of query blocks 0, the ragged last one and two random ones in
     every head, and dK/dV rows of key blocks selected by one or two query blocks
     (which bounds the oracle's work) in up to ten heads.  The mask comes from the oracle's own
-    routing (video) or is the dense causal one, so no oracle input comes from the
-    GPU; O and LSE for the backward come from the GPU forward on that mask."""
+    routing (video, long video) or is the dense causal one, so no oracle input comes
+    from the GPU; O and LSE for the backward come from the GPU forward on that mask."""
     import top_routed_block_b200 as fv
     rng = np.random.default_rng(61)
     Q, K, V = W.generate(w)
