@@ -227,7 +227,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     item = make_int4(rw, row_ptr[rw], c, 1);
                 }
                 const uint32_t k = it & 1;
-                if (!mbar_wait(&bar->sched_empty[k], ((it >> 1) & 1) ^ 1, abort_flag, dev_status)) break;
+                if (!mbar_wait_short(&bar->sched_empty[k], ((it >> 1) & 1) ^ 1, abort_flag, dev_status)) break;
                 bar->sched_item[k] = item;
                 mbar_arrive(&bar->sched_full[k]);
                 ++it;
@@ -244,7 +244,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     for (int kv = 0; kv < 2; ++kv) {
                         const uint32_t st = rc % NST;
-                        if (!mbar_wait(&bar->ring_empty[st], ((rc / NST) & 1) ^ 1, abort_flag, dev_status)) {
+                        if (!mbar_wait_short(&bar->ring_empty[st], ((rc / NST) & 1) ^ 1, abort_flag, dev_status)) {
                             ok = false;
                             break;
                         }
@@ -270,7 +270,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t it = 0, rc = 0, tc = 0, qn = 0, on = 0;  // items, ring loads, tiles, Q loads, outputs
             bool ok = true;
             auto wait = [&](uint64_t *b, uint32_t parity) {
-                if (ok && !mbar_wait(b, parity, abort_flag, dev_status)) ok = false;
+                if (ok && !mbar_wait_short(b, parity, abort_flag, dev_status)) ok = false;
                 return ok;
             };
             // D[dcol] = A[acol] (TMEM, 128 x d) * B^T, B a K-major tile of ring stage st
@@ -355,7 +355,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t it = 0, tc = 0, qn = 0, on = 0;
         while (true) {
             const uint32_t k = it & 1;
-            if (!mbar_wait(&bar->sched_full[k], (it >> 1) & 1, abort_flag, dev_status)) break;
+            if (!mbar_wait_short(&bar->sched_full[k], (it >> 1) & 1, abort_flag, dev_status)) break;
             const int4 item = bar->sched_item[k];
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar->sched_empty[k]);
@@ -406,7 +406,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 int lim = valid ? min(BS, N - key0) : 0;
                 if (causal) lim = min(lim, t_row - key0 + 1);
                 if (!row_in) lim = 0;
-                if (!mbar_wait(&bar->s_full, tc & 1, abort_flag, dev_status)) {
+                if (!mbar_wait_short(&bar->s_full, tc & 1, abort_flag, dev_status)) {
                     ok = false;
                     break;
                 }
@@ -430,7 +430,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         v[c] = __float_as_uint(c < lim ? ex2_approx(fmaf(__uint_as_float(v[c]), scale_log2, -lse2))
                                                        : 0.0f);
                 }
-                if (!mbar_wait(&bar->dp_full, tc & 1, abort_flag, dev_status)) {
+                if (!mbar_wait_short(&bar->dp_full, tc & 1, abort_flag, dev_status)) {
                     ok = false;
                     break;
                 }
@@ -458,7 +458,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!ok) break;
             if (count > 0) ++qn;
             // epilogue: dQ = (sum over blocks of dS K) / sqrt(d)
-            if (!mbar_wait(&bar->dq_full, on & 1, abort_flag, dev_status)) break;
+            if (!mbar_wait_short(&bar->dq_full, on & 1, abort_flag, dev_status)) break;
             ++on;
             tc_fence_after();
 #pragma unroll
@@ -593,7 +593,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 int4 item = make_int4(-1, 0, 0, 0);
                 if (cl >= 0) item = make_int4(cl, col_ptr[cl], col_ptr[cl + 1] - col_ptr[cl], 1);
                 const uint32_t k = it & 1;
-                if (!mbar_wait(&bar->sched_empty[k], ((it >> 1) & 1) ^ 1, abort_flag, dev_status)) break;
+                if (!mbar_wait_short(&bar->sched_empty[k], ((it >> 1) & 1) ^ 1, abort_flag, dev_status)) break;
                 bar->sched_item[k] = item;
                 mbar_arrive(&bar->sched_full[k]);
                 ++it;
@@ -601,7 +601,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (item.z <= 0) continue;
                 const int bh = cl / nb, kblk = cl % nb;
                 // the item's K and V tiles, once the previous item's MMAs are done with them
-                if (!mbar_wait(&bar->kv_empty, (kn & 1) ^ 1, abort_flag, dev_status)) break;
+                if (!mbar_wait_short(&bar->kv_empty, (kn & 1) ^ 1, abort_flag, dev_status)) break;
                 mbar_arrive_expect_tx(&bar->kv_full, 2 * C::STAGE_BYTES);
                 for (int kb = 0; kb < C::KBLK; ++kb) {
                     tma_load_3d(smem + kb * BS * 128, &tmap_k, &bar->kv_full, kb * 64, kblk * BS, bh);
@@ -617,7 +617,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     for (int kv = 0; kv < 2; ++kv) {
                         const uint32_t st = rc % NST;
-                        if (!mbar_wait(&bar->ring_empty[st], ((rc / NST) & 1) ^ 1, abort_flag, dev_status)) {
+                        if (!mbar_wait_short(&bar->ring_empty[st], ((rc / NST) & 1) ^ 1, abort_flag, dev_status)) {
                             ok = false;
                             break;
                         }
@@ -644,7 +644,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t it = 0, rc = 0, tc = 0, kn = 0, on = 0;
             bool ok = true;
             auto wait = [&](uint64_t *b, uint32_t parity) {
-                if (ok && !mbar_wait(b, parity, abort_flag, dev_status)) ok = false;
+                if (ok && !mbar_wait_short(b, parity, abort_flag, dev_status)) ok = false;
                 return ok;
             };
             // D[dcol] = A B^T with A (the item's K or V) and B (a ring tile) both K-major
@@ -731,7 +731,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t it = 0, tc = 0, on = 0;
         while (true) {
             const uint32_t k = it & 1;
-            if (!mbar_wait(&bar->sched_full[k], (it >> 1) & 1, abort_flag, dev_status)) break;
+            if (!mbar_wait_short(&bar->sched_full[k], (it >> 1) & 1, abort_flag, dev_status)) break;
             const int4 item = bar->sched_item[k];
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar->sched_empty[k]);
@@ -765,7 +765,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 int lo = 0, hi = min(BS, N - q0);  // allowed columns: [lo, hi)
                 if (causal) lo = max(0, ku - q0);
                 if (!key_in || qblk < 0 || qblk >= nb) hi = 0;
-                if (!mbar_wait(&bar->st_full, tc & 1, abort_flag, dev_status)) {
+                if (!mbar_wait_short(&bar->st_full, tc & 1, abort_flag, dev_status)) {
                     ok = false;
                     break;
                 }
@@ -774,7 +774,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int c0 = 0; c0 < BS; c0 += 32)
                     tmem_ld32(tmem + lane_base + C::T_S + c0, *reinterpret_cast<uint32_t(*)[32]>(&v[c0]));
-                if (!mbar_wait(&bar->meta[tc % 3], (tc / 3) & 1, abort_flag, dev_status)) {
+                if (!mbar_wait_short(&bar->meta[tc % 3], (tc / 3) & 1, abort_flag, dev_status)) {
                     ok = false;
                     break;
                 }
@@ -812,7 +812,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (lane == 0) mbar_arrive(&bar->p_full);
                 // the next block's LSE and D while the tensor cores work
                 if (j + 1 < count) stage_meta(j + 1, tc + 1);
-                if (!mbar_wait(&bar->dpt_full, tc & 1, abort_flag, dev_status)) {
+                if (!mbar_wait_short(&bar->dpt_full, tc & 1, abort_flag, dev_status)) {
                     ok = false;
                     break;
                 }
@@ -843,7 +843,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (!ok) break;
             // epilogue: dK = (sum of dS^T Q) / sqrt(d), dV = sum of P^T dO
-            if (!mbar_wait(&bar->acc_full, on & 1, abort_flag, dev_status)) break;
+            if (!mbar_wait_short(&bar->acc_full, on & 1, abort_flag, dev_status)) break;
             ++on;
             tc_fence_after();
 #pragma unroll

@@ -78,6 +78,39 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
     }
 }
 
+// try_wait without a suspend-time hint: the hardware parks the thread only for a
+// short, system-dependent time before returning, so it resumes sooner after the
+// phase completes.  The backward passes use it (measured faster there); the
+// forward kernel keeps the hinted wait.
+__device__ __forceinline__ bool mbar_try_wait_short(uint32_t bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(done)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
+// mbar_wait with short try_wait rounds (same bound, same abort and timeout handling).
+__device__ __forceinline__ bool mbar_wait_short(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                                int32_t *dev_status) {
+    const uint32_t a = smem_addr(bar);
+    if (mbar_try_wait_short(a, parity)) return true;
+    const long long t0 = clock64();
+    while (true) {
+        if (mbar_try_wait_short(a, parity)) return true;
+        if (*abort_flag) return false;
+        if (clock64() - t0 > kWaitLimitCycles) {
+            *abort_flag = 1;
+            record_error(dev_status, FVATTN_ERR_DEVICE_TIMEOUT);
+            return false;
+        }
+    }
+}
+
 // Same bound, no abort flag: used during teardown.
 __device__ __forceinline__ bool mbar_wait_teardown(uint64_t *bar, uint32_t parity) {
     const uint32_t a = smem_addr(bar);
