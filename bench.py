@@ -198,14 +198,22 @@ def barrier(world: int):
 
 # --------------------------------------------------------------- CPU oracle
 
-def oracle_sample(w: W.Workload, Q, K, V, budget_s: float, seed: int = 7):
-    """Times the oracle on a bounded sample: full routing, then whole query blocks
-    (128 rows each) drawn at random until the time budget is spent."""
+def oracle_route_timed(w: W.Workload, Q, K):
+    """The oracle's full fp64 routing of the workload and its wall time (s)."""
+    import oracle
+    t0 = time.perf_counter()
+    r = oracle.route(Q, K, w.p, w.bs, nthreads=oracle.default_threads())
+    return r, time.perf_counter() - t0
+
+
+def oracle_sample(w: W.Workload, Q, K, V, budget_s: float, seed: int = 7, routed=None):
+    """Times the oracle on a bounded sample: full routing (or a routing already timed,
+    ``routed`` = (result, seconds)), then whole query blocks (128 rows each) drawn at
+    random until the time budget is spent; the routing time is prorated to the
+    sampled share of the query blocks."""
     import oracle
     threads = oracle.default_threads()
-    t0 = time.perf_counter()
-    r = oracle.route(Q, K, w.p, w.bs, nthreads=threads)
-    t_route = time.perf_counter() - t0
+    r, t_route = routed if routed is not None else oracle_route_timed(w, Q, K)
     counts = r.counts
     rng = np.random.default_rng(seed)
     items = rng.permutation(w.rows)
@@ -244,9 +252,12 @@ def run_reference(args, w, rank, world):
         pass  # the oracle has no warm-up state
     vals = []
     cb = None
-    per_step = max(2.0, 20.0 / max(1, args.steps))
+    # the whole run stays near a minute and a half of oracle time for any --steps:
+    # the routing is timed once and prorated in every step's sample
+    routed = oracle_route_timed(w, Q, K)
+    per_step = min(2.0, max(0.05, 90.0 / max(1, args.steps)))
     for s in range(args.steps):
-        cb = oracle_sample(w, Q, K, V, budget_s=per_step, seed=1000 + s)
+        cb = oracle_sample(w, Q, K, V, budget_s=per_step, seed=1000 + s, routed=routed)
         vals.append(cb["value"])
     v = float(np.mean(vals))
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
