@@ -51,8 +51,13 @@ def _load():
         lib.oracle_attn_bwd.argtypes = [P, P, P, P, i32, i32, i32, i32, i32, i32, P, P, P, P, P, i32]
         lib.oracle_attn_bwd_sampled.argtypes = [P, P, P, P, i32, i32, i32, i32, i32, i32, P, P, P, i64, P, P, P,
                                                 i64, P, P, i32]
+        lib.oracle_quant_e4m3.argtypes = [P, i64, i32, i32, i32, P, P]
+        lib.oracle_e4m3_to_double.argtypes = [ctypes.c_uint8]
+        lib.oracle_e4m3_to_double.restype = dbl
+        lib.oracle_e4m3_from_double.argtypes = [dbl]
+        lib.oracle_e4m3_from_double.restype = ctypes.c_uint8
         for f in ("oracle_pool", "oracle_route", "oracle_attn_rows", "oracle_attn_tiled", "oracle_lpt_order",
-                  "oracle_attn_bwd", "oracle_attn_bwd_sampled"):
+                  "oracle_attn_bwd", "oracle_attn_bwd_sampled", "oracle_quant_e4m3"):
             getattr(lib, f).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -199,6 +204,40 @@ def attn_bwd_sampled(Q, K, V, dO, bs, causal, row_ptr, col_idx, q_tokens, k_toke
     dK[perm] = dKs[: ks.size]
     dV[perm] = dVs[: ks.size]
     return dQ[: q_tokens.size], dK, dV
+
+
+def e4m3_encode(x: float) -> int:
+    """The e4m3 code of one value: nearest, ties to the even code, saturating at 448."""
+    return int(_load().oracle_e4m3_from_double(float(x)))
+
+
+def e4m3_decode_table() -> np.ndarray:
+    """fp64 value of each of the 256 e4m3 codes (NaN for 0x7F and 0xFF)."""
+    lib = _load()
+    return np.array([lib.oracle_e4m3_to_double(c) for c in range(256)], dtype=np.float64)
+
+
+def quant_e4m3(X, bs):
+    """Block quantization of bf16 bit patterns [B,H,N,d] to e4m3: codes uint8
+    [B,H,N,d] and the power-of-two scale exponent of every (batch*head, block),
+    int32 [B,H,nb]; value = e4m3 value of the code * 2^exponent."""
+    X = _bits(X)
+    B, H, N, d = X.shape
+    nb = -(-N // bs)
+    codes = np.empty((B, H, N, d), dtype=np.uint8)
+    exps = np.empty((B, H, nb), dtype=np.int32)
+    rc = _load().oracle_quant_e4m3(_ptr(X), B * H, N, d, bs, _ptr(codes), _ptr(exps))
+    if rc != 0:
+        raise ValueError("oracle_quant_e4m3 failed")
+    return codes, exps
+
+
+def dequant_e4m3(codes, exps, bs):
+    """fp64 values of block-quantized e4m3 data (see :func:`quant_e4m3`)."""
+    B, H, N, d = codes.shape
+    table = e4m3_decode_table()
+    scale = np.ldexp(1.0, np.repeat(exps, bs, axis=2)[:, :, :N])
+    return table[codes] * scale[..., None]
 
 
 def lpt_order(row_ptr: np.ndarray) -> np.ndarray:

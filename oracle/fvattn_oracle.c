@@ -43,6 +43,10 @@
  *   attn_bwd_sampled  equal, value for value, to attn_bwd at the sampled
  *               tokens, and to fp64 torch autograd of dense attention
  *   lpt_order   brute-force sort on small inputs
+ *   e4m3 / quant_e4m3  the format's own values (known codes, ties to even,
+ *               saturation, NaN), round trip of every finite code, monotone
+ *               encoding, block scales putting the block maximum in (224, 448],
+ *               the half-ulp error bound, exact bf16 representability
  */
 #include <math.h>
 #include <pthread.h>
@@ -759,5 +763,79 @@ int oracle_attn_bwd_sampled(const uint16_t *Q, const uint16_t *K, const uint16_t
     bwd_sample_ctx c = {Q, K, V, dO, N, d, bs, causal ? 1 : 0, num_blocks(N, bs), row_ptr, col_idx,
                         1.0 / sqrt((double)d), nq, q_tok, dQ, k_tok, group_ptr, dK, dV};
     parallel_for(nq + ngroups, nthreads, bwd_sample_range, &c);
+    return 0;
+}
+
+/* --------------------------------------------- FP8 (e4m3) block quantization */
+
+/*
+ * For the FP8 attention variant (e4m3 Q, K, V).  The pages name FP8 only as a
+ * data type, so the reading here is the plainest exact one:
+ *   - e4m3 as in the OCP FP8 E4M3FN format: 1 sign bit, 4 exponent bits (bias
+ *     7), 3 mantissa bits, subnormals m * 2^-9, largest finite 448, no
+ *     infinities (0x7F / 0xFF are NaN);
+ *   - one power-of-two scale 2^e per (batch*head, block of bs tokens), the
+ *     smallest e with absmax * 2^-e <= 448 (e = 0 for an all-zero block), so
+ *     that dividing by the scale is exact in any precision;
+ *   - each value x * 2^-e rounded to the nearest e4m3 value, ties to the even
+ *     code, magnitudes above 448 saturated to 448.
+ * Dequantized value = e4m3 value * 2^e.
+ */
+double oracle_e4m3_to_double(uint8_t b) {
+    const int sign = b >> 7, ex = (b >> 3) & 15, man = b & 7;
+    if (ex == 15 && man == 7) return NAN;
+    const double mag = (ex == 0) ? ldexp((double)man, -9) : ldexp(1.0 + man / 8.0, ex - 7);
+    return sign ? -mag : mag;
+}
+
+uint8_t oracle_e4m3_from_double(double x) {
+    if (isnan(x)) return 0x7F;
+    const uint8_t sign = (x < 0.0 || (x == 0.0 && signbit(x))) ? 0x80 : 0x00;
+    const double a = fabs(x);
+    if (a >= 448.0) return (uint8_t)(sign | 0x7E);
+    /* the finite non-negative codes 0x00..0x7E are in increasing order of value:
+       find the two neighbours of a and take the nearer one, ties to the even code */
+    int lo = 0, hi = 0x7E;
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) / 2;
+        if (oracle_e4m3_to_double((uint8_t)mid) <= a) lo = mid;
+        else hi = mid;
+    }
+    const double vlo = oracle_e4m3_to_double((uint8_t)lo), vhi = oracle_e4m3_to_double((uint8_t)hi);
+    int code;
+    if (a - vlo < vhi - a) code = lo;
+    else if (a - vlo > vhi - a) code = hi;
+    else code = (lo % 2 == 0) ? lo : hi;
+    if (a <= vlo) code = lo;
+    return (uint8_t)(sign | code);
+}
+
+/* X: bf16 bit patterns [BH, N, d].  out: e4m3 codes [BH, N, d]; scale_exp: int32
+ * [BH, nb] (the e of each block's scale 2^e).  Rows past N do not exist. */
+int oracle_quant_e4m3(const uint16_t *X, int64_t BH, int N, int d, int bs, uint8_t *out, int32_t *scale_exp) {
+    if (!X || !out || !scale_exp || BH < 1 || N < 1 || d < 1 || bs < 1) return -1;
+    const int64_t nb = num_blocks(N, bs);
+    for (int64_t bh = 0; bh < BH; ++bh) {
+        for (int64_t b = 0; b < nb; ++b) {
+            const int64_t t0 = b * bs, t1 = (b + 1) * bs < N ? (b + 1) * bs : N;
+            double amax = 0.0;
+            for (int64_t t = t0; t < t1; ++t)
+                for (int ch = 0; ch < d; ++ch) {
+                    const double v = fabs(bf16_bits_to_double(X[(bh * N + t) * d + ch]));
+                    if (v > amax) amax = v;
+                }
+            int e = 0;
+            if (amax > 0.0) {
+                e = -200;
+                while (ldexp(amax, -e) > 448.0) ++e;
+            }
+            scale_exp[bh * nb + b] = e;
+            for (int64_t t = t0; t < t1; ++t)
+                for (int ch = 0; ch < d; ++ch) {
+                    const int64_t i = (bh * N + t) * d + ch;
+                    out[i] = oracle_e4m3_from_double(ldexp(bf16_bits_to_double(X[i]), -e));
+                }
+        }
+    }
     return 0;
 }

@@ -533,3 +533,71 @@ def test_attn_bwd_sampled_dense_matches_torch_autograd(oracle_mod):
     sq, sk, sv = oracle_mod.attn_bwd_sampled(Q, K, V, dO, bs, False, row_ptr, col_idx, toks, toks)
     for mine, ref in ((sq, q.grad), (sk, k.grad), (sv, v.grad)):
         assert np.max(np.abs(mine - ref.numpy().reshape(-1, d)[toks])) < 1e-11
+
+
+# ---------------------------------------------------------------- e4m3 quantization
+
+def test_e4m3_known_codes_ties_saturation_and_nan(oracle_mod):
+    """Values of the E4M3FN format itself: exponent bias 7, 3 mantissa bits,
+    subnormals m * 2^-9, largest finite 448, NaN at 0x7F; nearest rounding with
+    ties to the even code; saturation at 448."""
+    enc = oracle_mod.e4m3_encode
+    table = oracle_mod.e4m3_decode_table()
+    assert table[0x38] == 1.0 and table[0xB8] == -1.0 and table[0x7E] == 448.0 and table[0xFE] == -448.0
+    assert table[0x08] == 2.0 ** -6 and table[0x01] == 2.0 ** -9 and table[0x07] == 7 * 2.0 ** -9
+    assert table[0x39] == 1.125 and table[0x3F] == 1.875 and table[0x40] == 2.0
+    assert np.isnan(table[0x7F]) and np.isnan(table[0xFF])
+    assert enc(0.0) == 0x00 and enc(1.0) == 0x38 and enc(-2.0) == 0xC0 and enc(448.0) == 0x7E
+    assert enc(1.0625) == 0x38          # halfway 1 | 1.125: to the even code 0x38
+    assert enc(1.1875) == 0x3A          # halfway 1.125 | 1.25: to the even code 0x3A
+    assert enc(1.07) == 0x39 and enc(1.05) == 0x38
+    assert enc(2.0 ** -10) == 0x00      # halfway 0 | 2^-9: to the even code 0
+    assert enc(3 * 2.0 ** -10) == 0x02  # halfway 2^-9 | 2^-8: to the even code 2
+    assert enc(500.0) == 0x7E and enc(1e30) == 0x7E and enc(-1e30) == 0xFE and enc(464.0) == 0x7E
+    assert enc(float("nan")) == 0x7F
+
+
+def test_e4m3_round_trip_and_monotone(oracle_mod):
+    enc = oracle_mod.e4m3_encode
+    table = oracle_mod.e4m3_decode_table()
+    for c in range(256):
+        if c in (0x7F, 0xFF):
+            continue
+        assert enc(table[c]) == c or (c == 0x80 and enc(table[c]) in (0x00, 0x80)), hex(c)
+    xs = np.linspace(-460.0, 460.0, 20001)
+    vals = table[[enc(x) for x in xs]]
+    assert np.all(np.diff(vals) >= 0)
+
+
+def test_quant_e4m3_block_scales_and_error_bound(oracle_mod):
+    """Every block's scaled maximum lands in (224, 448]; an all-zero block gets the
+    scale 2^0 and zero codes; each value is within half an e4m3 step of the input
+    (relative 2^-4 in the normal range, 2^-10 * scale below it); the dequantized
+    values are exact bf16 values."""
+    rng = np.random.default_rng(31)
+    B, H, N, d, bs = 2, 2, 300, 16, 64
+    x = rng.standard_normal((B, H, N, d)).astype(np.float32)
+    x[0, 1, 64:128] = 0.0                               # an all-zero block
+    x[1, 0, 128:192] *= 1e-30                            # a tiny-magnitude block
+    x[1, 1, 256:] *= 1e20                                # a huge-magnitude ragged last block
+    X = f32_to_bf16_bits(x)
+    codes, exps = oracle_mod.quant_e4m3(X, bs)
+    xv = fvals(X)
+    nb = -(-N // bs)
+    for b in range(B):
+        for h in range(H):
+            for k in range(nb):
+                blk = xv[b, h, k * bs:(k + 1) * bs]
+                amax = np.max(np.abs(blk))
+                e = int(exps[b, h, k])
+                if amax == 0.0:
+                    assert e == 0 and np.all(codes[b, h, k * bs:(k + 1) * bs] == 0)
+                else:
+                    assert 224.0 < amax * 2.0 ** -e <= 448.0
+    deq = oracle_mod.dequant_e4m3(codes, exps, bs)
+    scale = np.ldexp(1.0, np.repeat(exps, bs, axis=2)[:, :, :N])[..., None]
+    err = np.abs(deq - xv)
+    normal = np.abs(xv) >= 2.0 ** -6 * scale
+    assert np.all(err[normal] <= 2.0 ** -4 * np.abs(xv[normal]))
+    assert np.all(err[~normal] <= 2.0 ** -10 * np.broadcast_to(scale, xv.shape)[~normal])
+    assert np.array_equal(fvals(f32_to_bf16_bits(deq.astype(np.float32))), deq)
