@@ -130,6 +130,25 @@ FVATTN_API int fvattn_lpt_order(const int32_t *row_ptr, int64_t rows, int max_co
                      size_t ws_bytes, int32_t *dev_status, fvattn_stream_t stream);
 
 /*
+ * fvattn_quant_e4m3 -- bf16 -> FP8 (e4m3) block quantization, the input step of
+ * the FP8 attention variant (the FVAttn review names FP8 only as a data type; the
+ * reading taken: OCP E4M3FN values -- exponent bias 7, 3 mantissa bits,
+ * subnormals m * 2^-9, largest finite 448).
+ *   X          device bf16 [B,H,N,d], 16-byte aligned.
+ *   out        device uint8 [B,H,N,d], 16-byte aligned: the e4m3 codes.
+ *   scale_exp  device int32 [B,H,ceil(N/block)]: per (batch, head, block of
+ *              `block` tokens) the exponent e of the power-of-two scale 2^e, the
+ *              smallest e with (block max |x|) * 2^-e <= 448 (0 for an all-zero
+ *              block or one holding inf).
+ * Each code is x * 2^-e rounded to the nearest e4m3 value, ties to the even
+ * code, magnitudes above 448 saturated to 448, NaN kept as NaN (0x7F / 0xFF);
+ * value = e4m3 value * 2^e.  d in {64, 128}, block in {64, 128}.  Asynchronous
+ * on `stream`; allocates nothing.  Returns FVATTN_OK or a host-side error.
+ */
+FVATTN_API int fvattn_quant_e4m3(const void *X, int B, int H, int N, int d, int block, uint8_t *out,
+                                 int32_t *scale_exp, fvattn_stream_t stream);
+
+/*
  * fvattn_sparse_fwd -- exact attention restricted to the CSR block mask
  * (FlashAttention review §Model: one fused kernel, tiled matmuls, tiled
  * online softmax; FVAttn review §1: only the selected key blocks are read).

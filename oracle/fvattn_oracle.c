@@ -776,7 +776,8 @@ int oracle_attn_bwd_sampled(const uint16_t *Q, const uint16_t *K, const uint16_t
  *     infinities (0x7F / 0xFF are NaN);
  *   - one power-of-two scale 2^e per (batch*head, block of bs tokens), the
  *     smallest e with absmax * 2^-e <= 448 (e = 0 for an all-zero block), so
- *     that dividing by the scale is exact in any precision;
+ *     that dividing by the scale is exact in any precision (a block holding
+ *     inf keeps 2^0; NaN does not count toward the maximum);
  *   - each value x * 2^-e rounded to the nearest e4m3 value, ties to the even
  *     code, magnitudes above 448 saturated to 448.
  * Dequantized value = e4m3 value * 2^e.
@@ -825,7 +826,7 @@ int oracle_quant_e4m3(const uint16_t *X, int64_t BH, int N, int d, int bs, uint8
                     if (v > amax) amax = v;
                 }
             int e = 0;
-            if (amax > 0.0) {
+            if (amax > 0.0 && isfinite(amax)) { /* a block holding inf keeps the scale 2^0 */
                 e = -200;
                 while (ldexp(amax, -e) > 448.0) ++e;
             }

@@ -95,6 +95,12 @@ def test_invalid_arguments_rejected_before_any_device_work(lib):
     # causal must be 0 or 1
     assert lib.fvattn_sparse_fwd(fake, fake, fake, fake, fake, 1, 1, 128, 64, 64, 2, fake, fake, fake, 1 << 20,
                                  fake, None) == -1
+    # e4m3 quantization: unsupported d, null pointers, misaligned input
+    assert lib.fvattn_quant_e4m3(fake, 1, 1, 128, 96, 64, fake, fake, None) == -2
+    assert lib.fvattn_quant_e4m3(None, 1, 1, 128, 64, 64, fake, fake, None) == -1
+    assert lib.fvattn_quant_e4m3(fake, 1, 1, 128, 64, 64, fake, None, None) == -1
+    assert lib.fvattn_quant_e4m3(P(18), 1, 1, 128, 64, 64, fake, fake, None) == -3
+    assert lib.fvattn_quant_e4m3(fake, 0, 1, 128, 64, 64, fake, fake, None) == -1
     # routing supports at most 1024 blocks per sequence
     assert lib.fvattn_route(fake, fake, 1, 1, 1025 * 64, 64, 64, 0.5, fake, fake, 4, fake, fake, 1 << 30, fake,
                             None) == -2

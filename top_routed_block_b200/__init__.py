@@ -65,6 +65,7 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         "fvattn_lpt_workspace_bytes": (SZ, [I64, I]),
         "fvattn_route": (I, [P, P, I, I, I, I, I, D, P, P, I64, P, P, SZ, P, P]),
         "fvattn_lpt_order": (I, [P, I64, I, P, P, SZ, P, P]),
+        "fvattn_quant_e4m3": (I, [P, I, I, I, I, I, P, P, P]),
         "fvattn_sparse_fwd": (I, [P, P, P, P, P, I, I, I, I, I, I, P, P, P, SZ, P, P]),
         "fvattn_sparse_fwd_noalloc": (I, [P, P, P, P, P, I, I, I, I, I, I, P, P, P, P]),
         "fvattn_test_sparse_fwd_stall": (I, [P, P, P, P, P, I, I, I, I, I, I, P, P, P, SZ, P, P]),
@@ -185,6 +186,22 @@ def fvattn_lpt_order(row_ptr: torch.Tensor, max_count: int, *, stream=None, orde
                               _ptr(dev_status), _stream_ptr(stream))
     _check(rc, "fvattn_lpt_order")
     return order[:rows], dev_status
+
+
+def fvattn_quant_e4m3(X: torch.Tensor, block: int, *, stream=None, out: torch.Tensor | None = None,
+                      scale_exp: torch.Tensor | None = None):
+    """bf16 [B,H,N,d] -> (e4m3 codes uint8 [B,H,N,d], scale exponents int32 [B,H,nb]);
+    value = e4m3 value of the code * 2^exponent."""
+    lib = load_library()
+    B, H, N, d = _shape(X)
+    nb = num_blocks(N, block)
+    if out is None:
+        out = torch.empty((B, H, N, d), dtype=torch.uint8, device=X.device)
+    if scale_exp is None:
+        scale_exp = torch.empty((B, H, nb), dtype=torch.int32, device=X.device)
+    rc = lib.fvattn_quant_e4m3(_ptr(X), B, H, N, d, int(block), _ptr(out), _ptr(scale_exp), _stream_ptr(stream))
+    _check(rc, "fvattn_quant_e4m3")
+    return out, scale_exp
 
 
 def fvattn_sparse_fwd(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, row_ptr: torch.Tensor, col_idx: torch.Tensor,

@@ -15,6 +15,7 @@
 #include "attn_fwd.cuh"
 #include "common.cuh"
 #include "lpt.cuh"
+#include "quant.cuh"
 #include "route.cuh"
 
 using namespace fvattn;
@@ -224,6 +225,17 @@ int fvattn_lpt_order(const int32_t *row_ptr, int64_t rows, int max_count, int32_
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if ((rc = from_cuda(cudaMemsetAsync(dev_status, 0, sizeof(int32_t), s))) != FVATTN_OK) return rc;
     return from_cuda(launch_lpt_order(row_ptr, rows, max_count, order, workspace, dev_status, s));
+}
+
+int fvattn_quant_e4m3(const void *X, int B, int H, int N, int d, int block, uint8_t *out, int32_t *scale_exp,
+                      fvattn_stream_t stream) {
+    int rc = check_shape(B, H, N, d, block);
+    if (rc != FVATTN_OK) return rc;
+    if (!X || !out || !scale_exp) return FVATTN_ERR_INVALID_ARG;
+    if (!aligned16(X) || !aligned16(out) || (reinterpret_cast<uintptr_t>(scale_exp) & 3u)) return FVATTN_ERR_ALIGNMENT;
+    if ((rc = check_device()) != FVATTN_OK) return rc;
+    return from_cuda(launch_quant_e4m3(X, static_cast<int64_t>(B) * H, N, d, block, out, scale_exp,
+                                       reinterpret_cast<cudaStream_t>(stream)));
 }
 
 static int sparse_fwd_impl(const void *Q, const void *K, const void *V, const int32_t *row_ptr,
