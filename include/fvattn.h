@@ -131,9 +131,12 @@ FVATTN_API int fvattn_lpt_order(const int32_t *row_ptr, int64_t rows, int max_co
 
 /*
  * fvattn_quant_e4m3 -- bf16 -> FP8 (e4m3) block quantization, the input step of
- * the FP8 attention variant (the FVAttn review names FP8 only as a data type; the
- * reading taken: OCP E4M3FN values -- exponent bias 7, 3 mantissa bits,
- * subnormals m * 2^-9, largest finite 448).
+ * the FP8 attention variant.  "Accelerating HunyuanVideo inference with
+ * ParaAttention" (WaveSpeed), § "FP8 dynamic quantization", quantizes weights and
+ * activations to FP8 at run time to use the 8-bit tensor cores, without naming a
+ * format or a scaling; the reading taken: OCP E4M3FN values -- exponent bias 7,
+ * 3 mantissa bits, subnormals m * 2^-9, largest finite 448 -- with scales
+ * computed from the data (dynamic), one per block.
  *   X          device bf16 [B,H,N,d], 16-byte aligned.
  *   out        device uint8 [B,H,N,d], 16-byte aligned: the e4m3 codes.
  *   scale_exp  device int32 [B,H,ceil(N/block)]: per (batch, head, block of

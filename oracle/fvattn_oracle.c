@@ -769,8 +769,10 @@ int oracle_attn_bwd_sampled(const uint16_t *Q, const uint16_t *K, const uint16_t
 /* --------------------------------------------- FP8 (e4m3) block quantization */
 
 /*
- * For the FP8 attention variant (e4m3 Q, K, V).  The pages name FP8 only as a
- * data type, so the reading here is the plainest exact one:
+ * For the FP8 attention variant (e4m3 Q, K, V).  "Accelerating HunyuanVideo
+ * inference with ParaAttention" (WaveSpeed), § "FP8 dynamic quantization",
+ * quantizes activations to FP8 at run time but names no format or scaling, so
+ * the reading here is the plainest exact one:
  *   - e4m3 as in the OCP FP8 E4M3FN format: 1 sign bit, 4 exponent bits (bias
  *     7), 3 mantissa bits, subnormals m * 2^-9, largest finite 448, no
  *     infinities (0x7F / 0xFF are NaN);

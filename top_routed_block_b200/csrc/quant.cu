@@ -1,4 +1,7 @@
-// quant.cu -- bf16 -> e4m3 block quantization for the FP8 attention variant.
+// quant.cu -- bf16 -> e4m3 block quantization for the FP8 attention variant
+// ("Accelerating HunyuanVideo inference with ParaAttention" (WaveSpeed), § "FP8
+// dynamic quantization": activations quantized to FP8 at run time; the format and
+// the per-block power-of-two scaling below are the reading taken).
 //
 // Per (batch*head, block of `bs` tokens): the block's largest magnitude fixes a
 // power-of-two scale 2^e, the smallest e with max * 2^-e <= 448; every value is
