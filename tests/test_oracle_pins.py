@@ -138,6 +138,44 @@ def test_attn_rows_matches_decimal_brute_force(oracle_mod, N, bs, d, causal):
                 assert abs(impl_lse[g] - float(ref_lse)) <= 1e-12
 
 
+@pytest.mark.parametrize("causal", [False, True])
+def test_attn_rows_equals_dense_attention_with_minus_inf_bias(oracle_mod, causal):
+    """Masked-dense equivalence: the sparse attention on a block mask M equals dense
+    softmax(Q K^T / sqrt(d) + bias) V over all N keys, with bias 0 on M (and u <= t if
+    causal) and -inf elsewhere, written as fp64 matrix algebra; rows whose bias is all
+    -inf give O = 0 and LSE = -inf.  Ragged last block, empty and full rows."""
+    rng = np.random.default_rng(17 + causal)
+    B, H, N, d, bs = 2, 2, 200, 16, 64
+    nb = -(-N // bs)
+    row_ptr, col_idx = random_csr(rng, B * H * nb, nb, p_keep=0.5, allow_empty=True)
+    Q, K, V = (rand_bf16(rng, (B, H, N, d)) for _ in range(3))
+    tokens = np.arange(B * H * N, dtype=np.int64)
+    O, LSE = oracle_mod.attn_rows(Q, K, V, bs, causal, row_ptr, col_idx, tokens)
+    Qf, Kf, Vf = fvals(Q), fvals(K), fvals(V)
+    for bh in range(B * H):
+        b, h = divmod(bh, H)
+        allowed = np.zeros((N, N), bool)  # [query token, key token]
+        for qb in range(nb):
+            row = bh * nb + qb
+            for kb in col_idx[row_ptr[row]:row_ptr[row + 1]]:
+                allowed[qb * bs:(qb + 1) * bs, kb * bs:(kb + 1) * bs] = True
+        if causal:
+            allowed &= np.tril(np.ones((N, N), bool))
+        S = Qf[b, h] @ Kf[b, h].T / math.sqrt(d) + np.where(allowed, 0.0, -np.inf)
+        m = S.max(axis=1, keepdims=True)
+        has = np.isfinite(m[:, 0])
+        E = np.where(has[:, None], np.exp(S - np.where(has[:, None], m, 0.0)), 0.0)
+        z = E.sum(axis=1)
+        ref_o = np.where(has[:, None], (E @ Vf[b, h]) / np.where(has, z, 1.0)[:, None], 0.0)
+        ref_lse = np.where(has, m[:, 0] + np.log(np.where(has, z, 1.0)), -np.inf)
+        got_o = O[bh * N:(bh + 1) * N]
+        got_lse = LSE[bh * N:(bh + 1) * N]
+        assert np.max(np.abs(got_o - ref_o)) < 1e-12
+        assert np.array_equal(np.isinf(got_lse), np.isinf(ref_lse))
+        fin = np.isfinite(ref_lse)
+        assert np.max(np.abs(got_lse[fin] - ref_lse[fin])) < 1e-12
+
+
 def test_attn_closed_form_zero_keys_gives_mean_of_values(oracle_mod):
     rng = np.random.default_rng(7)
     B, H, N, d, bs = 1, 1, 40, 8, 16
