@@ -137,7 +137,7 @@ def test_attention_sweep_sampled(w, oracle_mod):
     dQ, dK, dV = to_dev(Q), to_dev(K), to_dev(V)
     rp, ci, _ = gpu_route(dQ, dK, w.p, w.bs)
     O, LSE = run_fwd(dQ, dK, dV, rp, ci, w.bs, False)
-    tokens = W.sample_tokens(w, per_head_blocks=1, rows_per_block=12)
+    tokens = W.sample_tokens(w, per_head_blocks=2, rows_per_block=12)
     Oref, Lref = oracle_mod.attn_rows(Q, K, V, w.bs, False, rp, ci, tokens)
     compare_attention(O, LSE, Oref, Lref, tokens, w.d, w.name)
 
