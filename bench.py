@@ -34,7 +34,7 @@ METRIC = "effective TFLOP/s & tensor-pipe % of peak (sparse attn fwd, p=0.9); ro
 UNIT = "TFLOP/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 ROUTE_KERNELS_PER_CALL = 4      # pool, select, CSR scan, CSR scatter
-FWD_KERNELS_PER_CALL = 5        # item list, LPT rank, LPT offsets, LPT scatter, attention
+FWD_KERNELS_PER_CALL = 3        # head ranks, row order, attention
 
 
 def load_peaks():
@@ -48,7 +48,7 @@ def load_peaks():
 
 KERNEL_SOURCES = ("top_routed_block_b200/csrc/attn_fwd.cu", "top_routed_block_b200/csrc/ptx_sm100.cuh",
                   "top_routed_block_b200/csrc/common.cuh")
-TRAFFIC_SUMMARY = "profiles/dram_traffic_video_dit.md"
+TRAFFIC_RECORD = "profiles/dram_traffic_video_dit.json"
 
 
 def kernel_source_hash() -> str:
@@ -61,23 +61,32 @@ def kernel_source_hash() -> str:
 
 
 def recorded_traffic(workload: str):
-    """DRAM bytes per attention launch from the committed ncu summary, if it was
-    taken on this workload with the current kernel source; else None."""
-    p = os.path.join(ROOT, TRAFFIC_SUMMARY)
-    if not os.path.exists(p):
+    """DRAM bytes per attention launch from the committed ncu record (JSON), if it
+    was taken on this workload with the current kernel source; else None."""
+    p = os.path.join(ROOT, TRAFFIC_RECORD)
+    try:
+        with open(p) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
         return None
-    fields = {}
-    with open(p) as f:
-        for line in f:
-            if ":" in line and line.strip().startswith("- "):
-                k, v = line.strip()[2:].split(":", 1)
-                fields[k.strip()] = v.strip().strip("`")
-    if fields.get("workload") != workload or fields.get("kernel_source_sha256") != kernel_source_hash():
+    if rec.get("workload") != workload or rec.get("kernel_source_sha256") != kernel_source_hash():
         return None
     try:
-        return float(fields["traffic_bytes_per_launch"])
-    except (KeyError, ValueError):
+        return float(rec["dram_bytes_read"]) + float(rec["dram_bytes_write"])
+    except (KeyError, TypeError, ValueError):
         return None
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.lower().startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
 
 
 def eff_flops(nnz: int, w: W.Workload) -> float:
@@ -237,6 +246,7 @@ def oracle_sample(w: W.Workload, Q, K, V, budget_s: float, seed: int = 7, routed
         "value": done_flops / total_t / 1e12,
         "unit": UNIT,
         "cores": threads,
+        "cpu_model": cpu_model(),
         "kind": "oracle",
         "sample": (f"{w.name}: full fp64 routing ({t_route:.2f} s, prorated by {frac:.4f}) + {n_items} of "
                    f"{w.rows} query blocks of attention ({t_attn:.1f} s)"),
@@ -265,13 +275,82 @@ def run_reference(args, w, rank, world):
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "block": w.bs, "p": w.p,
                        "causal": w.causal, "l2": "inputs larger than L2"},
-            "cpu_baseline": {"value": v, "unit": UNIT, "cores": cb["cores"], "kind": "oracle",
-                             "sample": cb["sample"]},
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": cb["cores"], "cpu_model": cb["cpu_model"],
+                             "kind": "oracle", "sample": cb["sample"]},
             "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
 # ------------------------------------------------------------ GPU (ours)
+
+# Workloads timed beside the headline one, each for a few steps in the same run.
+CONFIG_SET = ("tiny", "dense", "dense_causal", "long_video", "sweep_d64_s1_p0.9", "sweep_d64_s05_8_p0.9",
+              "sweep_d128_s1_p0.9", "sweep_d128_s05_8_p0.9")
+
+
+def causal_block_csr(w: W.Workload, dev):
+    """The dense causal block mask (every key block kb <= qb of every head), the mask a
+    causal workload runs on (the pages define no causal top-p routing)."""
+    import torch
+    nb = w.nb
+    counts = torch.arange(1, nb + 1, dtype=torch.int64, device=dev).repeat(w.B * w.H)
+    row_ptr = torch.zeros(counts.numel() + 1, dtype=torch.int64, device=dev)
+    row_ptr[1:] = torch.cumsum(counts, 0)
+    tri = torch.tril_indices(nb, nb, device=dev)[1].to(torch.int32)      # row-major lower triangle: columns
+    col_idx = tri.repeat(w.B * w.H)
+    return row_ptr.to(torch.int32), col_idx.contiguous()
+
+
+def time_config(w: W.Workload, dev, stream, steps: int, burst: float) -> dict:
+    """Routing and attention of one more workload, timed like the headline one (CUDA events
+    per call on the launching stream, after 3 warm-up steps)."""
+    import torch
+
+    import top_routed_block_b200 as fv
+    Qh, Kh, Vh = W.generate(w)
+    dQ, dK, dV = (torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev) for a in (Qh, Kh, Vh))
+    del Qh, Kh, Vh
+    plan = fv.FvattnPlan(w.B, w.H, w.N, w.d, w.bs, device=dev)
+    rp = ci = None
+    if w.causal:
+        rp, ci = causal_block_csr(w, dev)
+
+    def route():
+        if not w.causal:
+            plan.run_route(dQ, dK, w.p, stream=stream)
+
+    def fwd():
+        plan.run_fwd(dQ, dK, dV, w.causal, row_ptr=rp, col_idx=ci, stream=stream)
+
+    for _ in range(3):
+        route()
+        fwd()
+    plan.check()
+    nnz = int((rp if w.causal else plan.route.row_ptr)[-1].item())
+    flops = eff_flops(nnz, w)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    torch.cuda.synchronize(dev)
+    for e0, e1, e2 in ev:
+        e0.record(stream)
+        route()
+        e1.record(stream)
+        fwd()
+        e2.record(stream)
+    torch.cuda.synchronize(dev)
+    plan.check()
+    r_ms = statistics.mean(a.elapsed_time(b) for a, b, _ in ev)
+    a_ms = statistics.mean(b.elapsed_time(c) for _, b, c in ev)
+    out = {"B": w.B, "H": w.H, "N": w.N, "d": w.d, "block": w.bs, "p": w.p, "causal": w.causal,
+           "nnz_blocks": nnz, "density": nnz / (w.B * w.H * w.nb * w.nb), "steps": steps,
+           "attn_ms": a_ms, "attn_tflops": flops / (a_ms * 1e-3) / 1e12,
+           "attn_frac_of_burst": flops / (a_ms * 1e-3) / 1e12 / burst,
+           "route_ms": None if w.causal else r_ms,
+           "route_frac": None if w.causal else r_ms / (r_ms + a_ms),
+           "step_tflops": flops / ((a_ms + (0.0 if w.causal else r_ms)) * 1e-3) / 1e12}
+    del dQ, dK, dV, plan
+    torch.cuda.empty_cache()
+    return out
+
 
 def run_ours(args, w, rank, world, local):
     import torch
@@ -290,14 +369,25 @@ def run_ours(args, w, rank, world, local):
     plan = fv.FvattnPlan(w.B, w.H, w.N, w.d, w.bs, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    def step():
-        plan.run_route(dQ, dK, w.p, stream=stream)
-        plan.run_fwd(dQ, dK, dV, w.causal, stream=stream)
+    # causal workloads run on the dense lower-triangle block mask, without routing
+    mask = causal_block_csr(w, dev) if w.causal else None
+
+    def route():
+        if mask is None:
+            plan.run_route(dQ, dK, w.p, stream=stream)
+
+    def fwd():
+        plan.run_fwd(dQ, dK, dV, w.causal, row_ptr=None if mask is None else mask[0],
+                     col_idx=None if mask is None else mask[1], stream=stream)
+
+    def mask_csr():
+        return (plan.route.row_ptr, plan.route.col_idx) if mask is None else mask
 
     for _ in range(max(3, args.warmup)):
-        step()
+        route()
+        fwd()
     plan.check()
-    nnz = int(plan.route.row_ptr[-1].item())
+    nnz = int(mask_csr()[0][-1].item())
     flops = eff_flops(nnz, w)
 
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
@@ -312,9 +402,9 @@ def run_ours(args, w, rank, world, local):
     for s in range(args.steps):
         e0, e1, e2 = ev[s]
         e0.record(stream)
-        plan.run_route(dQ, dK, w.p, stream=stream)
+        route()
         e1.record(stream)
-        plan.run_fwd(dQ, dK, dV, w.causal, stream=stream)
+        fwd()
         e2.record(stream)
     t_end.record(stream)
     torch.cuda.synchronize(dev)
@@ -360,13 +450,13 @@ def run_ours(args, w, rank, world, local):
     # Load balance over the SMs (outside the timed region): busy time of every CTA of the
     # persistent grid, with the head-major longest-first queue and with rows in index order.
     # The host-buffer path above routed chunk by chunk into the plan: route the whole batch again.
-    plan.run_route(dQ, dK, w.p, stream=stream)
+    route()
     balance = {}
     for name, natural in (("lpt", False), ("natural", True)):
         runs = []
         for _ in range(3):
             a.record(stream)
-            _, _, st, busy = fv.fvattn_sparse_fwd_profiled(dQ, dK, dV, plan.route.row_ptr, plan.route.col_idx, w.bs,
+            _, _, st, busy = fv.fvattn_sparse_fwd_profiled(dQ, dK, dV, *mask_csr(), w.bs,
                                                            w.causal, natural_order=natural, stream=stream, O=plan.O,
                                                            LSE=plan.LSE, workspace=plan.fwd_ws,
                                                            dev_status=plan.status[1:2])
@@ -381,7 +471,7 @@ def run_ours(args, w, rank, world, local):
     # Backward (outside the timed region): gradients of the same attention for a random dO.
     bwd = None
     if w.bs == 128:
-        plan.run_fwd(dQ, dK, dV, w.causal, stream=stream)
+        fwd()
         gen = torch.Generator(device=dev).manual_seed(1234)
         dO = torch.randn(dQ.shape, device=dev, dtype=torch.float32, generator=gen).to(torch.bfloat16)
         ws_b = torch.empty(fv.fvattn_bwd_workspace_bytes(w.B, w.H, w.N, w.bs), dtype=torch.uint8, device=dev)
@@ -389,7 +479,7 @@ def run_ours(args, w, rank, world, local):
         st_b = torch.zeros(1, dtype=torch.int32, device=dev)
 
         def bwd_call():
-            fv.fvattn_sparse_bwd(dQ, dK, dV, plan.O, plan.LSE, dO, plan.route.row_ptr, plan.route.col_idx, w.bs,
+            fv.fvattn_sparse_bwd(dQ, dK, dV, plan.O, plan.LSE, dO, *mask_csr(), w.bs,
                                  w.causal, stream=stream, dQ=gQ, dK=gK, dV=gV, workspace=ws_b, dev_status=st_b)
         for _ in range(2):
             bwd_call()
@@ -409,16 +499,30 @@ def run_ours(args, w, rank, world, local):
                        "outside the timed region"}
         del gQ, gK, gV, ws_b, dO
 
+    peaks, peak_src = load_peaks()
+    configs = None
+    if world == 1 and not args.no_configs:
+        # the other workloads, measured in the same run under their own clock record
+        del hO, hL
+        torch.cuda.empty_cache()
+        cfg_sampler = ClockSampler(gpu_selector(dev))
+        cfg_sampler.start()
+        configs = {name: time_config(W.ALL[name], dev, stream, args.config_steps, float(peaks["bf16_tflops"]))
+                   for name in CONFIG_SET if name != w.name}
+        configs["clocks"] = cfg_sampler.stop()
+        configs["note"] = ("each workload: 3 warm-up steps, then per-call CUDA events over config_steps steps; "
+                           "attn = the fvattn_sparse_fwd call, route = the fvattn_route call; the causal "
+                           "workload runs on the dense lower-triangle block mask, without routing")
     if rank != 0:
         return
-    peaks, peak_src = load_peaks()
-    peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
-    burst = float(peaks["bf16_tflops"])
+    peak = float(peaks["bf16_tflops"])
+    sustained = float(peaks.get("bf16_tflops_sustained", peak))
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         cpu = oracle_sample(w, Qh, Kh, Vh, budget_s=args.cpu_budget)
         cpu.pop("route_s_full", None)
-    counts = plan.route.head_counts.cpu().numpy()
+    rp_np = mask_csr()[0].cpu().numpy().astype(np.int64)
+    counts = (rp_np[w.nb::w.nb] - rp_np[0:-1:w.nb])
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -430,10 +534,12 @@ def run_ours(args, w, rank, world, local):
                    "parallelism": f"replicas x{world}"},
         "attn_tflops": attn_tflops, "attn_ms": attn_ms, "route_ms": r_ms, "timing": timing,
         "route_frac": r_ms / (r_ms + attn_ms),
-        "tensor_frac_of_burst_peak": attn_tflops / burst,
+        "tensor_frac_of_sustained_peak": attn_tflops / sustained,
         "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peak, "unit": "TFLOP/s",
                      "frac": attn_tflops / peak, "traffic": recorded_traffic(w.name),
-                     "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside back-to-back steps)",
+                     "frac_of_sustained": attn_tflops / sustained,
+                     "peak_source": f"{peak_src} bf16_tflops (burst: the timed region is well under a second "
+                                    f"of back-to-back steps); frac_of_sustained divides by bf16_tflops_sustained",
                      "note": "achieved = 4*block^2*d*nnz / mean CUDA-event time of the fvattn_sparse_fwd call "
                              "(its 3 small ordering kernels included)"},
         "route_roofline": {"bound": "hbm", "pool_bytes": 2 * elem * 2,
@@ -446,7 +552,8 @@ def run_ours(args, w, rank, world, local):
         "load_balance": dict(balance, note="LIF = max / mean busy time over the CTAs of the persistent grid "
                                            "(global timer, one call each); lpt = the head-major longest-first "
                                            "queue fvattn_sparse_fwd uses, natural = rows in index order"),
-        "bwd": None if bwd is None else dict(bwd, frac_of_sustained=bwd["tflops_effective"] / peak),
+        "bwd": None if bwd is None else dict(bwd, frac_of_burst=bwd["tflops_effective"] / peak,
+                                              frac_of_sustained=bwd["tflops_effective"] / sustained),
         "mufu": {"exp_per_s": float(nnz) * w.bs * w.bs / (attn_ms * 1e-3),
                  "ceiling_at_max_clock": 16.0 * sms * float(peaks.get("sm_max_mhz", 1965.0)) * 1e6,
                  "frac": float(nnz) * w.bs * w.bs / (attn_ms * 1e-3)
@@ -457,6 +564,7 @@ def run_ours(args, w, rank, world, local):
         "gpu_launches": args.steps * (ROUTE_KERNELS_PER_CALL + FWD_KERNELS_PER_CALL),
         "clocks": clocks,
         "cpu_baseline": cpu,
+        "configs": configs,
     }
     print(json.dumps(line), flush=True)
 
@@ -470,6 +578,8 @@ def main():
     ap.add_argument("--workload", default=W.VIDEO.name, choices=sorted(W.ALL))
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true", help="skip the other workloads' timings")
+    ap.add_argument("--config-steps", type=int, default=10)
     args = ap.parse_args()
     w = W.ALL[args.workload]
     if args.impl == "reference":

@@ -227,9 +227,12 @@ FVATTN_API int fvattn_attention_host(const void *hQ, const void *hK, const void 
  * exits.  Shapes that need more return FVATTN_ERR_CAPACITY without launching
  * anything (about 1M rows B*H*ceil(N/block) at most).
  *
- * The first call on each device looks up the array's device address
- * (cudaGetSymbolAddress, with that device current) and caches it; make that first
- * call before any stream capture.  The call allocates nothing: no cudaMalloc,
+ * Each call made outside stream capture looks up the array's device address
+ * (cudaGetSymbolAddress, with the call's device current; a lookup allocates
+ * nothing) and keeps it per device; a call made while `stream` is capturing uses
+ * the address kept by the last call outside capture, so the first call on each
+ * device must come before any stream capture, and a call after a device reset
+ * must also come before capture.  The call allocates nothing: no cudaMalloc,
  * cudaFree or allocating library routine.  All calls on a device share the one
  * array, which keeps the previous call's contents (the parts that must start at
  * zero are cleared on the stream by each call), so calls whose executions overlap
@@ -303,6 +306,25 @@ FVATTN_API int fvattn_sparse_fwd_profiled(const void *Q, const void *K, const vo
                                           const int32_t *col_idx, int B, int H, int N, int d, int block, int causal,
                                           void *O, float *LSE, void *workspace, size_t ws_bytes, int32_t *dev_status,
                                           int order_mode, int64_t *cta_busy_ns, int *grid, fvattn_stream_t stream);
+
+/*
+ * fvattn_attn_work_order -- the order in which fvattn_sparse_fwd takes its work
+ * items (CSR rows, one query block of one head each), written to order[0 .. rows)
+ * with rows = B*H*ceil(N/block).  FVAttn review §1 "RLB" balances per-head work at
+ * run time once the mask is known; on one GPU the SMs pop the rows from this queue:
+ * heads by their total selected blocks (descending, equal totals by lower head
+ * index), and inside a head its rows by block count (descending, equal counts by
+ * lower row index).  The same kernels run inside fvattn_sparse_fwd; this call
+ * exposes their result (for checks and diagnostics).
+ *   row_ptr    device int32[rows+1], the CSR of fvattn_route (or a caller's mask).
+ *   order      device int32[rows] (out): global row ids r = (b*H+h)*nb + i.
+ *   workspace  device, fvattn_fwd_workspace_bytes(B,H,N,block) bytes, 16-byte aligned.
+ * Asynchronous on `stream`.  Errors: bad sizes or null pointers
+ * FVATTN_ERR_INVALID_ARG; B*H > 4096 or ceil(N/block) > 4096
+ * FVATTN_ERR_UNSUPPORTED; short workspace FVATTN_ERR_CAPACITY.
+ */
+FVATTN_API int fvattn_attn_work_order(const int32_t *row_ptr, int B, int H, int N, int block, int32_t *order,
+                                      void *workspace, size_t ws_bytes, fvattn_stream_t stream);
 
 /* Compiled-in build description (architecture, version), static string. */
 FVATTN_API const char *fvattn_build_info(void);

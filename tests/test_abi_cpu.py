@@ -115,3 +115,11 @@ def test_binding_fails_loudly_without_library(tmp_path):
             fv.load_library(str(tmp_path / "missing.so"))
     finally:
         fv._lib = saved
+
+
+def test_noalloc_rejects_shapes_beyond_its_scratch_without_a_gpu(lib):
+    # Null pointers everywhere: the size check must fail first; were it to regress,
+    # the null-pointer check would still stop the call before any device work.
+    B, H, N, block = 16, 256, 65536, 128
+    assert lib.fvattn_sparse_fwd_noalloc(None, None, None, None, None, B, H, N, 128, block, 0, None, None, None,
+                                         None) == -4

@@ -41,3 +41,45 @@ def test_lpt_count_out_of_range_reported():
     order, st = fv.fvattn_lpt_order(torch.from_numpy(rp).cuda(), 8)
     torch.cuda.synchronize()
     assert int(st.item()) == fv.FVATTN_ERR_BAD_CSR
+
+
+def _head_major_order(rp, BH, nb):
+    """Brute force: heads by total selected blocks (descending, ties by lower head),
+    then the rows of each head by block count (descending, ties by lower row)."""
+    counts = np.diff(rp.astype(np.int64)).reshape(BH, nb)
+    heads = sorted(range(BH), key=lambda h: (-int(counts[h].sum()), h))
+    out = []
+    for h in heads:
+        out += [h * nb + i for i in sorted(range(nb), key=lambda i: (-int(counts[h, i]), i))]
+    return np.array(out, np.int32)
+
+
+@pytest.mark.parametrize("B,H,N,block,maxc,seed", [(1, 1, 128, 128, 1, 0), (1, 3, 1000, 128, 8, 1),
+                                                   (2, 5, 4000, 64, 63, 2), (1, 40, 32760, 128, 256, 3),
+                                                   (4, 1024, 1280, 128, 10, 4)])
+def test_attention_work_order_is_head_major_longest_first(B, H, N, block, maxc, seed):
+    """The queue fvattn_sparse_fwd pops its work items from, against a brute-force sort
+    (many equal counts and equal head totals, so the tie-breaks are exercised)."""
+    import top_routed_block_b200 as fv
+    rng = np.random.default_rng(seed)
+    nb = -(-N // block)
+    BH = B * H
+    counts = rng.integers(0, min(maxc, nb) + 1, size=(BH, nb))
+    counts[rng.random((BH, nb)) < 0.4] = min(maxc, nb) // 2
+    if BH >= 4:
+        counts[1] = counts[3]                     # two heads with equal totals
+    rp = np.zeros(BH * nb + 1, np.int32)
+    rp[1:] = np.cumsum(counts.reshape(-1))
+    order = fv.fvattn_attn_work_order(torch.from_numpy(rp).cuda(), B, H, N, block)
+    torch.cuda.synchronize()
+    assert np.array_equal(order.cpu().numpy(), _head_major_order(rp, BH, nb))
+
+
+def test_attention_work_order_on_routed_mask():
+    import top_routed_block_b200 as fv
+    w = W.VIDEO
+    Q, K, _ = W.generate(w)
+    rp, _, _ = gpu_route(to_dev(Q), to_dev(K), w.p, w.bs)
+    order = fv.fvattn_attn_work_order(torch.from_numpy(rp).cuda(), w.B, w.H, w.N, w.bs)
+    torch.cuda.synchronize()
+    assert np.array_equal(order.cpu().numpy(), _head_major_order(rp, w.B * w.H, w.nb))

@@ -70,6 +70,7 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         "fvattn_sparse_fwd_noalloc": (I, [P, P, P, P, P, I, I, I, I, I, I, P, P, P, P]),
         "fvattn_test_sparse_fwd_stall": (I, [P, P, P, P, P, I, I, I, I, I, I, P, P, P, SZ, P, P]),
         "fvattn_sparse_fwd_profiled": (I, [P, P, P, P, P, I, I, I, I, I, I, P, P, P, SZ, P, I, P, P, P]),
+        "fvattn_attn_work_order": (I, [P, I, I, I, I, P, P, SZ, P]),
         "fvattn_bwd_workspace_bytes": (SZ, [I, I, I, I]),
         "fvattn_sparse_bwd": (I, [P, P, P, P, P, P, P, P, I, I, I, I, I, I, P, P, P, P, SZ, P, P]),
         "fvattn_attention_host": (I, [P, P, P, I, I, I, I, I, D, I, P, P, P, P, P, P, P, P, P, I64, P, P, SZ, P, SZ,
@@ -259,6 +260,22 @@ def fvattn_sparse_fwd_profiled(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor
                                         _stream_ptr(stream))
     _check(rc, "fvattn_sparse_fwd_profiled")
     return O, LSE, dev_status, busy[: grid.value]
+
+
+def fvattn_attn_work_order(row_ptr: torch.Tensor, B: int, H: int, N: int, block: int, *, stream=None,
+                           order: torch.Tensor | None = None, workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """The queue order of fvattn_sparse_fwd's work items (global CSR row ids)."""
+    lib = load_library()
+    dev = row_ptr.device
+    rows = fvattn_num_rows(B, H, N, block)
+    if order is None:
+        order = torch.empty(rows, dtype=torch.int32, device=dev)
+    if workspace is None:
+        workspace = _empty_bytes(fvattn_fwd_workspace_bytes(B, H, N, block), dev)
+    rc = lib.fvattn_attn_work_order(_ptr(row_ptr), B, H, N, block, _ptr(order), _ptr(workspace), workspace.numel(),
+                                    _stream_ptr(stream))
+    _check(rc, "fvattn_attn_work_order")
+    return order
 
 
 def fvattn_bwd_workspace_bytes(B: int, H: int, N: int, block: int) -> int:

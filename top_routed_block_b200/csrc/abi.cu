@@ -328,6 +328,24 @@ int fvattn_sparse_fwd_profiled(const void *Q, const void *K, const void *V, cons
                            dev_status, stream, 0, order_mode, cta_busy_ns, grid);
 }
 
+int fvattn_attn_work_order(const int32_t *row_ptr, int B, int H, int N, int block, int32_t *order, void *workspace,
+                           size_t ws_bytes, fvattn_stream_t stream) {
+    if (B < 1 || H < 1 || N < 1 || !row_ptr || !order || !workspace) return FVATTN_ERR_INVALID_ARG;
+    if (block != 64 && block != 128) return FVATTN_ERR_UNSUPPORTED;
+    const int64_t BH = static_cast<int64_t>(B) * H;
+    const int64_t nb = ceil_div(N, block);
+    if (BH > kMaxHeads || nb > kMaxCount) return FVATTN_ERR_UNSUPPORTED;
+    if (!aligned16(workspace)) return FVATTN_ERR_ALIGNMENT;
+    if ((reinterpret_cast<uintptr_t>(row_ptr) | reinterpret_cast<uintptr_t>(order)) & 3u) return FVATTN_ERR_ALIGNMENT;
+    if (ws_bytes < fvattn_fwd_workspace_bytes(B, H, N, block)) return FVATTN_ERR_CAPACITY;
+    int rc = check_device();
+    if (rc != FVATTN_OK) return rc;
+    const FwdWorkspace w = fwd_layout(attn_num_items(BH, static_cast<int>(nb)), BH);
+    int32_t *head_rank = reinterpret_cast<int32_t *>(static_cast<char *>(workspace) + w.head_rank);
+    return from_cuda(launch_item_order(row_ptr, BH, static_cast<int>(nb), head_rank, order,
+                                       reinterpret_cast<cudaStream_t>(stream)));
+}
+
 size_t fvattn_bwd_workspace_bytes(int B, int H, int N, int block) {
     if (B < 1 || H < 1 || N < 1 || block != 128) return 0;
     const int64_t nb = ceil_div(N, block);
@@ -512,14 +530,20 @@ __device__ __align__(256) unsigned char g_fwd_scratch[FVATTN_NOALLOC_SCRATCH_BYT
 
 // Device address of g_fwd_scratch on the current device.  In host code the symbol
 // g_fwd_scratch is only a host-side stand-in, so the address is looked up with
-// cudaGetSymbolAddress once per device (with that device current) and cached.
-int static_scratch(void **out) {
+// cudaGetSymbolAddress (with that device current).  The lookup allocates nothing; it
+// is repeated on every call made outside stream capture, so the address follows the
+// module if the device was reset and the library's module reloaded.  During capture
+// the address of the last call outside capture is used (the first call on a device
+// must therefore come before any capture).
+int static_scratch(cudaStream_t stream, void **out) {
     static std::mutex mu;
     static void *addr[64] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FVATTN_ERR_CUDA;
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess) return FVATTN_ERR_CUDA;
     std::lock_guard<std::mutex> g(mu);
-    if (addr[dev] == nullptr) {
+    if (addr[dev] == nullptr || cap == cudaStreamCaptureStatusNone) {
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, g_fwd_scratch) != cudaSuccess || p == nullptr) return FVATTN_ERR_CUDA;
         addr[dev] = p;
@@ -539,7 +563,7 @@ extern "C" int fvattn_sparse_fwd_noalloc(const void *Q, const void *K, const voi
     if (need == 0) return FVATTN_ERR_INVALID_ARG;
     if (need > FVATTN_NOALLOC_SCRATCH_BYTES) return FVATTN_ERR_CAPACITY;
     void *scratch = nullptr;
-    if ((rc = static_scratch(&scratch)) != FVATTN_OK) return rc;
+    if ((rc = static_scratch(reinterpret_cast<cudaStream_t>(stream), &scratch)) != FVATTN_OK) return rc;
     // Same launches as fvattn_sparse_fwd; the work-queue counter in the scratch is
     // cleared there on the stream before the attention kernel starts, and every other
     // scratch word is written before it is read, so stale contents never matter.
