@@ -295,10 +295,11 @@ FVATTN_API int fvattn_sparse_bwd(const void *Q, const void *K, const void *V, co
  * A diagnostic entry point: results equal those of fvattn_sparse_fwd.
  *   order_mode   0: the head-major longest-first work queue fvattn_sparse_fwd uses;
  *                1: rows in index order, the comparison point.
- *   cta_busy_ns  device int64[number of SMs], 8-byte aligned: entry c receives the
- *                global-timer nanoseconds from CTA c's start to the end of its last
- *                work item (entries past *grid are left untouched).
- *   grid         out (host): number of CTAs launched (at most the number of SMs).
+ *   cta_busy_ns  device int64[2 x number of SMs], 8-byte aligned: entry c receives
+ *                the global-timer nanoseconds from CTA c's start to the end of its
+ *                last work item (entries past *grid are left untouched).  The
+ *                persistent grid runs two CTAs per SM.
+ *   grid         out (host): number of CTAs launched (at most 2 x the number of SMs).
  * Other arguments, layouts and errors as fvattn_sparse_fwd; order_mode outside
  * {0,1} or a null cta_busy_ns / grid is FVATTN_ERR_INVALID_ARG.
  */

@@ -252,7 +252,7 @@ def fvattn_sparse_fwd_profiled(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor
     if workspace is None:
         workspace = _empty_bytes(fvattn_fwd_workspace_bytes(B, H, N, block), dev)
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
-    busy = torch.zeros(sms, dtype=torch.int64, device=dev)
+    busy = torch.zeros(2 * sms, dtype=torch.int64, device=dev)   # the persistent grid runs two CTAs per SM
     grid = ctypes.c_int(0)
     rc = lib.fvattn_sparse_fwd_profiled(_ptr(Q), _ptr(K), _ptr(V), _ptr(row_ptr), _ptr(col_idx), B, H, N, d, block,
                                         1 if causal else 0, _ptr(O), _ptr(LSE), _ptr(workspace), workspace.numel(),

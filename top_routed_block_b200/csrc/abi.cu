@@ -267,8 +267,9 @@ static int sparse_fwd_impl(const void *Q, const void *K, const void *V, const in
     int32_t *head_rank = reinterpret_cast<int32_t *>(ws + w.head_rank);
     int *counter = reinterpret_cast<int *>(ws + w.counter);
 
-    CUtensorMap mk, mv;
-    if (!make_map(&mk, K, BH, N, d, block) || !make_map(&mv, V, BH, N, d, block)) return FVATTN_ERR_CUDA;
+    CUtensorMap mq, mk, mv;
+    if (!make_map(&mq, Q, BH, N, d, block) || !make_map(&mk, K, BH, N, d, block) || !make_map(&mv, V, BH, N, d, block))
+        return FVATTN_ERR_CUDA;
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if ((rc = from_cuda(cudaMemsetAsync(dev_status, 0, sizeof(int32_t), s))) != FVATTN_OK) return rc;
@@ -279,9 +280,9 @@ static int sparse_fwd_impl(const void *Q, const void *K, const void *V, const in
     if ((rc = from_cuda(cudaMemsetAsync(counter, 0, sizeof(int), s))) != FVATTN_OK) return rc;
 
     AttnLaunch a{};
+    a.tmap_q = &mq;
     a.tmap_k = &mk;
     a.tmap_v = &mv;
-    a.Q = Q;
     a.row_ptr = row_ptr;
     a.col_idx = col_idx;
     a.order = order;

@@ -9,26 +9,32 @@
 //
 // B200 design:
 //   * One work item = one query block of one head (a CSR row).  A persistent
-//     grid of one CTA per SM pops items from a queue ordered head-major and
+//     grid of two CTAs per SM pops items from a queue ordered head-major and
 //     longest-first (FVAttn §1 "RLB" balances per-head work at run time; here
 //     the SMs are balanced instead, and the head order keeps one or two heads'
 //     K and V in L2 while all SMs work on them).
+//   * Two CTAs per SM, each with its own query block, its own softmax
+//     warpgroup and half of the tensor memory: while one CTA's softmax
+//     warpgroup works on its tile, the tensor cores run the other CTA's
+//     O += P V and next S = Q K^T.  The per-tile critical path of one
+//     softmax warp per sub-partition (the MUFU exponentials, the row maximum,
+//     tensor-memory traffic) is thereby overlapped twice over per SM.
 //   * Warps 0-3 run the softmax and the epilogue (thread = query row = TMEM
-//     lane); warp 4 issues TMA loads of K and V tiles into a ring of shared
-//     memory stages; warp 5 issues the tcgen05 MMAs.
-//   * Tensor memory (512 columns) holds Q twice (the current and the next
-//     item, bf16), S twice and O once (fp32): S = Q K^T of key block j+2 is
-//     computed while the softmax works on block j+1 and the tensor cores run
-//     O += P_j V_j, so the tensor cores never wait for the softmax of the block
-//     they need next.  Q comes from TMEM (TS MMA: only K is read from shared
-//     memory for S), P is written as bf16 into the columns of its S buffer and
-//     read from there by the PV MMA (V from shared memory, MN-major).
-//   * tcgen05 MMAs of one thread execute in issue order: S of block j+2 is
-//     issued after PV of block j, which reads the P in the same columns.
+//     lane); warp 4 issues TMA loads (the item's Q tile, then its K and V
+//     tiles into a ring of shared-memory stages); warp 5 issues the tcgen05
+//     MMAs; warps 6-7 only complete the second warpgroup, which hands
+//     registers to the softmax warpgroup (setmaxnreg).
+//   * Tensor memory (256 columns per CTA): S (fp32, the block's columns) and
+//     O (fp32, d columns).  S = Q K^T is an SS MMA (Q and K from shared
+//     memory); the softmax warps read S with tcgen05.ld, write P as bf16 pairs
+//     into the first columns of S, and O += P V runs as a TS MMA (P from
+//     TMEM, V from shared memory, MN-major).  tcgen05 MMAs of one thread
+//     execute in issue order: S of block j+1 is issued right behind PV of
+//     block j, which reads the P in the same columns, and the completion of S
+//     of block j+1 also tells the softmax warps that O holds PV of block j.
 //   * O stays in TMEM for the whole item; the epilogue divides by l, converts
-//     to bf16 and stores; LSE = (m + log2 l) ln 2.  The softmax warps load the
-//     next item's Q into TMEM before the epilogue, so the next item's first two
-//     S tiles overlap it.
+//     to bf16 and stores; LSE = (m + log2 l) ln 2.  The next item's Q tile is
+//     loaded as soon as this item's last S has read the current one.
 //   * Every mbarrier wait is bounded; a timeout raises the CTA abort flag and
 //     records FVATTN_ERR_DEVICE_TIMEOUT; all roles then drain and exit.
 #include <cuda.h>
@@ -47,35 +53,53 @@ namespace {
 using namespace ptx;
 
 constexpr int kRowsM = 128;           // query rows per tile (tcgen05 M)
-constexpr int kThreads = 192;         // softmax warpgroup + TMA warp + MMA warp
+constexpr int kThreads = 256;         // softmax warpgroup + issue warpgroup
+constexpr int kCtasPerSm = 2;
 constexpr int kTmaWarp = 4;
-constexpr int kMmaWarp = 5;
-constexpr uint32_t kTmemCols = 512;
+constexpr int kMmaWarp = 5;           // warps 6 and 7 only take part in the register hand-over
+// Register hand-over (setmaxnreg): two CTAs of 256 threads share the SM's 65,536
+// registers, 128 per thread at launch; the issue warpgroup drops to kIssueRegs and
+// the softmax warpgroup, which holds a whole S row per thread, rises to
+// kSoftmaxRegs.  The split must not exceed what the launch allocates (checked on
+// the host before the first launch).
+constexpr int kLaunchRegs = 65536 / (kCtasPerSm * kThreads);
+constexpr int kIssueRegs = 48;
+constexpr int kSoftmaxRegs = 208;
+static_assert(128 * kSoftmaxRegs + 128 * kIssueRegs <= kThreads * kLaunchRegs, "register split exceeds the pool");
+static_assert(kSoftmaxRegs % 8 == 0 && kIssueRegs % 8 == 0, "setmaxnreg takes multiples of 8");
+constexpr uint32_t kTmemCols = 256;
 constexpr int kMaxStages = 12;
+// Dynamic shared memory one CTA may take so that two fit on an SM (228 KB per SM,
+// 1 KB of it reserved per CTA).
+constexpr int kSmemPerCta = 113 * 1024;
 
 template <int D, int BS>
 struct Cfg {
     static constexpr int KBLK = D / 64;                   // 128-byte (64 x bf16) column blocks along d
     static constexpr int STAGE_BYTES = KBLK * BS * 128;   // one K or V tile
-    static constexpr int NST = (192 * 1024) / STAGE_BYTES < kMaxStages ? (192 * 1024) / STAGE_BYTES : kMaxStages;
-    static constexpr int TILE_BYTES = NST * STAGE_BYTES;
+    static constexpr int Q_CHUNK = kRowsM * 128;          // one 64-column block of the Q tile (128 rows)
+    static constexpr int Q_BYTES = KBLK * Q_CHUNK;
+    static constexpr int NST_FIT = (kSmemPerCta - Q_BYTES - 1024 - 512) / STAGE_BYTES;
+    static constexpr int NST = NST_FIT < kMaxStages ? NST_FIT : kMaxStages;
+    static_assert(NST >= 2, "the ring needs a K and a V stage");
+    static constexpr int TILE_BYTES = Q_BYTES + NST * STAGE_BYTES;
     static constexpr int SMEM_BYTES = TILE_BYTES + 1024 /*alignment slack*/ + 512 /*barriers*/;
-    // TMEM columns: Q buffers (bf16 pairs), S buffers (fp32; P as bf16 pairs in the
-    // first BS/2 columns), O (fp32)
-    static constexpr uint32_t Q_COLS = D / 2;
-    static constexpr uint32_t T_Q0 = 0, T_Q1 = Q_COLS, T_S0 = 128, T_S1 = 128 + BS, T_O = 128 + 2 * BS;
-    static_assert(T_O + D <= kTmemCols, "TMEM layout exceeds 512 columns");
+    static_assert(SMEM_BYTES <= kSmemPerCta, "two CTAs per SM do not fit");
+    // TMEM columns: S (fp32; P as bf16 pairs in its first BS/2 columns), O (fp32)
+    static constexpr uint32_t T_S = 0, T_O = 128;
+    static_assert(T_O + D <= kTmemCols && BS <= 128, "TMEM layout exceeds the CTA's columns");
     static constexpr uint32_t IDESC_S = idesc_bf16_f32(kRowsM, BS, 0, 0);
     static constexpr uint32_t IDESC_PV = idesc_bf16_f32(kRowsM, D, 0, 1);
 };
 
 struct Barriers {
     uint64_t ring_full[kMaxStages], ring_empty[kMaxStages];
-    uint64_t q_full[2], s_full[2], p_full[2];
-    uint64_t pv_done, o_full, o_empty;
+    uint64_t q_full, q_empty, s_full, p_full;
+    uint64_t o_full, o_empty;
     uint64_t sched_full[2], sched_empty[2];
     uint64_t drain;
     int4 sched_item[2];  // {row, col start, count, valid item}
+    long long t_start;   // diagnostic: global timer at the start of the CTA's work
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -102,9 +126,9 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 }
 
 template <int D, int BS>
-__global__ void __launch_bounds__(kThreads, 1)
-    sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
-                           const __nv_bfloat16 *__restrict__ Qg, const int32_t *__restrict__ row_ptr,
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+    sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
+                           const __grid_constant__ CUtensorMap tmap_v, const int32_t *__restrict__ row_ptr,
                            const int32_t *__restrict__ col_idx, const int32_t *__restrict__ order, int n_items,
                            int *__restrict__ work_counter, int N, int nb, int causal, float scale_log2,
                            __nv_bfloat16 *__restrict__ O, float *__restrict__ LSE, int32_t *dev_status,
@@ -114,8 +138,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     // 1024-byte alignment for the 128-byte-swizzled tiles
     const uint32_t base_addr = smem_addr(smem_raw);
-    unsigned char *ring = smem_raw + ((1024 - (base_addr & 1023)) & 1023);  // stage s at s * STAGE_BYTES
-    Barriers *bar = reinterpret_cast<Barriers *>(ring + C::TILE_BYTES);
+    unsigned char *qtile = smem_raw + ((1024 - (base_addr & 1023)) & 1023);  // Q tile, then the ring
+    unsigned char *ring = qtile + C::Q_BYTES;                                 // stage s at s * STAGE_BYTES
+    Barriers *bar = reinterpret_cast<Barriers *>(qtile + C::TILE_BYTES);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -126,19 +151,27 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&bar->ring_full[s], 1);
             mbar_init(&bar->ring_empty[s], 1);
         }
+        mbar_init(&bar->q_full, 1);
+        mbar_init(&bar->q_empty, 1);
+        mbar_init(&bar->s_full, 1);
+        mbar_init(&bar->p_full, 4);
+        mbar_init(&bar->o_full, 1);
+        mbar_init(&bar->o_empty, 4);
         for (int x = 0; x < 2; ++x) {
-            mbar_init(&bar->q_full[x], 4);
-            mbar_init(&bar->s_full[x], 1);
-            mbar_init(&bar->p_full[x], 4);
             mbar_init(&bar->sched_full[x], 1);
             mbar_init(&bar->sched_empty[x], 1 + 4);
         }
-        mbar_init(&bar->pv_done, 1);
-        mbar_init(&bar->o_full, 1);
-        mbar_init(&bar->o_empty, 4);
         mbar_init(&bar->drain, 1);
         bar->abort_flag = 0;
         fence_barrier_init();
+    }
+    if (BS < kRowsM) {
+        // Q rows BS..127 of every column block stay zero (TMA fills only the block's rows)
+        for (int i = threadIdx.x; i < C::Q_BYTES / 16; i += kThreads) {
+            if ((i * 16) % C::Q_CHUNK >= BS * 128)
+                reinterpret_cast<uint4 *>(qtile)[i] = make_uint4(0, 0, 0, 0);
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
     if (warp == kMmaWarp) {
         tmem_alloc(&bar->tmem_base, kTmemCols);
@@ -148,15 +181,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = bar->tmem_base;
-    long long t_start = 0;  // global timer (ns) when this CTA starts its items, if busy times are asked for
-    if (cta_busy_ns && threadIdx.x == 0) asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_start));
+    // global timer (ns) when this CTA starts its items, if busy times are asked for (kept in
+    // shared memory: nothing of the prologue stays live in registers across the hand-over)
+    if (cta_busy_ns && threadIdx.x == 0) {
+        long long t0;
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+        bar->t_start = t0;
+    }
 
+    if (warp >= kTmaWarp) {
+    // The register hand-over and the code that uses the new count sit in the same
+    // branch, so the compiler allocates each role's registers against its own limit.
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kIssueRegs));
     if (warp == kTmaWarp) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
+            prefetch_tensormap(&tmap_q);
             prefetch_tensormap(&tmap_k);
             prefetch_tensormap(&tmap_v);
-            uint32_t it = 0, rc = 0;  // items published, ring loads issued
+            uint32_t it = 0, rc = 0, qn = 0;  // items published, ring loads issued, Q loads issued
             bool ok = true;
             while (ok) {
                 const int idx = atomicAdd(work_counter, 1);
@@ -176,9 +219,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mbar_arrive(&bar->sched_full[k]);
                 ++it;
                 if (rw < 0) break;
-                const int bh = rw / nb;
+                if (item.z == 0) continue;
+                const int bh = rw / nb, qb = rw % nb;
+                // the item's Q tile, once the previous item's last S has read the buffer
+                if (!mbar_wait(&bar->q_empty, (qn & 1) ^ 1, abort_flag, dev_status)) break;
+                // Test hook: CTA 0 never loads its first Q tile, so the MMA warp's bounded
+                // wait for it runs out (exercises the timeout path).
+                if (!(test_stall && blockIdx.x == 0 && qn == 0)) {
+                    mbar_arrive_expect_tx(&bar->q_full, C::KBLK * BS * 128);
+                    for (int kb = 0; kb < C::KBLK; ++kb)
+                        tma_load_3d(qtile + kb * C::Q_CHUNK, &tmap_q, &bar->q_full, kb * 64, qb * BS, bh);
+                }
+                ++qn;
                 int prev = -1;
-                int kblk_next = item.z > 0 ? __ldg(col_idx + item.y) : 0;  // loaded one tile ahead
+                int kblk_next = __ldg(col_idx + item.y);  // loaded one tile ahead
                 for (int j = 0; j < item.z && ok; ++j) {
                     int kblk = kblk_next;
                     if (j + 1 < item.z) kblk_next = __ldg(col_idx + item.y + j + 1);
@@ -209,34 +263,43 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mbar_wait_teardown(&bar->ring_full[st], (times - 1) & 1);
                 }
             }
+            if (qn > 0 && !(test_stall && blockIdx.x == 0 && qn == 1)) mbar_wait_teardown(&bar->q_full, (qn - 1) & 1);
         }
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             const uint32_t r0 = smem_addr(ring);
-            uint32_t it = 0, rc = 0, tc = 0, qn = 0, on = 0;  // items, ring loads, tiles, Q loads, outputs
+            const uint32_t q0 = smem_addr(qtile);
+            uint32_t it = 0, rc = 0, tc = 0, qn = 0, on = 0;  // items, ring loads, tiles, Q tiles, outputs
             bool ok = true;
             auto wait = [&](uint64_t *b, uint32_t parity) {
                 if (ok && !mbar_wait(b, parity, abort_flag, dev_status)) ok = false;
                 return ok;
             };
-            // S[scol] = Q[qcol] K^T, K from ring stage st (A from TMEM, B K-major in shared memory)
-            auto issue_s = [&](uint32_t qcol, uint32_t scol, uint32_t st) {
-                const uint32_t kbase = r0 + st * C::STAGE_BYTES;
+            // S = Q K^T, Q from the Q tile, K from ring stage st (both K-major in shared memory)
+            // (descriptors of each k-step: one base descriptor plus the step's byte offset >> 4;
+            // shared-memory addresses stay below 2^18, so the 14-bit address field never carries)
+            // (kept as loops: the issue warpgroup runs on few registers)
+            const uint64_t qdesc = smem_desc_sw128(q0, 16, 1024);
+            auto issue_s = [&](uint32_t st) {
+                const uint64_t kdesc = smem_desc_sw128(r0 + st * C::STAGE_BYTES, 16, 1024);
+#pragma unroll 1
+                for (int kb = 0; kb < C::KBLK; ++kb) {
 #pragma unroll
-                for (int k = 0; k < D / 16; ++k) {
-                    const uint32_t kb = k >> 2, ko = (k & 3) * 32;
-                    const uint64_t db = smem_desc_sw128(kbase + kb * BS * 128 + ko, 16, 1024);
-                    mma_ts(tmem + scol, tmem + qcol + k * 8, db, C::IDESC_S, k > 0 ? 1u : 0u);
+                    for (int k = 0; k < 4; ++k)
+                        mma_ss_nc(tmem + C::T_S, qdesc + ((kb * C::Q_CHUNK + k * 32) >> 4),
+                                  kdesc + ((kb * BS * 128 + k * 32) >> 4), C::IDESC_S, (kb | k) ? 1u : 0u);
                 }
             };
-            // O (+)= P V, P from the S buffer at scol, V from ring stage st (MN-major)
-            auto issue_pv = [&](uint32_t scol, uint32_t st, bool first) {
-                const uint32_t vbase = r0 + st * C::STAGE_BYTES;
+            // O (+)= P V, P from the S columns, V from ring stage st (MN-major)
+            auto issue_pv = [&](uint32_t st, bool first) {
+                const uint64_t vdesc = smem_desc_sw128(r0 + st * C::STAGE_BYTES, BS * 128, 1024);
+#pragma unroll 1
+                for (int k0 = 0; k0 < BS / 16; k0 += 4) {
 #pragma unroll
-                for (int k = 0; k < BS / 16; ++k) {
-                    const uint64_t dv = smem_desc_sw128(vbase + k * 16 * 128, BS * 128, 1024);
-                    mma_ts(tmem + C::T_O, tmem + scol + k * 8, dv, C::IDESC_PV, (!first || k > 0) ? 1u : 0u);
+                    for (int k = k0; k < k0 + 4; ++k)
+                        mma_ts_nc(tmem + C::T_O, tmem + C::T_S + k * 8, vdesc + ((k * 16 * 128) >> 4), C::IDESC_PV,
+                                  (!first || k > 0) ? 1u : 0u);
                 }
             };
             while (ok) {
@@ -253,34 +316,31 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ++on;
                     continue;
                 }
-                if (!wait(&bar->q_full[qn & 1], (qn >> 1) & 1)) break;
+                if (!wait(&bar->q_full, qn & 1)) break;
+                // S of the first key block
+                if (!wait(&bar->ring_full[rc % NST], (rc / NST) & 1)) break;
                 tc_fence_after();
-                const uint32_t qcol = (qn & 1) ? C::T_Q1 : C::T_Q0;
-                // S of the first two key blocks, into both S buffers
-                for (int j = 0; j < 2 && j < count; ++j) {
-                    const uint32_t ki = rc + 2 * j;
-                    if (!wait(&bar->ring_full[ki % NST], (ki / NST) & 1)) break;
-                    const uint32_t sb = (tc + j) & 1;
-                    issue_s(qcol, sb ? C::T_S1 : C::T_S0, ki % NST);
-                    mma_commit(&bar->s_full[sb]);
-                    mma_commit(&bar->ring_empty[ki % NST]);
-                }
+                issue_s(rc % NST);
+                mma_commit(&bar->s_full);
+                mma_commit(&bar->ring_empty[rc % NST]);
+                if (count == 1) mma_commit(&bar->q_empty);
                 for (int j = 0; j < count && ok; ++j) {
-                    const uint32_t t = tc + j, sb = t & 1, scol = sb ? C::T_S1 : C::T_S0;
-                    if (!wait(&bar->p_full[sb], (t >> 1) & 1)) break;
+                    const uint32_t t = tc + j;
+                    if (!wait(&bar->p_full, t & 1)) break;
                     if (j == 0 && !wait(&bar->o_empty, (on & 1) ^ 1)) break;
                     const uint32_t vi = rc + 2 * j + 1;
                     if (!wait(&bar->ring_full[vi % NST], (vi / NST) & 1)) break;
                     tc_fence_after();
-                    issue_pv(scol, vi % NST, j == 0);
+                    issue_pv(vi % NST, j == 0);
                     mma_commit(&bar->ring_empty[vi % NST]);
-                    mma_commit(&bar->pv_done);
-                    if (j + 2 < count) {  // the S buffer just read by PV takes block j+2
-                        const uint32_t ki = rc + 2 * (j + 2);
+                    if (j + 1 < count) {  // S of the next block, behind the PV that reads P in its columns
+                        const uint32_t ki = rc + 2 * (j + 1);
                         if (!wait(&bar->ring_full[ki % NST], (ki / NST) & 1)) break;
-                        issue_s(qcol, scol, ki % NST);
-                        mma_commit(&bar->s_full[sb]);
+                        tc_fence_after();
+                        issue_s(ki % NST);
+                        mma_commit(&bar->s_full);
                         mma_commit(&bar->ring_empty[ki % NST]);
+                        if (j + 2 == count) mma_commit(&bar->q_empty);  // the item's last S has read Q
                     }
                 }
                 if (!ok) break;
@@ -294,12 +354,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_commit(&bar->drain);
             mbar_wait_teardown(&bar->drain, 0);
         }
+    }
     } else {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
         // ------------------------------------------------ softmax / epilogue (warps 0-3)
         const int r = threadIdx.x;                                  // tile row = TMEM lane
         const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-        uint32_t it = 0, tc = 0, qn = 0, on = 0;  // items read, tiles, Q loads, outputs
-        bool ok = true;
+        const uint32_t tS = tmem + lane_base + C::T_S;
+        const uint32_t tO = tmem + lane_base + C::T_O;
+        uint32_t it = 0, tc = 0, on = 0;  // items read, tiles, outputs
         auto next_item = [&](int4 &out) {
             const uint32_t k = it & 1;
             if (!mbar_wait(&bar->sched_full[k], (it >> 1) & 1, abort_flag, dev_status)) return false;
@@ -309,171 +372,129 @@ __global__ void __launch_bounds__(kThreads, 1)
             ++it;
             return true;
         };
-        // This thread's query row of `itm` (zeros past the block or past N) into the
-        // Q buffer of Q load number qn, as bf16 pairs: column c holds (q[2c], q[2c+1]).
-        auto load_q = [&](const int4 &itm) {
-            const int64_t bhq = itm.x / nb;
-            const int tq = (itm.x % nb) * BS + r;
-            const bool in = r < BS && tq < N;
-            const uint4 *src = reinterpret_cast<const uint4 *>(Qg + (bhq * N + (in ? tq : 0)) * D);
-            const uint32_t tQ = tmem + lane_base + ((qn & 1) ? C::T_Q1 : C::T_Q0);
-#pragma unroll
-            for (int c0 = 0; c0 < D / 2; c0 += 32) {
-                uint32_t q[32];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const uint4 x = in ? __ldg(src + c0 / 4 + i) : make_uint4(0, 0, 0, 0);
-                    q[4 * i] = x.x;
-                    q[4 * i + 1] = x.y;
-                    q[4 * i + 2] = x.z;
-                    q[4 * i + 3] = x.w;
-                }
-                tmem_st32(tQ + c0, q);
-            }
-            tmem_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            // Test hook: CTA 0 never reports its first Q as loaded, so the MMA warp's
-            // bounded wait for it runs out (exercises the timeout path).
-            if (lane == 0 && !(test_stall && blockIdx.x == 0 && qn == 0)) mbar_arrive(&bar->q_full[qn & 1]);
-        };
         int4 item;
-        if (next_item(item)) {
-            if (item.w && item.z > 0) load_q(item);
-            while (item.w) {
-                const int row = item.x, start = item.y, count = item.z;
-                const int64_t bh = row / nb;
-                const int qb = row % nb;
-                const int t_row = qb * BS + r;  // token index of this thread's row
-                float m = -CUDART_INF_F, l = 0.0f;
-                int prev = -1;
-                int kblk_next = count > 0 ? __ldg(col_idx + start) : 0;  // loaded one tile ahead
-                for (int j = 0; j < count; ++j) {
-                    const int kblk = kblk_next;
-                    if (j + 1 < count) kblk_next = __ldg(col_idx + start + j + 1);
-                    const bool valid = kblk >= 0 && kblk < nb && kblk > prev;
-                    if (valid) prev = kblk;
-                    const int key0 = kblk * BS;
-                    // keys of this block that exist and are allowed for this row
-                    int lim = valid ? min(BS, N - key0) : 0;
-                    if (causal) lim = min(lim, t_row - key0 + 1);
-                    const uint32_t sb = tc & 1;
-                    if (!mbar_wait(&bar->s_full[sb], (tc >> 1) & 1, abort_flag, dev_status)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint32_t tS = tmem + lane_base + (sb ? C::T_S1 : C::T_S0);
-                    // the whole S row of this thread: BS fp32 values
-                    uint32_t v[BS];
-#pragma unroll
-                    for (int c0 = 0; c0 < BS; c0 += 32)
-                        tmem_ld32(tS + c0, *reinterpret_cast<uint32_t(*)[32]>(&v[c0]));
-                    tmem_wait_ld();
-                    if (lim < BS) {  // ragged last block, causal diagonal, or a skipped index
-#pragma unroll
-                        for (int c = 0; c < BS; ++c)
-                            if (c >= lim) v[c] = __float_as_uint(-CUDART_INF_F);
-                    }
-                    float mq[4] = {-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F};
-#pragma unroll
-                    for (int c = 0; c < BS; c += 8) {
-#pragma unroll
-                        for (int q = 0; q < 4; ++q)
-                            mq[q] = max3f(mq[q], __uint_as_float(v[c + 2 * q]), __uint_as_float(v[c + 2 * q + 1]));
-                    }
-                    const float mxs = max3f(mq[0], mq[1], fmaxf(mq[2], mq[3])) * scale_log2;
-                    // The reference maximum only moves when the row maximum exceeds it by
-                    // more than 2^8: P stays below 256 and the rescale of O is rare.  O and
-                    // l always share the same reference, so the final O / l is exact.
-                    const bool need = mxs > m + kRescaleLog2;
-                    const float m_new = need ? mxs : m;
-                    const float alpha = need ? ex2_approx(m - m_new) : 1.0f;
-                    const float neg_m = (m_new == -CUDART_INF_F) ? 0.0f : -m_new;
-                    float rs[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-                    // P packed as bf16 pairs in place, v[c/2] <- (p[c], p[c+1]); one loop for
-                    // full and masked tiles (masked scores are -inf, and 2^-inf = 0)
-#pragma unroll
-                    for (int c = 0; c < BS; c += 2) {
-                        const float p0 = ex2_approx(fmaf(__uint_as_float(v[c]), scale_log2, neg_m));
-                        const float p1 = ex2_approx(fmaf(__uint_as_float(v[c + 1]), scale_log2, neg_m));
-                        rs[(c >> 1) & 3] += p0 + p1;
-                        v[c >> 1] = pack_bf16(p0, p1);
-                    }
-#pragma unroll
-                    for (int c0 = 0; c0 < BS / 2; c0 += 32)
-                        tmem_st32(tS + c0, *reinterpret_cast<const uint32_t(*)[32]>(&v[c0]));
-                    l = l * alpha + ((rs[0] + rs[1]) + (rs[2] + rs[3]));
-                    // Rescale the running output.  The PV of the previous block may still be
-                    // accumulating into O: wait for it first (its completion is phase tc-1
-                    // of pv_done; the PV of this block cannot start before P is published).
-                    if (__any_sync(0xffffffffu, need && j > 0)) {
-                        if (!mbar_wait(&bar->pv_done, (tc - 1) & 1, abort_flag, dev_status)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-                        const uint32_t tO = tmem + lane_base + C::T_O;
-#pragma unroll
-                        for (int c0 = 0; c0 < D; c0 += 32) {
-                            uint32_t o[32];
-                            tmem_ld32(tO + c0, o);
-                            tmem_wait_ld();
-#pragma unroll
-                            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-                            tmem_st32(tO + c0, o);
-                        }
-                    }
-                    tmem_wait_st();
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&bar->p_full[sb]);
-                    m = m_new;
-                    ++tc;
+        bool ok = next_item(item);
+        while (ok && item.w) {
+            const int row = item.x, start = item.y, count = item.z;
+            const int64_t bh = row / nb;
+            const int qb = row % nb;
+            const int t_row = qb * BS + r;  // token index of this thread's row
+            float m = -CUDART_INF_F, l = 0.0f;
+            int prev = -1;
+            int kblk_next = count > 0 ? __ldg(col_idx + start) : 0;  // loaded one tile ahead
+            for (int j = 0; j < count; ++j) {
+                const int kblk = kblk_next;
+                if (j + 1 < count) kblk_next = __ldg(col_idx + start + j + 1);
+                const bool valid = kblk >= 0 && kblk < nb && kblk > prev;
+                if (valid) prev = kblk;
+                const int key0 = kblk * BS;
+                // keys of this block that exist and are allowed for this row
+                int lim = valid ? min(BS, N - key0) : 0;
+                if (causal) lim = min(lim, t_row - key0 + 1);
+                if (!mbar_wait(&bar->s_full, tc & 1, abort_flag, dev_status)) {
+                    ok = false;
+                    break;
                 }
-                if (!ok) break;
-                if (count > 0) ++qn;
-                // the next item's Q goes into TMEM before this item's epilogue, so its first
-                // S tiles overlap the epilogue
-                int4 nxt;
-                if (!next_item(nxt)) break;
-                if (nxt.w && nxt.z > 0) load_q(nxt);
-                // epilogue
-                if (!mbar_wait(&bar->o_full, on & 1, abort_flag, dev_status)) break;
-                ++on;
                 tc_fence_after();
-                const bool row_ok = r < BS && t_row < N;
-                const float inv_l = (l > 0.0f) ? 1.0f / l : 0.0f;
-                __nv_bfloat16 *orow = O + (bh * N + t_row) * D;
-                const uint32_t tO = tmem + lane_base + C::T_O;
+                // the whole S row of this thread: BS fp32 values
+                uint32_t v[BS];
 #pragma unroll
-                for (int c0 = 0; c0 < D; c0 += 32) {
-                    uint32_t o[32];
-                    if (count > 0) {
+                for (int c0 = 0; c0 < BS; c0 += 32)
+                    tmem_ld32(tS + c0, *reinterpret_cast<uint32_t(*)[32]>(&v[c0]));
+                tmem_wait_ld();
+                if (lim < BS) {  // ragged last block, causal diagonal, or a skipped index
+#pragma unroll
+                    for (int c = 0; c < BS; ++c)
+                        if (c >= lim) v[c] = __float_as_uint(-CUDART_INF_F);
+                }
+                float mq[4] = {-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F};
+#pragma unroll
+                for (int c = 0; c < BS; c += 8) {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        mq[q] = max3f(mq[q], __uint_as_float(v[c + 2 * q]), __uint_as_float(v[c + 2 * q + 1]));
+                }
+                const float mxs = max3f(mq[0], mq[1], fmaxf(mq[2], mq[3])) * scale_log2;
+                // The reference maximum only moves when the row maximum exceeds it by
+                // more than 2^8: P stays below 256 and the rescale of O is rare.  O and
+                // l always share the same reference, so the final O / l is exact.
+                const bool need = mxs > m + kRescaleLog2;
+                const float m_new = need ? mxs : m;
+                const float alpha = need ? ex2_approx(m - m_new) : 1.0f;
+                const float neg_m = (m_new == -CUDART_INF_F) ? 0.0f : -m_new;
+                float rs[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+                // P packed as bf16 pairs in place, v[c/2] <- (p[c], p[c+1]); one loop for
+                // full and masked tiles (masked scores are -inf, and 2^-inf = 0)
+#pragma unroll
+                for (int c = 0; c < BS; c += 2) {
+                    const float p0 = ex2_approx(fmaf(__uint_as_float(v[c]), scale_log2, neg_m));
+                    const float p1 = ex2_approx(fmaf(__uint_as_float(v[c + 1]), scale_log2, neg_m));
+                    rs[(c >> 1) & 3] += p0 + p1;
+                    v[c >> 1] = pack_bf16(p0, p1);
+                }
+#pragma unroll
+                for (int c0 = 0; c0 < BS / 2; c0 += 32)
+                    tmem_st32(tS + c0, *reinterpret_cast<const uint32_t(*)[32]>(&v[c0]));
+                l = l * alpha + ((rs[0] + rs[1]) + (rs[2] + rs[3]));
+                // Rescale the running output.  S of this block completed after PV of the
+                // previous one (one issuing thread, in order), so O is complete here.
+                if (__any_sync(0xffffffffu, need && j > 0)) {
+#pragma unroll
+                    for (int c0 = 0; c0 < D; c0 += 32) {
+                        uint32_t o[32];
                         tmem_ld32(tO + c0, o);
                         tmem_wait_ld();
-                    } else {
 #pragma unroll
-                        for (int c = 0; c < 32; ++c) o[c] = 0u;
-                    }
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int c = 0; c < 32; c += 2)
-                        pk[c >> 1] = pack_bf16(__uint_as_float(o[c]) * inv_l, __uint_as_float(o[c + 1]) * inv_l);
-                    if (row_ok) {
-                        uint4 *dst = reinterpret_cast<uint4 *>(orow + c0);
-#pragma unroll
-                        for (int q = 0; q < 4; ++q)
-                            dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+                        for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+                        tmem_st32(tO + c0, o);
                     }
                 }
-                if (row_ok)
-                    LSE[bh * N + t_row] = (l > 0.0f) ? (m + __log2f(l)) * 0.69314718055994531f : -CUDART_INF_F;
+                tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&bar->o_empty);
-                item = nxt;
+                if (lane == 0) mbar_arrive(&bar->p_full);
+                m = m_new;
+                ++tc;
             }
+            if (!ok) break;
+            // the next item from the queue, so that its Q tile and first K/V tiles load
+            // while this one finishes
+            int4 nxt;
+            if (!next_item(nxt)) break;
+            // epilogue
+            if (!mbar_wait(&bar->o_full, on & 1, abort_flag, dev_status)) break;
+            ++on;
+            tc_fence_after();
+            const bool row_ok = r < BS && t_row < N;
+            const float inv_l = (l > 0.0f) ? 1.0f / l : 0.0f;
+            __nv_bfloat16 *orow = O + (bh * N + t_row) * D;
+#pragma unroll
+            for (int c0 = 0; c0 < D; c0 += 32) {
+                uint32_t o[32];
+                if (count > 0) {
+                    tmem_ld32(tO + c0, o);
+                    tmem_wait_ld();
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) o[c] = 0u;
+                }
+                uint32_t pk[16];
+#pragma unroll
+                for (int c = 0; c < 32; c += 2)
+                    pk[c >> 1] = pack_bf16(__uint_as_float(o[c]) * inv_l, __uint_as_float(o[c + 1]) * inv_l);
+                if (row_ok) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(orow + c0);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+                }
+            }
+            if (row_ok)
+                LSE[bh * N + t_row] = (l > 0.0f) ? (m + __log2f(l)) * 0.69314718055994531f : -CUDART_INF_F;
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar->o_empty);
+            item = nxt;
         }
     }
     tc_fence_before();
@@ -482,7 +503,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (cta_busy_ns && threadIdx.x == 0) {
         long long t_end;
         asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_end));
-        cta_busy_ns[blockIdx.x] = t_end - t_start;
+        cta_busy_ns[blockIdx.x] = t_end - bar->t_start;
     }
     if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
 }
@@ -575,7 +596,7 @@ int attn_smem_bytes(int d, int bs) {
     return Cfg<64, 64>::SMEM_BYTES;
 }
 
-int attn_ctas_per_sm() { return 1; }
+int attn_ctas_per_sm() { return kCtasPerSm; }
 
 int64_t attn_num_items(int64_t BH, int nb) { return BH * nb; }
 
@@ -605,12 +626,28 @@ cudaError_t launch_natural_order(int64_t n, int32_t *order, cudaStream_t stream)
 template <int D, int BS>
 static cudaError_t launch_t(const AttnLaunch &a, cudaStream_t stream) {
     auto kern = sparse_attn_fwd_kernel<D, BS>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<D, BS>::SMEM_BYTES);
-    if (e != cudaSuccess) return e;
+    // Checked once per instantiation: the register hand-over waits until the pool
+    // holds the requested registers, so it must fit in what the launch allocates,
+    // and two CTAs must be resident per SM (the grid is sized for that).
+    static int state = 0;  // 0 unknown, 1 ok, -1 not launchable as designed
+    if (state == 0) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<D, BS>::SMEM_BYTES);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+        if (e != cudaSuccess) return e;
+        cudaFuncAttributes fa{};
+        if ((e = cudaFuncGetAttributes(&fa, kern)) != cudaSuccess) return e;
+        int per_sm = 0;
+        if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, Cfg<D, BS>::SMEM_BYTES)) !=
+            cudaSuccess)
+            return e;
+        state = (128 * kSoftmaxRegs + 128 * kIssueRegs <= fa.numRegs * kThreads && per_sm >= kCtasPerSm) ? 1 : -1;
+    }
+    if (state < 0) return cudaErrorInvalidConfiguration;
     kern<<<a.grid, kThreads, Cfg<D, BS>::SMEM_BYTES, stream>>>(
-        *a.tmap_k, *a.tmap_v, static_cast<const __nv_bfloat16 *>(a.Q), a.row_ptr, a.col_idx, a.order, a.n_items,
-        a.work_counter, a.N, a.nb, a.causal, a.scale_log2, static_cast<__nv_bfloat16 *>(a.O), a.LSE, a.dev_status,
-        a.test_stall, a.cta_busy_ns);
+        *a.tmap_q, *a.tmap_k, *a.tmap_v, a.row_ptr, a.col_idx, a.order, a.n_items, a.work_counter, a.N, a.nb,
+        a.causal, a.scale_log2, static_cast<__nv_bfloat16 *>(a.O), a.LSE, a.dev_status, a.test_stall,
+        a.cta_busy_ns);
     return cudaGetLastError();
 }
 

@@ -8,8 +8,7 @@
 namespace fvattn {
 
 struct AttnLaunch {
-    const CUtensorMap *tmap_k, *tmap_v;  // host copies, passed by value as kernel parameters
-    const void *Q;                       // bf16 [B,H,N,d], read row by row into tensor memory
+    const CUtensorMap *tmap_q, *tmap_k, *tmap_v;  // host copies, passed by value as kernel parameters
     const int32_t *row_ptr, *col_idx, *order;  // order: work items (CSR rows), head-major, longest first
     int n_items;
     int *work_counter;  // zeroed before the launch
