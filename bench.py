@@ -506,6 +506,54 @@ def run_ours(args, w, rank, world, local):
                        "outside the timed region"}
         del gQ, gK, gV, ws_b, dO
 
+    # FP8 variant (outside the timed step): e4m3 block quantization of Q, K and V, then
+    # the e4m3 forward on the same mask
+    fp8 = None
+    if w.d == 128 and not args.no_fp8:
+        q8 = [fv.fvattn_quant_e4m3(x, w.bs, stream=stream) for x in (dQ, dK, dV)]
+        O8 = torch.empty_like(dQ)
+        L8 = torch.empty_like(plan.LSE)
+        st8 = torch.zeros(1, dtype=torch.int32, device=dev)
+
+        def quant_call():
+            for x, (c, e) in zip((dQ, dK, dV), q8):
+                fv.fvattn_quant_e4m3(x, w.bs, stream=stream, out=c, scale_exp=e)
+
+        def fp8_call():
+            fv.fvattn_sparse_fwd_fp8(q8[0][0], q8[1][0], q8[2][0], q8[0][1], q8[1][1], q8[2][1], *mask_csr(), w.bs,
+                                     w.causal, stream=stream, O=O8, LSE=L8, workspace=plan.fwd_ws, dev_status=st8)
+        fwd()
+        for _ in range(3):
+            quant_call()
+            fp8_call()
+        torch.cuda.synchronize(dev)
+        fv.check_status(st8, "fvattn_sparse_fwd_fp8")
+        reps = max(5, min(args.steps, 20))
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(reps)]
+        for e0, e1, e2 in evs:
+            e0.record(stream)
+            quant_call()
+            e1.record(stream)
+            fp8_call()
+            e2.record(stream)
+        torch.cuda.synchronize(dev)
+        fv.check_status(st8, "fvattn_sparse_fwd_fp8")
+        q_ms = statistics.mean(a.elapsed_time(b) for a, b, _ in evs)
+        a8_ms = statistics.mean(b.elapsed_time(c) for _, b, c in evs)
+        diff = (O8.float() - plan.O.float()).abs()
+        fp8_peak = 2.0 * float(load_peaks()[0]["bf16_tflops"])
+        fp8 = {"attn_ms": a8_ms, "attn_tflops": flops / (a8_ms * 1e-3) / 1e12,
+               "frac_of_fp8_peak": flops / (a8_ms * 1e-3) / 1e12 / fp8_peak, "fp8_peak": fp8_peak,
+               "speedup_vs_bf16_attn": attn_ms / a8_ms, "quant_ms": q_ms,
+               "o_vs_bf16_path": {"max_abs": diff.max().item(), "mean_abs": diff.mean().item()},
+               "note": "attention on e4m3 Q, K, V with power-of-two block scales (fvattn_sparse_fwd_fp8) on the "
+                       "routing mask of the bf16 step; quant = three fvattn_quant_e4m3 calls; fp8_peak = measured "
+                       "bf16 burst peak x 2 (the nominal e4m3/bf16 tensor ratio); o_vs_bf16_path compares with "
+                       "the bf16 forward's O (the e4m3 rounding of the inputs included); mean of the timed "
+                       "calls, outside the timed step"}
+        del q8, O8, L8
+        torch.cuda.empty_cache()
+
     peaks, peak_src = load_peaks()
     configs = None
     if world == 1 and not args.no_configs:
@@ -572,6 +620,7 @@ def run_ours(args, w, rank, world, local):
         "clocks": clocks,
         "cpu_baseline": cpu,
         "configs": configs,
+        "fp8": fp8,
     }
     print(json.dumps(line), flush=True)
 
@@ -586,6 +635,7 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-configs", action="store_true", help="skip the other workloads' timings")
+    ap.add_argument("--no-fp8", action="store_true", help="skip the e4m3 forward's timing")
     ap.add_argument("--config-steps", type=int, default=10)
     args = ap.parse_args()
     w = W.ALL[args.workload]

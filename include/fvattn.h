@@ -75,6 +75,14 @@ typedef enum {
 /* Human-readable name of a status code (static string, never NULL). */
 FVATTN_API const char *fvattn_status_string(int status);
 
+/*
+ * The reason for the calling host thread's most recent FVATTN_ERR_CUDA: the CUDA
+ * error name of the failing call, or a description of the launch check that
+ * refused it.  A static string ("" if there was none); not cleared by successful
+ * calls.
+ */
+FVATTN_API const char *fvattn_last_error(void);
+
 /* Number of rows B*H*ceil(N/block) (0 on bad arguments). */
 FVATTN_API int64_t fvattn_num_rows(int B, int H, int N, int block);
 
@@ -295,11 +303,11 @@ FVATTN_API int fvattn_sparse_bwd(const void *Q, const void *K, const void *V, co
  * A diagnostic entry point: results equal those of fvattn_sparse_fwd.
  *   order_mode   0: the head-major longest-first work queue fvattn_sparse_fwd uses;
  *                1: rows in index order, the comparison point.
- *   cta_busy_ns  device int64[2 x number of SMs], 8-byte aligned: entry c receives
- *                the global-timer nanoseconds from CTA c's start to the end of its
- *                last work item (entries past *grid are left untouched).  The
- *                persistent grid runs two CTAs per SM.
- *   grid         out (host): number of CTAs launched (at most 2 x the number of SMs).
+ *   cta_busy_ns  device int64[number of SMs], 8-byte aligned: entry c receives the
+ *                global-timer nanoseconds from CTA c's start to the end of its last
+ *                work item (entries past *grid are left untouched).  The persistent
+ *                grid runs one CTA per SM, each with two work items in flight.
+ *   grid         out (host): number of CTAs launched (at most the number of SMs).
  * Other arguments, layouts and errors as fvattn_sparse_fwd; order_mode outside
  * {0,1} or a null cta_busy_ns / grid is FVATTN_ERR_INVALID_ARG.
  */
@@ -307,6 +315,29 @@ FVATTN_API int fvattn_sparse_fwd_profiled(const void *Q, const void *K, const vo
                                           const int32_t *col_idx, int B, int H, int N, int d, int block, int causal,
                                           void *O, float *LSE, void *workspace, size_t ws_bytes, int32_t *dev_status,
                                           int order_mode, int64_t *cta_busy_ns, int *grid, fvattn_stream_t stream);
+
+/*
+ * fvattn_sparse_fwd_fp8 -- the block-sparse attention forward of fvattn_sparse_fwd
+ * on FP8 operands ("Accelerating HunyuanVideo inference with ParaAttention"
+ * (WaveSpeed), § "FP8 dynamic quantization": attention computed on activations
+ * quantized to FP8 at run time).  Q, K, V are given as fvattn_quant_e4m3 returns
+ * them: e4m3 codes (OCP E4M3FN) with one power-of-two scale per (head, block), the
+ * value of a code being its e4m3 value times 2^exponent.  Both GEMMs run on the
+ * tensor cores as e4m3 x e4m3 with fp32 accumulation; P is rounded to e4m3 before
+ * P V (an approximation: about 2^-4 relative per probability), the row sums use
+ * the unrounded P.
+ *   Q8, K8, V8          device uint8 [B,H,N,d] e4m3 codes, 16-byte aligned.
+ *   q_exp, k_exp, v_exp device int32 [B,H,ceil(N/block)] block exponents.
+ *   Other arguments, layouts, outputs (O bf16, LSE fp32 natural log), workspace
+ *   (fvattn_fwd_workspace_bytes) and errors as fvattn_sparse_fwd.
+ * Supported: d = 128 (an e4m3 row fills one 128-byte swizzle span), block 64 or
+ * 128; other d give FVATTN_ERR_UNSUPPORTED.
+ */
+FVATTN_API int fvattn_sparse_fwd_fp8(const void *Q8, const void *K8, const void *V8, const int32_t *q_exp,
+                                     const int32_t *k_exp, const int32_t *v_exp, const int32_t *row_ptr,
+                                     const int32_t *col_idx, int B, int H, int N, int d, int block, int causal,
+                                     void *O, float *LSE, void *workspace, size_t ws_bytes, int32_t *dev_status,
+                                     fvattn_stream_t stream);
 
 /*
  * fvattn_attn_work_order -- the order in which fvattn_sparse_fwd takes its work

@@ -41,7 +41,13 @@ _lib = None
 class FvattnError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
-        super().__init__(f"{where}: {status} ({status_string(status)})")
+        detail = ""
+        if status == FVATTN_ERR_CUDA:
+            try:
+                detail = ": " + load_library().fvattn_last_error().decode()
+            except Exception:
+                pass
+        super().__init__(f"{where}: {status} ({status_string(status)}{detail})")
 
 
 def load_library(path: str | None = None) -> ctypes.CDLL:
@@ -58,6 +64,7 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     sig = {
         "fvattn_status_string": (ctypes.c_char_p, [I]),
         "fvattn_build_info": (ctypes.c_char_p, []),
+        "fvattn_last_error": (ctypes.c_char_p, []),
         "fvattn_num_rows": (I64, [I, I, I, I]),
         "fvattn_route_max_nnz": (I64, [I, I, I, I]),
         "fvattn_route_workspace_bytes": (SZ, [I, I, I, I, I]),
@@ -71,6 +78,7 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         "fvattn_test_sparse_fwd_stall": (I, [P, P, P, P, P, I, I, I, I, I, I, P, P, P, SZ, P, P]),
         "fvattn_sparse_fwd_profiled": (I, [P, P, P, P, P, I, I, I, I, I, I, P, P, P, SZ, P, I, P, P, P]),
         "fvattn_attn_work_order": (I, [P, I, I, I, I, P, P, SZ, P]),
+        "fvattn_sparse_fwd_fp8": (I, [P, P, P, P, P, P, P, P, I, I, I, I, I, I, P, P, P, SZ, P, P]),
         "fvattn_bwd_workspace_bytes": (SZ, [I, I, I, I]),
         "fvattn_sparse_bwd": (I, [P, P, P, P, P, P, P, P, I, I, I, I, I, I, P, P, P, P, SZ, P, P]),
         "fvattn_attention_host": (I, [P, P, P, I, I, I, I, I, D, I, P, P, P, P, P, P, P, P, P, I64, P, P, SZ, P, SZ,
@@ -252,7 +260,7 @@ def fvattn_sparse_fwd_profiled(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor
     if workspace is None:
         workspace = _empty_bytes(fvattn_fwd_workspace_bytes(B, H, N, block), dev)
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
-    busy = torch.zeros(2 * sms, dtype=torch.int64, device=dev)   # the persistent grid runs two CTAs per SM
+    busy = torch.zeros(sms, dtype=torch.int64, device=dev)
     grid = ctypes.c_int(0)
     rc = lib.fvattn_sparse_fwd_profiled(_ptr(Q), _ptr(K), _ptr(V), _ptr(row_ptr), _ptr(col_idx), B, H, N, d, block,
                                         1 if causal else 0, _ptr(O), _ptr(LSE), _ptr(workspace), workspace.numel(),
@@ -260,6 +268,31 @@ def fvattn_sparse_fwd_profiled(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor
                                         _stream_ptr(stream))
     _check(rc, "fvattn_sparse_fwd_profiled")
     return O, LSE, dev_status, busy[: grid.value]
+
+
+def fvattn_sparse_fwd_fp8(Q8: torch.Tensor, K8: torch.Tensor, V8: torch.Tensor, q_exp: torch.Tensor,
+                          k_exp: torch.Tensor, v_exp: torch.Tensor, row_ptr: torch.Tensor, col_idx: torch.Tensor,
+                          block: int, causal: bool = False, *, stream=None, O: torch.Tensor | None = None,
+                          LSE: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                          dev_status: torch.Tensor | None = None):
+    """Block-sparse attention on e4m3 operands (codes uint8 [B,H,N,d] and int32 block
+    exponents [B,H,nb], as fvattn_quant_e4m3 returns them).  Returns (O, LSE, dev_status)."""
+    lib = load_library()
+    B, H, N, d = (int(x) for x in Q8.shape)
+    dev = Q8.device
+    if O is None:
+        O = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev)
+    if LSE is None:
+        LSE = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    if dev_status is None:
+        dev_status = torch.zeros(1, dtype=torch.int32, device=dev)
+    if workspace is None:
+        workspace = _empty_bytes(fvattn_fwd_workspace_bytes(B, H, N, block), dev)
+    rc = lib.fvattn_sparse_fwd_fp8(_ptr(Q8), _ptr(K8), _ptr(V8), _ptr(q_exp), _ptr(k_exp), _ptr(v_exp), _ptr(row_ptr),
+                                   _ptr(col_idx), B, H, N, d, block, 1 if causal else 0, _ptr(O), _ptr(LSE),
+                                   _ptr(workspace), workspace.numel(), _ptr(dev_status), _stream_ptr(stream))
+    _check(rc, "fvattn_sparse_fwd_fp8")
+    return O, LSE, dev_status
 
 
 def fvattn_attn_work_order(row_ptr: torch.Tensor, B: int, H: int, N: int, block: int, *, stream=None,

@@ -21,6 +21,12 @@
 using namespace fvattn;
 
 namespace {
+thread_local const char *t_last_error = "";
+}  // namespace
+
+void fvattn::set_last_error(const char *what) { t_last_error = what ? what : ""; }
+
+namespace {
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
@@ -84,17 +90,20 @@ int check_device() {
     return FVATTN_OK;
 }
 
-// 3-D map over a contiguous bf16 [B*H, N, d] tensor; box = 64 columns (128 bytes,
-// the swizzle width) x `rows` tokens x 1 head; out-of-range rows read as zero.
-bool make_map(CUtensorMap *m, const void *base, int64_t BH, int N, int d, int rows) {
+// 3-D map over a contiguous [B*H, N, d] tensor of bf16 (elem_bytes 2) or of 8-bit
+// codes (elem_bytes 1); box = 128 bytes of columns (the swizzle width) x `rows`
+// tokens x 1 head; out-of-range rows read as zero.
+bool make_map(CUtensorMap *m, const void *base, int64_t BH, int N, int d, int rows, int elem_bytes = 2) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;
+    const cuuint64_t eb = static_cast<cuuint64_t>(elem_bytes);
     cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
-    cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(N) * d * 2};
-    cuuint32_t box[3] = {64, static_cast<cuuint32_t>(rows), 1};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * eb, static_cast<cuuint64_t>(N) * d * eb};
+    cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / elem_bytes), static_cast<cuuint32_t>(rows), 1};
     cuuint32_t estr[3] = {1, 1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+    return enc(m, elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 3,
+               const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -113,7 +122,11 @@ FwdWorkspace fwd_layout(int64_t items, int64_t BH) {
     return w;
 }
 
-int from_cuda(cudaError_t e) { return e == cudaSuccess ? FVATTN_OK : FVATTN_ERR_CUDA; }
+int from_cuda(cudaError_t e) {
+    if (e == cudaSuccess) return FVATTN_OK;
+    set_last_error(cudaGetErrorName(e));
+    return FVATTN_ERR_CUDA;
+}
 
 struct BwdWorkspace {
     size_t D, col_ptr, csc_idx, order_q, order_k, head_rank, counters, total;
@@ -158,7 +171,9 @@ const char *fvattn_status_string(int status) {
     }
 }
 
-const char *fvattn_build_info(void) { return "libfvattn 0.1 sm_100a (tcgen05/TMA/TMEM)"; }
+const char *fvattn_build_info(void) { return "libfvattn 0.2 sm_100a (tcgen05/TMA/TMEM)"; }
+
+const char *fvattn_last_error(void) { return t_last_error; }
 
 int64_t fvattn_num_rows(int B, int H, int N, int block) {
     if (B < 1 || H < 1 || N < 1 || block < 1) return 0;
@@ -238,13 +253,20 @@ int fvattn_quant_e4m3(const void *X, int B, int H, int N, int d, int block, uint
                                        reinterpret_cast<cudaStream_t>(stream)));
 }
 
+// exps: e4m3 operands (Q, K, V are codes) with their block exponents {q, k, v}, or null for bf16.
 static int sparse_fwd_impl(const void *Q, const void *K, const void *V, const int32_t *row_ptr,
                            const int32_t *col_idx, int B, int H, int N, int d, int block, int causal, void *O,
                            float *LSE, void *workspace, size_t ws_bytes, int32_t *dev_status, fvattn_stream_t stream,
                            int test_stall, int order_mode = 0, int64_t *cta_busy_ns = nullptr,
-                           int *grid_out = nullptr) {
+                           int *grid_out = nullptr, const int32_t *const *exps = nullptr) {
     int rc = check_shape(B, H, N, d, block);
     if (rc != FVATTN_OK) return rc;
+    const bool fp8 = exps != nullptr;
+    if (fp8 && d != 128) return FVATTN_ERR_UNSUPPORTED;
+    if (fp8 && (!exps[0] || !exps[1] || !exps[2])) return FVATTN_ERR_INVALID_ARG;
+    if (fp8 && ((reinterpret_cast<uintptr_t>(exps[0]) | reinterpret_cast<uintptr_t>(exps[1]) |
+                 reinterpret_cast<uintptr_t>(exps[2])) & 3u))
+        return FVATTN_ERR_ALIGNMENT;
     if (!Q || !K || !V || !row_ptr || !col_idx || !O || !LSE || !workspace || !dev_status)
         return FVATTN_ERR_INVALID_ARG;
     if (causal != 0 && causal != 1) return FVATTN_ERR_INVALID_ARG;
@@ -268,7 +290,9 @@ static int sparse_fwd_impl(const void *Q, const void *K, const void *V, const in
     int *counter = reinterpret_cast<int *>(ws + w.counter);
 
     CUtensorMap mq, mk, mv;
-    if (!make_map(&mq, Q, BH, N, d, block) || !make_map(&mk, K, BH, N, d, block) || !make_map(&mv, V, BH, N, d, block))
+    const int eb = fp8 ? 1 : 2;
+    if (!make_map(&mq, Q, BH, N, d, block, eb) || !make_map(&mk, K, BH, N, d, block, eb) ||
+        !make_map(&mv, V, BH, N, d, block, eb))
         return FVATTN_ERR_CUDA;
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -295,12 +319,25 @@ static int sparse_fwd_impl(const void *Q, const void *K, const void *V, const in
     a.O = O;
     a.LSE = LSE;
     a.dev_status = dev_status;
-    const int64_t max_grid = static_cast<int64_t>(attn_ctas_per_sm()) * info.sms;
-    a.grid = static_cast<int>(items < max_grid ? items : max_grid);
+    a.sms = info.sms;
+    a.grid_out = grid_out;
     a.test_stall = test_stall;
     a.cta_busy_ns = reinterpret_cast<long long *>(cta_busy_ns);
-    if (grid_out) *grid_out = a.grid;
-    return from_cuda(launch_sparse_attn(a, d, block, s));
+    if (fp8) {
+        a.q_exp = exps[0];
+        a.k_exp = exps[1];
+        a.v_exp = exps[2];
+    }
+    return from_cuda(fp8 ? launch_sparse_attn_fp8(a, block, s) : launch_sparse_attn(a, d, block, s));
+}
+
+int fvattn_sparse_fwd_fp8(const void *Q8, const void *K8, const void *V8, const int32_t *q_exp, const int32_t *k_exp,
+                          const int32_t *v_exp, const int32_t *row_ptr, const int32_t *col_idx, int B, int H, int N,
+                          int d, int block, int causal, void *O, float *LSE, void *workspace, size_t ws_bytes,
+                          int32_t *dev_status, fvattn_stream_t stream) {
+    const int32_t *exps[3] = {q_exp, k_exp, v_exp};
+    return sparse_fwd_impl(Q8, K8, V8, row_ptr, col_idx, B, H, N, d, block, causal, O, LSE, workspace, ws_bytes,
+                           dev_status, stream, 0, 0, nullptr, nullptr, exps);
 }
 
 int fvattn_sparse_fwd(const void *Q, const void *K, const void *V, const int32_t *row_ptr, const int32_t *col_idx,

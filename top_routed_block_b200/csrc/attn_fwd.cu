@@ -9,23 +9,26 @@
 //
 // B200 design:
 //   * One work item = one query block of one head (a CSR row).  A persistent
-//     grid of two CTAs per SM pops items from a queue ordered head-major and
+//     grid of one CTA per SM pops items from a queue ordered head-major and
 //     longest-first (FVAttn §1 "RLB" balances per-head work at run time; here
 //     the SMs are balanced instead, and the head order keeps one or two heads'
 //     K and V in L2 while all SMs work on them).
-//   * Two CTAs per SM, each with its own query block, its own softmax
-//     warpgroup and half of the tensor memory: while one CTA's softmax
-//     warpgroup works on its tile, the tensor cores run the other CTA's
-//     O += P V and next S = Q K^T.  The per-tile critical path of one
-//     softmax warp per sub-partition (the MUFU exponentials, the row maximum,
-//     tensor-memory traffic) is thereby overlapped twice over per SM.
-//   * Warps 0-3 run the softmax and the epilogue (thread = query row = TMEM
-//     lane); warp 4 issues TMA loads (the item's Q tile, then its K and V
-//     tiles into a ring of shared-memory stages); warp 5 issues the tcgen05
-//     MMAs; warps 6-7 only complete the second warpgroup, which hands
-//     registers to the softmax warpgroup (setmaxnreg).
-//   * Tensor memory (256 columns per CTA): S (fp32, the block's columns) and
-//     O (fp32, d columns).  S = Q K^T is an SS MMA (Q and K from shared
+//   * Two slots per CTA, each an independent pipeline with its own work item,
+//     its own softmax warpgroup and half of the tensor memory: while one
+//     slot's softmax warpgroup works on its tile, the tensor cores run the
+//     other slot's O += P V and next S = Q K^T.  The per-tile critical path of
+//     one softmax warp per sub-partition (the MUFU exponentials, the row
+//     maximum, tensor-memory traffic) is thereby overlapped twice over per SM.
+//     (Two CTAs per SM would do the same, but kernels that hold tensor memory
+//     are resident one CTA per SM.)
+//   * Warps 0-3 and 4-7 run the softmax and the epilogue of slots 0 and 1
+//     (thread = query row = TMEM lane); warps 8 and 9 issue the TMA loads of
+//     slots 0 and 1 (the item's Q tile, then its K and V tiles into the slot's
+//     ring of shared-memory stages); warps 10 and 11 issue the slots' tcgen05
+//     MMAs.  The third warpgroup hands registers to the softmax warpgroups
+//     (setmaxnreg).
+//   * Tensor memory (256 of the 512 columns per slot): S (fp32, the block's
+//     columns) and O (fp32, d columns).  S = Q K^T is an SS MMA (Q and K from shared
 //     memory); the softmax warps read S with tcgen05.ld, write P as bf16 pairs
 //     into the first columns of S, and O += P V runs as a TS MMA (P from
 //     TMEM, V from shared memory, MN-major).  tcgen05 MMAs of one thread
@@ -37,6 +40,20 @@
 //     loaded as soon as this item's last S has read the current one.
 //   * Every mbarrier wait is bounded; a timeout raises the CTA abort flag and
 //     records FVATTN_ERR_DEVICE_TIMEOUT; all roles then drain and exit.
+//
+// FP8 variant ("Accelerating HunyuanVideo inference with ParaAttention"
+// (WaveSpeed), § "FP8 dynamic quantization": attention run on FP8 activations):
+// Q, K and V arrive as e4m3 codes with one power-of-two scale 2^e per (head,
+// block) (the block quantization of quant.cu), and both GEMMs run as tcgen05
+// kind::f8f6f4 MMAs (e4m3 x e4m3, fp32 accumulation; twice the bf16 rate).
+//   * S: the codes' dot products are exact products summed in fp32; the tile's
+//     scale 2^(e_q + e_k) is folded into the softmax scale of that tile.
+//   * PV: P is rounded to e4m3 (one scale for all rows of a tile: the key block's
+//     2^(e_v - E), E the largest e_v of the item's blocks so far, so that P <= 256
+//     stays in range) and written four codes per TMEM column; the row sum l uses
+//     the unrounded P.  When a later block has a larger e_v, O is rescaled by the
+//     exact power of two 2^(E_old - E_new) (together with the maximum rescale).
+//     The epilogue multiplies by 2^E / l.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -53,57 +70,67 @@ namespace {
 using namespace ptx;
 
 constexpr int kRowsM = 128;           // query rows per tile (tcgen05 M)
-constexpr int kThreads = 256;         // softmax warpgroup + issue warpgroup
-constexpr int kCtasPerSm = 2;
-constexpr int kTmaWarp = 4;
-constexpr int kMmaWarp = 5;           // warps 6 and 7 only take part in the register hand-over
-// Register hand-over (setmaxnreg): two CTAs of 256 threads share the SM's 65,536
-// registers, 128 per thread at launch; the issue warpgroup drops to kIssueRegs and
-// the softmax warpgroup, which holds a whole S row per thread, rises to
-// kSoftmaxRegs.  The split must not exceed what the launch allocates (checked on
-// the host before the first launch).
-constexpr int kLaunchRegs = 65536 / (kCtasPerSm * kThreads);
-constexpr int kIssueRegs = 48;
-constexpr int kSoftmaxRegs = 208;
-static_assert(128 * kSoftmaxRegs + 128 * kIssueRegs <= kThreads * kLaunchRegs, "register split exceeds the pool");
+constexpr int kSlots = 2;             // work items in flight per CTA, one softmax warpgroup each
+constexpr int kThreads = 384;         // two softmax warpgroups + the issue warpgroup
+constexpr int kCtasPerSm = 1;         // kernels that hold tensor memory are resident one CTA per SM
+constexpr int kTmaWarp = 8;           // warps 8 and 9: TMA producers of slots 0 and 1
+constexpr int kMmaWarp = 10;          // warps 10 and 11: MMA issuers of slots 0 and 1
+// Register hand-over (setmaxnreg): 384 threads share the SM's 65,536 registers,
+// 168 per thread at launch; the issue warpgroup drops to kIssueRegs and the two
+// softmax warpgroups, which hold a whole S row per thread, rise to kSoftmaxRegs.
+// The split must not exceed what the launch allocates (checked on the host before
+// the first launch).
+constexpr int kLaunchRegs = 168;
+constexpr int kIssueRegs = 56;
+constexpr int kSoftmaxRegs = 216;
+static_assert(2 * 128 * kSoftmaxRegs + 128 * kIssueRegs <= kThreads * kLaunchRegs, "register split exceeds the pool");
 static_assert(kSoftmaxRegs % 8 == 0 && kIssueRegs % 8 == 0, "setmaxnreg takes multiples of 8");
-constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTmemSlot = 256;   // TMEM columns per slot
 constexpr int kMaxStages = 12;
-// Dynamic shared memory one CTA may take so that two fit on an SM (228 KB per SM,
-// 1 KB of it reserved per CTA).
-constexpr int kSmemPerCta = 113 * 1024;
+constexpr int kSmemPerCta = 227 * 1024;  // largest dynamic shared memory of one CTA
+constexpr int kSharedBytes = 1024;       // barriers and flags, after the tiles
 
-template <int D, int BS>
+template <int D, int BS, bool F8>
 struct Cfg {
-    static constexpr int KBLK = D / 64;                   // 128-byte (64 x bf16) column blocks along d
+    static constexpr int EB = F8 ? 1 : 2;                 // bytes per operand element (e4m3 or bf16)
+    static_assert((D * EB) % 128 == 0, "rows of d operands must fill whole 128-byte swizzle spans");
+    static constexpr int KBLK = D * EB / 128;             // 128-byte column blocks along d
+    static constexpr int X_CHUNK = 128 / EB;              // elements per 128-byte column block
+    static constexpr int KSTEP_PV = 32 / EB;              // keys per PV MMA (an MMA's K spans 32 bytes)
     static constexpr int STAGE_BYTES = KBLK * BS * 128;   // one K or V tile
     static constexpr int Q_CHUNK = kRowsM * 128;          // one 64-column block of the Q tile (128 rows)
     static constexpr int Q_BYTES = KBLK * Q_CHUNK;
-    static constexpr int NST_FIT = (kSmemPerCta - Q_BYTES - 1024 - 512) / STAGE_BYTES;
+    // per slot: the Q tile and a ring of NST stages
+    static constexpr int NST_FIT = ((kSmemPerCta - 1024 - kSharedBytes) / kSlots - Q_BYTES) / STAGE_BYTES;
     static constexpr int NST = NST_FIT < kMaxStages ? NST_FIT : kMaxStages;
     static_assert(NST >= 2, "the ring needs a K and a V stage");
-    static constexpr int TILE_BYTES = Q_BYTES + NST * STAGE_BYTES;
-    static constexpr int SMEM_BYTES = TILE_BYTES + 1024 /*alignment slack*/ + 512 /*barriers*/;
-    static_assert(SMEM_BYTES <= kSmemPerCta, "two CTAs per SM do not fit");
-    // TMEM columns: S (fp32; P as bf16 pairs in its first BS/2 columns), O (fp32)
+    static constexpr int SLOT_BYTES = Q_BYTES + NST * STAGE_BYTES;
+    static constexpr int SMEM_BYTES = kSlots * SLOT_BYTES + 1024 /*alignment slack*/ + kSharedBytes;
+    static_assert(SMEM_BYTES <= kSmemPerCta, "shared memory exceeds one CTA's limit");
+    // TMEM columns of a slot: S (fp32; P as bf16 pairs or e4m3 quads in its first
+    // columns), O (fp32)
     static constexpr uint32_t T_S = 0, T_O = 128;
-    static_assert(T_O + D <= kTmemCols && BS <= 128, "TMEM layout exceeds the CTA's columns");
-    static constexpr uint32_t IDESC_S = idesc_bf16_f32(kRowsM, BS, 0, 0);
-    static constexpr uint32_t IDESC_PV = idesc_bf16_f32(kRowsM, D, 0, 1);
+    static_assert(T_O + D <= kTmemSlot && BS <= 128, "TMEM layout exceeds the slot's columns");
+    static constexpr uint32_t IDESC_S = F8 ? idesc_e4m3_f32(kRowsM, BS, 0, 0) : idesc_bf16_f32(kRowsM, BS, 0, 0);
+    static constexpr uint32_t IDESC_PV = F8 ? idesc_e4m3_f32(kRowsM, D, 0, 1) : idesc_bf16_f32(kRowsM, D, 0, 1);
 };
 
-struct Barriers {
+struct Barriers {  // one slot's pipeline
     uint64_t ring_full[kMaxStages], ring_empty[kMaxStages];
     uint64_t q_full, q_empty, s_full, p_full;
     uint64_t o_full, o_empty;
     uint64_t sched_full[2], sched_empty[2];
     uint64_t drain;
     int4 sched_item[2];  // {row, col start, count, valid item}
+};
+struct SharedState {
+    Barriers slot[kSlots];
     long long t_start;   // diagnostic: global timer at the start of the CTA's work
     uint32_t tmem_base;
-    int abort_flag;
+    int abort_flag;      // raised by a timed-out wait; every role of both slots drains
 };
-static_assert(sizeof(Barriers) <= 512, "barrier block exceeds its shared-memory reservation");
+static_assert(sizeof(SharedState) <= kSharedBytes, "barrier block exceeds its shared-memory reservation");
 
 constexpr float kRescaleLog2 = 8.0f;  // rescale O only when the row max grows by more than 2^8
 
@@ -125,75 +152,97 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
-template <int D, int BS>
+// Four fp32 values -> four e4m3 codes (a in the low byte): nearest, ties to even,
+// saturating (the inputs here are at most 256, inside the e4m3 range).
+__device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float d) {
+    uint16_t lo, hi;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(lo) : "f"(b), "f"(a));
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(hi) : "f"(d), "f"(c));
+    return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+}
+
+// x * 2^e for the block-scale exponents (exact; the clamp keeps absurd exponent
+// sums of degenerate blocks finite).
+__device__ __forceinline__ float pow2_scale(float x, int e) { return ldexpf(x, max(-200, min(e, 126))); }
+
+template <int D, int BS, bool F8>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                            const __grid_constant__ CUtensorMap tmap_v, const int32_t *__restrict__ row_ptr,
                            const int32_t *__restrict__ col_idx, const int32_t *__restrict__ order, int n_items,
                            int *__restrict__ work_counter, int N, int nb, int causal, float scale_log2,
                            __nv_bfloat16 *__restrict__ O, float *__restrict__ LSE, int32_t *dev_status,
-                           int test_stall, long long *__restrict__ cta_busy_ns) {
-    using C = Cfg<D, BS>;
+                           int test_stall, long long *__restrict__ cta_busy_ns, const int32_t *__restrict__ q_exp,
+                           const int32_t *__restrict__ k_exp, const int32_t *__restrict__ v_exp) {
+    using C = Cfg<D, BS, F8>;
     constexpr int NST = C::NST;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     // 1024-byte alignment for the 128-byte-swizzled tiles
     const uint32_t base_addr = smem_addr(smem_raw);
-    unsigned char *qtile = smem_raw + ((1024 - (base_addr & 1023)) & 1023);  // Q tile, then the ring
-    unsigned char *ring = qtile + C::Q_BYTES;                                 // stage s at s * STAGE_BYTES
-    Barriers *bar = reinterpret_cast<Barriers *>(qtile + C::TILE_BYTES);
+    unsigned char *tiles = smem_raw + ((1024 - (base_addr & 1023)) & 1023);  // per slot: Q tile, then the ring
+    SharedState *sh = reinterpret_cast<SharedState *>(tiles + kSlots * C::SLOT_BYTES);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    volatile int *abort_flag = &bar->abort_flag;
+    volatile int *abort_flag = &sh->abort_flag;
+    // this thread's slot: softmax warpgroups 0 and 1; producers 8, 9; MMA issuers 10, 11
+    const int slot = warp < kTmaWarp ? (warp >> 2) : ((warp - kTmaWarp) & 1);
+    unsigned char *qtile = tiles + slot * C::SLOT_BYTES;
+    unsigned char *ring = qtile + C::Q_BYTES;  // stage s at s * STAGE_BYTES
+    Barriers *bar = &sh->slot[slot];
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < NST; ++s) {
-            mbar_init(&bar->ring_full[s], 1);
-            mbar_init(&bar->ring_empty[s], 1);
+        for (int z = 0; z < kSlots; ++z) {
+            Barriers *b = &sh->slot[z];
+            for (int s = 0; s < NST; ++s) {
+                mbar_init(&b->ring_full[s], 1);
+                mbar_init(&b->ring_empty[s], 1);
+            }
+            mbar_init(&b->q_full, 1);
+            mbar_init(&b->q_empty, 1);
+            mbar_init(&b->s_full, 1);
+            mbar_init(&b->p_full, 4);
+            mbar_init(&b->o_full, 1);
+            mbar_init(&b->o_empty, 4);
+            for (int x = 0; x < 2; ++x) {
+                mbar_init(&b->sched_full[x], 1);
+                mbar_init(&b->sched_empty[x], 1 + 4);
+            }
+            mbar_init(&b->drain, 1);
         }
-        mbar_init(&bar->q_full, 1);
-        mbar_init(&bar->q_empty, 1);
-        mbar_init(&bar->s_full, 1);
-        mbar_init(&bar->p_full, 4);
-        mbar_init(&bar->o_full, 1);
-        mbar_init(&bar->o_empty, 4);
-        for (int x = 0; x < 2; ++x) {
-            mbar_init(&bar->sched_full[x], 1);
-            mbar_init(&bar->sched_empty[x], 1 + 4);
-        }
-        mbar_init(&bar->drain, 1);
-        bar->abort_flag = 0;
+        sh->abort_flag = 0;
         fence_barrier_init();
     }
     if (BS < kRowsM) {
         // Q rows BS..127 of every column block stay zero (TMA fills only the block's rows)
-        for (int i = threadIdx.x; i < C::Q_BYTES / 16; i += kThreads) {
-            if ((i * 16) % C::Q_CHUNK >= BS * 128)
-                reinterpret_cast<uint4 *>(qtile)[i] = make_uint4(0, 0, 0, 0);
+        for (int i = threadIdx.x; i < kSlots * C::SLOT_BYTES / 16; i += kThreads) {
+            const int in_slot = (i * 16) % C::SLOT_BYTES;
+            if (in_slot < C::Q_BYTES && in_slot % C::Q_CHUNK >= BS * 128)
+                reinterpret_cast<uint4 *>(tiles)[i] = make_uint4(0, 0, 0, 0);
         }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
     if (warp == kMmaWarp) {
-        tmem_alloc(&bar->tmem_base, kTmemCols);
+        tmem_alloc(&sh->tmem_base, kTmemCols);
         tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem = bar->tmem_base;
+    const uint32_t tmem = sh->tmem_base + slot * kTmemSlot;  // this slot's columns
     // global timer (ns) when this CTA starts its items, if busy times are asked for (kept in
     // shared memory: nothing of the prologue stays live in registers across the hand-over)
     if (cta_busy_ns && threadIdx.x == 0) {
         long long t0;
         asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
-        bar->t_start = t0;
+        sh->t_start = t0;
     }
 
     if (warp >= kTmaWarp) {
     // The register hand-over and the code that uses the new count sit in the same
     // branch, so the compiler allocates each role's registers against its own limit.
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kIssueRegs));
-    if (warp == kTmaWarp) {
+    if (warp < kMmaWarp) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             prefetch_tensormap(&tmap_q);
@@ -223,12 +272,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                 const int bh = rw / nb, qb = rw % nb;
                 // the item's Q tile, once the previous item's last S has read the buffer
                 if (!mbar_wait(&bar->q_empty, (qn & 1) ^ 1, abort_flag, dev_status)) break;
-                // Test hook: CTA 0 never loads its first Q tile, so the MMA warp's bounded
-                // wait for it runs out (exercises the timeout path).
-                if (!(test_stall && blockIdx.x == 0 && qn == 0)) {
+                // Test hook: slot 0 of CTA 0 never loads its first Q tile, so the MMA
+                // warp's bounded wait for it runs out (exercises the timeout path).
+                if (!(test_stall && blockIdx.x == 0 && slot == 0 && qn == 0)) {
                     mbar_arrive_expect_tx(&bar->q_full, C::KBLK * BS * 128);
                     for (int kb = 0; kb < C::KBLK; ++kb)
-                        tma_load_3d(qtile + kb * C::Q_CHUNK, &tmap_q, &bar->q_full, kb * 64, qb * BS, bh);
+                        tma_load_3d(qtile + kb * C::Q_CHUNK, &tmap_q, &bar->q_full, kb * C::X_CHUNK, qb * BS, bh);
                 }
                 ++qn;
                 int prev = -1;
@@ -251,7 +300,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                         mbar_arrive_expect_tx(&bar->ring_full[st], C::STAGE_BYTES);
                         for (int kb = 0; kb < C::KBLK; ++kb)
                             tma_load_3d(ring + st * C::STAGE_BYTES + kb * BS * 128, kv == 0 ? &tmap_k : &tmap_v,
-                                        &bar->ring_full[st], kb * 64, kblk * BS, bh);
+                                        &bar->ring_full[st], kb * C::X_CHUNK, kblk * BS, bh);
                         ++rc;
                     }
                 }
@@ -263,9 +312,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                     mbar_wait_teardown(&bar->ring_full[st], (times - 1) & 1);
                 }
             }
-            if (qn > 0 && !(test_stall && blockIdx.x == 0 && qn == 1)) mbar_wait_teardown(&bar->q_full, (qn - 1) & 1);
+            if (qn > 0 && !(test_stall && blockIdx.x == 0 && slot == 0 && qn == 1))
+                mbar_wait_teardown(&bar->q_full, (qn - 1) & 1);
         }
-    } else if (warp == kMmaWarp) {
+    } else {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             const uint32_t r0 = smem_addr(ring);
@@ -286,20 +336,31 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 #pragma unroll 1
                 for (int kb = 0; kb < C::KBLK; ++kb) {
 #pragma unroll
-                    for (int k = 0; k < 4; ++k)
-                        mma_ss_nc(tmem + C::T_S, qdesc + ((kb * C::Q_CHUNK + k * 32) >> 4),
-                                  kdesc + ((kb * BS * 128 + k * 32) >> 4), C::IDESC_S, (kb | k) ? 1u : 0u);
+                    for (int k = 0; k < 4; ++k) {
+                        const uint64_t da = qdesc + ((kb * C::Q_CHUNK + k * 32) >> 4);
+                        const uint64_t db = kdesc + ((kb * BS * 128 + k * 32) >> 4);
+                        if (F8)
+                            mma_ss_f8_nc(tmem + C::T_S, da, db, C::IDESC_S, (kb | k) ? 1u : 0u);
+                        else
+                            mma_ss_nc(tmem + C::T_S, da, db, C::IDESC_S, (kb | k) ? 1u : 0u);
+                    }
                 }
             };
             // O (+)= P V, P from the S columns, V from ring stage st (MN-major)
             auto issue_pv = [&](uint32_t st, bool first) {
                 const uint64_t vdesc = smem_desc_sw128(r0 + st * C::STAGE_BYTES, BS * 128, 1024);
 #pragma unroll 1
-                for (int k0 = 0; k0 < BS / 16; k0 += 4) {
+                for (int k0 = 0; k0 < BS / C::KSTEP_PV; k0 += 2) {
 #pragma unroll
-                    for (int k = k0; k < k0 + 4; ++k)
-                        mma_ts_nc(tmem + C::T_O, tmem + C::T_S + k * 8, vdesc + ((k * 16 * 128) >> 4), C::IDESC_PV,
-                                  (!first || k > 0) ? 1u : 0u);
+                    for (int k = k0; k < k0 + 2; ++k) {
+                        const uint64_t dv = vdesc + ((k * C::KSTEP_PV * 128) >> 4);
+                        if (F8)
+                            mma_ts_f8_nc(tmem + C::T_O, tmem + C::T_S + k * 8, dv, C::IDESC_PV,
+                                         (!first || k > 0) ? 1u : 0u);
+                        else
+                            mma_ts_nc(tmem + C::T_O, tmem + C::T_S + k * 8, dv, C::IDESC_PV,
+                                      (!first || k > 0) ? 1u : 0u);
+                    }
                 }
             };
             while (ok) {
@@ -357,9 +418,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     }
     } else {
         asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
-        // ------------------------------------------------ softmax / epilogue (warps 0-3)
-        const int r = threadIdx.x;                                  // tile row = TMEM lane
-        const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+        // ------------------------------------------------ softmax / epilogue (warps 0-7)
+        const int r = threadIdx.x & (kRowsM - 1);                   // tile row = TMEM lane
+        const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
         const uint32_t tS = tmem + lane_base + C::T_S;
         const uint32_t tO = tmem + lane_base + C::T_O;
         uint32_t it = 0, tc = 0, on = 0;  // items read, tiles, outputs
@@ -382,11 +443,24 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             float m = -CUDART_INF_F, l = 0.0f;
             int prev = -1;
             int kblk_next = count > 0 ? __ldg(col_idx + start) : 0;  // loaded one tile ahead
+            // e4m3 operands: the item's Q exponent, the running V reference exponent E
+            const int eq = F8 ? __ldg(q_exp + row) : 0;
+            int e_ref = 0;
+            bool have_ref = false;
             for (int j = 0; j < count; ++j) {
                 const int kblk = kblk_next;
                 if (j + 1 < count) kblk_next = __ldg(col_idx + start + j + 1);
                 const bool valid = kblk >= 0 && kblk < nb && kblk > prev;
                 if (valid) prev = kblk;
+                // this tile's score scale (log2 units) and, for e4m3, its V exponent
+                float sc = scale_log2;
+                int ev = 0;
+                if (F8 && valid) {
+                    sc = pow2_scale(scale_log2, eq + __ldg(k_exp + bh * nb + kblk));
+                    ev = __ldg(v_exp + bh * nb + kblk);
+                }
+                const bool e_up = F8 && valid && (!have_ref || ev > e_ref);
+                const int e_new = e_up ? ev : e_ref;
                 const int key0 = kblk * BS;
                 // keys of this block that exist and are allowed for this row
                 int lim = valid ? min(BS, N - key0) : 0;
@@ -414,31 +488,50 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                     for (int q = 0; q < 4; ++q)
                         mq[q] = max3f(mq[q], __uint_as_float(v[c + 2 * q]), __uint_as_float(v[c + 2 * q + 1]));
                 }
-                const float mxs = max3f(mq[0], mq[1], fmaxf(mq[2], mq[3])) * scale_log2;
+                const float mxs = max3f(mq[0], mq[1], fmaxf(mq[2], mq[3])) * sc;
                 // The reference maximum only moves when the row maximum exceeds it by
                 // more than 2^8: P stays below 256 and the rescale of O is rare.  O and
                 // l always share the same reference, so the final O / l is exact.
                 const bool need = mxs > m + kRescaleLog2;
                 const float m_new = need ? mxs : m;
-                const float alpha = need ? ex2_approx(m - m_new) : 1.0f;
+                const float alpha_m = need ? ex2_approx(m - m_new) : 1.0f;  // rescale of l and O
+                float alpha = alpha_m;
                 const float neg_m = (m_new == -CUDART_INF_F) ? 0.0f : -m_new;
                 float rs[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-                // P packed as bf16 pairs in place, v[c/2] <- (p[c], p[c+1]); one loop for
-                // full and masked tiles (masked scores are -inf, and 2^-inf = 0)
+                if (!F8) {
+                    // P packed as bf16 pairs in place, v[c/2] <- (p[c], p[c+1]); one loop for
+                    // full and masked tiles (masked scores are -inf, and 2^-inf = 0)
 #pragma unroll
-                for (int c = 0; c < BS; c += 2) {
-                    const float p0 = ex2_approx(fmaf(__uint_as_float(v[c]), scale_log2, neg_m));
-                    const float p1 = ex2_approx(fmaf(__uint_as_float(v[c + 1]), scale_log2, neg_m));
-                    rs[(c >> 1) & 3] += p0 + p1;
-                    v[c >> 1] = pack_bf16(p0, p1);
+                    for (int c = 0; c < BS; c += 2) {
+                        const float p0 = ex2_approx(fmaf(__uint_as_float(v[c]), sc, neg_m));
+                        const float p1 = ex2_approx(fmaf(__uint_as_float(v[c + 1]), sc, neg_m));
+                        rs[(c >> 1) & 3] += p0 + p1;
+                        v[c >> 1] = pack_bf16(p0, p1);
+                    }
+#pragma unroll
+                    for (int c0 = 0; c0 < BS / 2; c0 += 32)
+                        tmem_st32(tS + c0, *reinterpret_cast<const uint32_t(*)[32]>(&v[c0]));
+                } else {
+                    // P * 2^(e_v - E) as e4m3 quads in place, v[c/4] <- (p[c] .. p[c+3])
+                    const float fv = pow2_scale(1.0f, ev - e_new);
+#pragma unroll
+                    for (int c = 0; c < BS; c += 4) {
+                        const float p0 = ex2_approx(fmaf(__uint_as_float(v[c]), sc, neg_m));
+                        const float p1 = ex2_approx(fmaf(__uint_as_float(v[c + 1]), sc, neg_m));
+                        const float p2 = ex2_approx(fmaf(__uint_as_float(v[c + 2]), sc, neg_m));
+                        const float p3 = ex2_approx(fmaf(__uint_as_float(v[c + 3]), sc, neg_m));
+                        rs[(c >> 2) & 3] += (p0 + p1) + (p2 + p3);
+                        v[c >> 2] = pack_e4m3x4(p0 * fv, p1 * fv, p2 * fv, p3 * fv);
+                    }
+#pragma unroll
+                    for (int c0 = 0; c0 < BS / 4; c0 += 32)
+                        tmem_st32(tS + c0, *reinterpret_cast<const uint32_t(*)[32]>(&v[c0]));
+                    if (e_up && have_ref) alpha = pow2_scale(alpha_m, e_ref - e_new);  // O in units of 2^E
                 }
-#pragma unroll
-                for (int c0 = 0; c0 < BS / 2; c0 += 32)
-                    tmem_st32(tS + c0, *reinterpret_cast<const uint32_t(*)[32]>(&v[c0]));
-                l = l * alpha + ((rs[0] + rs[1]) + (rs[2] + rs[3]));
+                l = l * alpha_m + ((rs[0] + rs[1]) + (rs[2] + rs[3]));
                 // Rescale the running output.  S of this block completed after PV of the
                 // previous one (one issuing thread, in order), so O is complete here.
-                if (__any_sync(0xffffffffu, need && j > 0)) {
+                if (__any_sync(0xffffffffu, (need && j > 0) || (e_up && have_ref))) {
 #pragma unroll
                     for (int c0 = 0; c0 < D; c0 += 32) {
                         uint32_t o[32];
@@ -454,6 +547,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bar->p_full);
                 m = m_new;
+                e_ref = e_new;
+                have_ref = have_ref || e_up;
                 ++tc;
             }
             if (!ok) break;
@@ -466,7 +561,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             ++on;
             tc_fence_after();
             const bool row_ok = r < BS && t_row < N;
-            const float inv_l = (l > 0.0f) ? 1.0f / l : 0.0f;
+            const float inv_l = (l > 0.0f) ? (F8 ? pow2_scale(1.0f / l, e_ref) : 1.0f / l) : 0.0f;
             __nv_bfloat16 *orow = O + (bh * N + t_row) * D;
 #pragma unroll
             for (int c0 = 0; c0 < D; c0 += 32) {
@@ -503,9 +598,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     if (cta_busy_ns && threadIdx.x == 0) {
         long long t_end;
         asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_end));
-        cta_busy_ns[blockIdx.x] = t_end - bar->t_start;
+        cta_busy_ns[blockIdx.x] = t_end - sh->t_start;
     }
-    if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
+    if (warp == kMmaWarp) tmem_dealloc(sh->tmem_base, kTmemCols);
 }
 
 // Natural order (rows by index), the comparison point for the load-imbalance factor.
@@ -590,10 +685,10 @@ __global__ void __launch_bounds__(kOrderThreads) row_order_kernel(const int32_t 
 // ------------------------------------------------------------------ launcher
 
 int attn_smem_bytes(int d, int bs) {
-    if (d == 128 && bs == 128) return Cfg<128, 128>::SMEM_BYTES;
-    if (d == 128 && bs == 64) return Cfg<128, 64>::SMEM_BYTES;
-    if (d == 64 && bs == 128) return Cfg<64, 128>::SMEM_BYTES;
-    return Cfg<64, 64>::SMEM_BYTES;
+    if (d == 128 && bs == 128) return Cfg<128, 128, false>::SMEM_BYTES;
+    if (d == 128 && bs == 64) return Cfg<128, 64, false>::SMEM_BYTES;
+    if (d == 64 && bs == 128) return Cfg<64, 128, false>::SMEM_BYTES;
+    return Cfg<64, 64, false>::SMEM_BYTES;
 }
 
 int attn_ctas_per_sm() { return kCtasPerSm; }
@@ -623,39 +718,56 @@ cudaError_t launch_natural_order(int64_t n, int32_t *order, cudaStream_t stream)
     return cudaGetLastError();
 }
 
-template <int D, int BS>
+template <int D, int BS, bool F8>
 static cudaError_t launch_t(const AttnLaunch &a, cudaStream_t stream) {
-    auto kern = sparse_attn_fwd_kernel<D, BS>;
+    auto kern = sparse_attn_fwd_kernel<D, BS, F8>;
     // Checked once per instantiation: the register hand-over waits until the pool
-    // holds the requested registers, so it must fit in what the launch allocates,
-    // and two CTAs must be resident per SM (the grid is sized for that).
-    static int state = 0;  // 0 unknown, 1 ok, -1 not launchable as designed
-    if (state == 0) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<D, BS>::SMEM_BYTES);
+    // holds the requested registers, so it must fit in what the launch allocates;
+    // the number of resident CTAs per SM sizes the persistent grid.
+    static int per_sm = 0;  // 0 unknown, > 0 resident CTAs per SM, < 0 not launchable
+    if (per_sm == 0) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<D, BS, F8>::SMEM_BYTES);
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
         if (e != cudaSuccess) return e;
         cudaFuncAttributes fa{};
         if ((e = cudaFuncGetAttributes(&fa, kern)) != cudaSuccess) return e;
-        int per_sm = 0;
-        if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, Cfg<D, BS>::SMEM_BYTES)) !=
+        int occ = 0;
+        if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kThreads, Cfg<D, BS, F8>::SMEM_BYTES)) !=
             cudaSuccess)
             return e;
-        state = (128 * kSoftmaxRegs + 128 * kIssueRegs <= fa.numRegs * kThreads && per_sm >= kCtasPerSm) ? 1 : -1;
+        if (2 * 128 * kSoftmaxRegs + 128 * kIssueRegs > fa.numRegs * kThreads) {
+            set_last_error("attention kernel: register hand-over exceeds the launch's registers");
+            per_sm = -1;
+        } else if (occ < 1) {
+            set_last_error("attention kernel: no CTA fits on an SM");
+            per_sm = -1;
+        } else {
+            per_sm = occ < kCtasPerSm ? occ : kCtasPerSm;
+        }
     }
-    if (state < 0) return cudaErrorInvalidConfiguration;
-    kern<<<a.grid, kThreads, Cfg<D, BS>::SMEM_BYTES, stream>>>(
+    if (per_sm < 0) return cudaErrorInvalidConfiguration;
+    const int64_t cap = static_cast<int64_t>(per_sm) * a.sms;
+    const int grid = static_cast<int>(a.n_items < cap ? a.n_items : cap);
+    if (a.grid_out) *a.grid_out = grid;
+    if (grid <= 0) return cudaSuccess;
+    kern<<<grid, kThreads, Cfg<D, BS, F8>::SMEM_BYTES, stream>>>(
         *a.tmap_q, *a.tmap_k, *a.tmap_v, a.row_ptr, a.col_idx, a.order, a.n_items, a.work_counter, a.N, a.nb,
         a.causal, a.scale_log2, static_cast<__nv_bfloat16 *>(a.O), a.LSE, a.dev_status, a.test_stall,
-        a.cta_busy_ns);
+        a.cta_busy_ns, a.q_exp, a.k_exp, a.v_exp);
     return cudaGetLastError();
 }
 
 cudaError_t launch_sparse_attn(const AttnLaunch &a, int d, int bs, cudaStream_t stream) {
-    if (d == 128 && bs == 128) return launch_t<128, 128>(a, stream);
-    if (d == 128 && bs == 64) return launch_t<128, 64>(a, stream);
-    if (d == 64 && bs == 128) return launch_t<64, 128>(a, stream);
-    return launch_t<64, 64>(a, stream);
+    if (d == 128 && bs == 128) return launch_t<128, 128, false>(a, stream);
+    if (d == 128 && bs == 64) return launch_t<128, 64, false>(a, stream);
+    if (d == 64 && bs == 128) return launch_t<64, 128, false>(a, stream);
+    return launch_t<64, 64, false>(a, stream);
+}
+
+cudaError_t launch_sparse_attn_fp8(const AttnLaunch &a, int bs, cudaStream_t stream) {
+    if (bs == 128) return launch_t<128, 128, true>(a, stream);
+    return launch_t<128, 64, true>(a, stream);
 }
 
 }  // namespace fvattn

@@ -17,9 +17,12 @@ struct AttnLaunch {
     void *O;
     float *LSE;
     int32_t *dev_status;
-    int grid;
+    int sms;            // multiprocessors of the device; the launcher sizes the persistent grid
+    int *grid_out;      // receives the number of CTAs launched, or null
     int test_stall;     // nonzero only from the test hook: one bounded wait runs out
     long long *cta_busy_ns;  // per-CTA busy time (global timer, ns), or null
+    // e4m3 operands only: power-of-two scale exponents per (head, block), int32 [B*H, nb]
+    const int32_t *q_exp, *k_exp, *v_exp;
 };
 
 int attn_smem_bytes(int d, int bs);
@@ -33,5 +36,7 @@ cudaError_t launch_item_order(const int32_t *row_ptr, int64_t BH, int nb, int32_
 cudaError_t launch_natural_order(int64_t n, int32_t *order, cudaStream_t stream);
 int attn_ctas_per_sm();  // resident CTAs per SM the launch grid is sized for
 cudaError_t launch_sparse_attn(const AttnLaunch &a, int d, int bs, cudaStream_t stream);
+// e4m3 operands (tmap_* over uint8 codes), d = 128, bs in {64, 128}.
+cudaError_t launch_sparse_attn_fp8(const AttnLaunch &a, int bs, cudaStream_t stream);
 
 }  // namespace fvattn

@@ -16,6 +16,10 @@ __device__ __forceinline__ void record_error(int32_t *dev_status, int32_t code) 
 }
 
 __host__ __device__ constexpr int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// Host side: records the reason of the calling thread's latest FVATTN_ERR_CUDA (a
+// static string), read back through fvattn_last_error().
+void set_last_error(const char *what);
 __host__ __device__ constexpr size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // Workspace carving: every region starts on a 256-byte boundary.

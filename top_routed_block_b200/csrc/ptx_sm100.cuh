@@ -193,6 +193,27 @@ __device__ __forceinline__ void mma_ts_nc(uint32_t d_tmem, uint32_t a_tmem, uint
         "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate));
 }
 
+// D[tmem] (+)= A[smem desc] * B[smem desc]^T, kind::f8f6f4 (both e4m3 per the
+// instruction descriptor, fp32 accumulate; K = 32 elements per instruction).
+__device__ __forceinline__ void mma_ss_f8_nc(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate));
+}
+
+// D[tmem] (+)= A[tmem] * B[smem desc], kind::f8f6f4 (A: four e4m3 codes per TMEM column).
+__device__ __forceinline__ void mma_ts_f8_nc(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate));
+}
+
 // Arrives once on `bar` when every tcgen05 operation issued so far by this
 // thread has completed.
 __device__ __forceinline__ void mma_commit(uint64_t *bar) {
@@ -252,6 +273,18 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn_maj
     return (1u << 4)                                   // D format: f32
            | (1u << 7)                                 // A format: bf16
            | (1u << 10)                                // B format: bf16
+           | (static_cast<uint32_t>(a_mn_major) << 15) //
+           | (static_cast<uint32_t>(b_mn_major) << 16) //
+           | (static_cast<uint32_t>(N >> 3) << 17)     //
+           | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// Instruction descriptor for kind::f8f6f4 with e4m3 A/B and fp32 D (format code 0
+// is E4M3 for both operands; MN-major operands are allowed for 8-bit formats).
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N, int a_mn_major, int b_mn_major) {
+    return (1u << 4)                                   // D format: f32
+           | (0u << 7)                                 // A format: e4m3
+           | (0u << 10)                                // B format: e4m3
            | (static_cast<uint32_t>(a_mn_major) << 15) //
            | (static_cast<uint32_t>(b_mn_major) << 16) //
            | (static_cast<uint32_t>(N >> 3) << 17)     //
