@@ -253,9 +253,9 @@ FVATTN_API int fvattn_sparse_fwd_noalloc(const void *Q, const void *K, const voi
 
 /*
  * fvattn_test_sparse_fwd_stall -- test hook for failure detection, not for
- * production use.  Same arguments as fvattn_sparse_fwd; the CTA that takes the
- * first work item never receives that item's Q tile, so one of its bounded
- * waits runs out (after about one second) and the call ends with
+ * production use.  Same arguments as fvattn_sparse_fwd; the pipeline that takes
+ * the first work item of the queue never reports that item's Q as loaded, so one
+ * of its bounded waits runs out (after about one second) and the call ends with
  * *dev_status = FVATTN_ERR_DEVICE_TIMEOUT, the rest of the grid finishing its
  * items.  No fault, trap or hang: the CUDA context stays usable.
  */

@@ -289,11 +289,10 @@ static int sparse_fwd_impl(const void *Q, const void *K, const void *V, const in
     int32_t *head_rank = reinterpret_cast<int32_t *>(ws + w.head_rank);
     int *counter = reinterpret_cast<int *>(ws + w.counter);
 
-    CUtensorMap mq, mk, mv;
+    // K and V are read one key block per TMA box
+    CUtensorMap mk, mv;
     const int eb = fp8 ? 1 : 2;
-    if (!make_map(&mq, Q, BH, N, d, block, eb) || !make_map(&mk, K, BH, N, d, block, eb) ||
-        !make_map(&mv, V, BH, N, d, block, eb))
-        return FVATTN_ERR_CUDA;
+    if (!make_map(&mk, K, BH, N, d, block, eb) || !make_map(&mv, V, BH, N, d, block, eb)) return FVATTN_ERR_CUDA;
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if ((rc = from_cuda(cudaMemsetAsync(dev_status, 0, sizeof(int32_t), s))) != FVATTN_OK) return rc;
@@ -304,7 +303,7 @@ static int sparse_fwd_impl(const void *Q, const void *K, const void *V, const in
     if ((rc = from_cuda(cudaMemsetAsync(counter, 0, sizeof(int), s))) != FVATTN_OK) return rc;
 
     AttnLaunch a{};
-    a.tmap_q = &mq;
+    a.Q = Q;
     a.tmap_k = &mk;
     a.tmap_v = &mv;
     a.row_ptr = row_ptr;

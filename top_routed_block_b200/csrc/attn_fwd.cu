@@ -13,31 +13,26 @@
 //     longest-first (FVAttn §1 "RLB" balances per-head work at run time; here
 //     the SMs are balanced instead, and the head order keeps one or two heads'
 //     K and V in L2 while all SMs work on them).
-//   * Two slots per CTA, each an independent pipeline with its own work item,
-//     its own softmax warpgroup and half of the tensor memory: while one
-//     slot's softmax warpgroup works on its tile, the tensor cores run the
-//     other slot's O += P V and next S = Q K^T.  The per-tile critical path of
-//     one softmax warp per sub-partition (the MUFU exponentials, the row
-//     maximum, tensor-memory traffic) is thereby overlapped twice over per SM.
-//     (Two CTAs per SM would do the same, but kernels that hold tensor memory
-//     are resident one CTA per SM.)
-//   * Warps 0-3 and 4-7 run the softmax and the epilogue of slots 0 and 1
-//     (thread = query row = TMEM lane); warps 8 and 9 issue the TMA loads of
-//     slots 0 and 1 (the item's Q tile, then its K and V tiles into the slot's
-//     ring of shared-memory stages); warps 10 and 11 issue the slots' tcgen05
-//     MMAs.  The third warpgroup hands registers to the softmax warpgroups
-//     (setmaxnreg).
-//   * Tensor memory (256 of the 512 columns per slot): S (fp32, the block's
-//     columns) and O (fp32, d columns).  S = Q K^T is an SS MMA (Q and K from shared
-//     memory); the softmax warps read S with tcgen05.ld, write P as bf16 pairs
-//     into the first columns of S, and O += P V runs as a TS MMA (P from
-//     TMEM, V from shared memory, MN-major).  tcgen05 MMAs of one thread
-//     execute in issue order: S of block j+1 is issued right behind PV of
-//     block j, which reads the P in the same columns, and the completion of S
-//     of block j+1 also tells the softmax warps that O holds PV of block j.
+//   * Warps 0-3 run the softmax and the epilogue (thread = query row = TMEM
+//     lane); warp 4 issues TMA loads of K and V tiles into a ring of shared
+//     memory stages; warp 5 issues the tcgen05 MMAs.
+//   * Tensor memory (512 columns) holds Q twice (the current and the next
+//     item), S twice and O once (fp32): S = Q K^T of key block j+2 is computed
+//     while the softmax works on block j+1 and the tensor cores run
+//     O += P_j V_j, so the tensor cores never wait for the softmax of the block
+//     they need next.  Q comes from TMEM (TS MMA: only K is read from shared
+//     memory for S), P is written into the columns of its S buffer and read
+//     from there by the PV MMA (V from shared memory, MN-major).
+//   * tcgen05 MMAs of one thread execute in issue order: S of block j+2 is
+//     issued after PV of block j, which reads the P in the same columns.
+//   * The softmax reads the whole S row of its thread (tcgen05.ld), takes the
+//     row maximum, and writes P in place; the running reference maximum moves
+//     only when a row's maximum exceeds it by more than 2^8, so the rescale of
+//     O in tensor memory is rare.
 //   * O stays in TMEM for the whole item; the epilogue divides by l, converts
-//     to bf16 and stores; LSE = (m + log2 l) ln 2.  The next item's Q tile is
-//     loaded as soon as this item's last S has read the current one.
+//     to bf16 and stores; LSE = (m + log2 l) ln 2.  The softmax warps load the
+//     next item's Q into TMEM before the epilogue, so the next item's first two
+//     S tiles overlap it.
 //   * Every mbarrier wait is bounded; a timeout raises the CTA abort flag and
 //     records FVATTN_ERR_DEVICE_TIMEOUT; all roles then drain and exit.
 //
@@ -70,26 +65,13 @@ namespace {
 using namespace ptx;
 
 constexpr int kRowsM = 128;           // query rows per tile (tcgen05 M)
-constexpr int kSlots = 2;             // work items in flight per CTA, one softmax warpgroup each
-constexpr int kThreads = 384;         // two softmax warpgroups + the issue warpgroup
+constexpr int kThreads = 192;         // softmax warpgroup + TMA warp + MMA warp
 constexpr int kCtasPerSm = 1;         // kernels that hold tensor memory are resident one CTA per SM
-constexpr int kTmaWarp = 8;           // warps 8 and 9: TMA producers of slots 0 and 1
-constexpr int kMmaWarp = 10;          // warps 10 and 11: MMA issuers of slots 0 and 1
-// Register hand-over (setmaxnreg): 384 threads share the SM's 65,536 registers,
-// 168 per thread at launch; the issue warpgroup drops to kIssueRegs and the two
-// softmax warpgroups, which hold a whole S row per thread, rise to kSoftmaxRegs.
-// The split must not exceed what the launch allocates (checked on the host before
-// the first launch).
-constexpr int kLaunchRegs = 168;
-constexpr int kIssueRegs = 56;
-constexpr int kSoftmaxRegs = 216;
-static_assert(2 * 128 * kSoftmaxRegs + 128 * kIssueRegs <= kThreads * kLaunchRegs, "register split exceeds the pool");
-static_assert(kSoftmaxRegs % 8 == 0 && kIssueRegs % 8 == 0, "setmaxnreg takes multiples of 8");
+constexpr int kTmaWarp = 4;
+constexpr int kMmaWarp = 5;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemSlot = 256;   // TMEM columns per slot
 constexpr int kMaxStages = 12;
-constexpr int kSmemPerCta = 227 * 1024;  // largest dynamic shared memory of one CTA
-constexpr int kSharedBytes = 1024;       // barriers and flags, after the tiles
+constexpr int kRingBytes = 192 * 1024;
 
 template <int D, int BS, bool F8>
 struct Cfg {
@@ -97,40 +79,32 @@ struct Cfg {
     static_assert((D * EB) % 128 == 0, "rows of d operands must fill whole 128-byte swizzle spans");
     static constexpr int KBLK = D * EB / 128;             // 128-byte column blocks along d
     static constexpr int X_CHUNK = 128 / EB;              // elements per 128-byte column block
-    static constexpr int KSTEP_PV = 32 / EB;              // keys per PV MMA (an MMA's K spans 32 bytes)
+    static constexpr int KSTEP = 32 / EB;                 // K of one MMA (32 bytes of operand)
     static constexpr int STAGE_BYTES = KBLK * BS * 128;   // one K or V tile
-    static constexpr int Q_CHUNK = kRowsM * 128;          // one 64-column block of the Q tile (128 rows)
-    static constexpr int Q_BYTES = KBLK * Q_CHUNK;
-    // per slot: the Q tile and a ring of NST stages
-    static constexpr int NST_FIT = ((kSmemPerCta - 1024 - kSharedBytes) / kSlots - Q_BYTES) / STAGE_BYTES;
-    static constexpr int NST = NST_FIT < kMaxStages ? NST_FIT : kMaxStages;
-    static_assert(NST >= 2, "the ring needs a K and a V stage");
-    static constexpr int SLOT_BYTES = Q_BYTES + NST * STAGE_BYTES;
-    static constexpr int SMEM_BYTES = kSlots * SLOT_BYTES + 1024 /*alignment slack*/ + kSharedBytes;
-    static_assert(SMEM_BYTES <= kSmemPerCta, "shared memory exceeds one CTA's limit");
-    // TMEM columns of a slot: S (fp32; P as bf16 pairs or e4m3 quads in its first
-    // columns), O (fp32)
-    static constexpr uint32_t T_S = 0, T_O = 128;
-    static_assert(T_O + D <= kTmemSlot && BS <= 128, "TMEM layout exceeds the slot's columns");
+    static constexpr int NST = kRingBytes / STAGE_BYTES < kMaxStages ? kRingBytes / STAGE_BYTES : kMaxStages;
+    static constexpr int TILE_BYTES = NST * STAGE_BYTES;
+    static constexpr int SMEM_BYTES = TILE_BYTES + 1024 /*alignment slack*/ + 512 /*barriers*/;
+    // TMEM columns: Q buffers (packed operands), S buffers (fp32; P as bf16 pairs or
+    // e4m3 quads in their first columns), O (fp32)
+    static constexpr uint32_t Q_COLS = D * EB / 4;
+    static constexpr uint32_t T_Q0 = 0, T_Q1 = Q_COLS, T_S0 = 128, T_S1 = 128 + BS, T_O = 128 + 2 * BS;
+    static_assert(2 * Q_COLS <= 128 && T_O + D <= kTmemCols, "TMEM layout exceeds 512 columns");
     static constexpr uint32_t IDESC_S = F8 ? idesc_e4m3_f32(kRowsM, BS, 0, 0) : idesc_bf16_f32(kRowsM, BS, 0, 0);
     static constexpr uint32_t IDESC_PV = F8 ? idesc_e4m3_f32(kRowsM, D, 0, 1) : idesc_bf16_f32(kRowsM, D, 0, 1);
 };
 
-struct Barriers {  // one slot's pipeline
+struct Barriers {
     uint64_t ring_full[kMaxStages], ring_empty[kMaxStages];
-    uint64_t q_full, q_empty, s_full, p_full;
-    uint64_t o_full, o_empty;
+    uint64_t q_full[2], s_full[2], p_full[2];
+    uint64_t pv_done, o_full, o_empty;
     uint64_t sched_full[2], sched_empty[2];
     uint64_t drain;
-    int4 sched_item[2];  // {row, col start, count, valid item}
-};
-struct SharedState {
-    Barriers slot[kSlots];
+    int4 sched_item[2];  // {row, col start, count, queue index + 1 (0: no more items)}
     long long t_start;   // diagnostic: global timer at the start of the CTA's work
     uint32_t tmem_base;
-    int abort_flag;      // raised by a timed-out wait; every role of both slots drains
+    int abort_flag;
 };
-static_assert(sizeof(SharedState) <= kSharedBytes, "barrier block exceeds its shared-memory reservation");
+static_assert(sizeof(Barriers) <= 512, "barrier block exceeds its shared-memory reservation");
 
 constexpr float kRescaleLog2 = 8.0f;  // rescale O only when the row max grows by more than 2^8
 
@@ -167,8 +141,8 @@ __device__ __forceinline__ float pow2_scale(float x, int e) { return ldexpf(x, m
 
 template <int D, int BS, bool F8>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
-    sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
-                           const __grid_constant__ CUtensorMap tmap_v, const int32_t *__restrict__ row_ptr,
+    sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
+                           const unsigned char *__restrict__ Qg, const int32_t *__restrict__ row_ptr,
                            const int32_t *__restrict__ col_idx, const int32_t *__restrict__ order, int n_items,
                            int *__restrict__ work_counter, int N, int nb, int causal, float scale_log2,
                            __nv_bfloat16 *__restrict__ O, float *__restrict__ LSE, int32_t *dev_status,
@@ -179,76 +153,52 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     // 1024-byte alignment for the 128-byte-swizzled tiles
     const uint32_t base_addr = smem_addr(smem_raw);
-    unsigned char *tiles = smem_raw + ((1024 - (base_addr & 1023)) & 1023);  // per slot: Q tile, then the ring
-    SharedState *sh = reinterpret_cast<SharedState *>(tiles + kSlots * C::SLOT_BYTES);
+    unsigned char *ring = smem_raw + ((1024 - (base_addr & 1023)) & 1023);  // stage s at s * STAGE_BYTES
+    Barriers *bar = reinterpret_cast<Barriers *>(ring + C::TILE_BYTES);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    volatile int *abort_flag = &sh->abort_flag;
-    // this thread's slot: softmax warpgroups 0 and 1; producers 8, 9; MMA issuers 10, 11
-    const int slot = warp < kTmaWarp ? (warp >> 2) : ((warp - kTmaWarp) & 1);
-    unsigned char *qtile = tiles + slot * C::SLOT_BYTES;
-    unsigned char *ring = qtile + C::Q_BYTES;  // stage s at s * STAGE_BYTES
-    Barriers *bar = &sh->slot[slot];
+    volatile int *abort_flag = &bar->abort_flag;
 
     if (threadIdx.x == 0) {
-        for (int z = 0; z < kSlots; ++z) {
-            Barriers *b = &sh->slot[z];
-            for (int s = 0; s < NST; ++s) {
-                mbar_init(&b->ring_full[s], 1);
-                mbar_init(&b->ring_empty[s], 1);
-            }
-            mbar_init(&b->q_full, 1);
-            mbar_init(&b->q_empty, 1);
-            mbar_init(&b->s_full, 1);
-            mbar_init(&b->p_full, 4);
-            mbar_init(&b->o_full, 1);
-            mbar_init(&b->o_empty, 4);
-            for (int x = 0; x < 2; ++x) {
-                mbar_init(&b->sched_full[x], 1);
-                mbar_init(&b->sched_empty[x], 1 + 4);
-            }
-            mbar_init(&b->drain, 1);
+        for (int s = 0; s < NST; ++s) {
+            mbar_init(&bar->ring_full[s], 1);
+            mbar_init(&bar->ring_empty[s], 1);
         }
-        sh->abort_flag = 0;
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(&bar->q_full[x], 4);
+            mbar_init(&bar->s_full[x], 1);
+            mbar_init(&bar->p_full[x], 4);
+            mbar_init(&bar->sched_full[x], 1);
+            mbar_init(&bar->sched_empty[x], 1 + 4);
+        }
+        mbar_init(&bar->pv_done, 1);
+        mbar_init(&bar->o_full, 1);
+        mbar_init(&bar->o_empty, 4);
+        mbar_init(&bar->drain, 1);
+        bar->abort_flag = 0;
         fence_barrier_init();
     }
-    if (BS < kRowsM) {
-        // Q rows BS..127 of every column block stay zero (TMA fills only the block's rows)
-        for (int i = threadIdx.x; i < kSlots * C::SLOT_BYTES / 16; i += kThreads) {
-            const int in_slot = (i * 16) % C::SLOT_BYTES;
-            if (in_slot < C::Q_BYTES && in_slot % C::Q_CHUNK >= BS * 128)
-                reinterpret_cast<uint4 *>(tiles)[i] = make_uint4(0, 0, 0, 0);
-        }
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    }
     if (warp == kMmaWarp) {
-        tmem_alloc(&sh->tmem_base, kTmemCols);
+        tmem_alloc(&bar->tmem_base, kTmemCols);
         tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem = sh->tmem_base + slot * kTmemSlot;  // this slot's columns
-    // global timer (ns) when this CTA starts its items, if busy times are asked for (kept in
-    // shared memory: nothing of the prologue stays live in registers across the hand-over)
+    const uint32_t tmem = bar->tmem_base;
     if (cta_busy_ns && threadIdx.x == 0) {
         long long t0;
         asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
-        sh->t_start = t0;
+        bar->t_start = t0;
     }
 
-    if (warp >= kTmaWarp) {
-    // The register hand-over and the code that uses the new count sit in the same
-    // branch, so the compiler allocates each role's registers against its own limit.
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kIssueRegs));
-    if (warp < kMmaWarp) {
+    if (warp == kTmaWarp) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
-            prefetch_tensormap(&tmap_q);
             prefetch_tensormap(&tmap_k);
             prefetch_tensormap(&tmap_v);
-            uint32_t it = 0, rc = 0, qn = 0;  // items published, ring loads issued, Q loads issued
+            uint32_t it = 0, rc = 0;  // items published, ring loads issued
             bool ok = true;
             while (ok) {
                 const int idx = atomicAdd(work_counter, 1);
@@ -260,7 +210,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                         record_error(dev_status, FVATTN_ERR_BAD_CSR);
                         c = 0;
                     }
-                    item = make_int4(rw, row_ptr[rw], c, 1);
+                    item = make_int4(rw, row_ptr[rw], c, idx + 1);
                 }
                 const uint32_t k = it & 1;
                 if (!mbar_wait(&bar->sched_empty[k], ((it >> 1) & 1) ^ 1, abort_flag, dev_status)) break;
@@ -268,20 +218,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                 mbar_arrive(&bar->sched_full[k]);
                 ++it;
                 if (rw < 0) break;
-                if (item.z == 0) continue;
-                const int bh = rw / nb, qb = rw % nb;
-                // the item's Q tile, once the previous item's last S has read the buffer
-                if (!mbar_wait(&bar->q_empty, (qn & 1) ^ 1, abort_flag, dev_status)) break;
-                // Test hook: slot 0 of CTA 0 never loads its first Q tile, so the MMA
-                // warp's bounded wait for it runs out (exercises the timeout path).
-                if (!(test_stall && blockIdx.x == 0 && slot == 0 && qn == 0)) {
-                    mbar_arrive_expect_tx(&bar->q_full, C::KBLK * BS * 128);
-                    for (int kb = 0; kb < C::KBLK; ++kb)
-                        tma_load_3d(qtile + kb * C::Q_CHUNK, &tmap_q, &bar->q_full, kb * C::X_CHUNK, qb * BS, bh);
-                }
-                ++qn;
+                const int bh = rw / nb;
                 int prev = -1;
-                int kblk_next = __ldg(col_idx + item.y);  // loaded one tile ahead
+                int kblk_next = item.z > 0 ? __ldg(col_idx + item.y) : 0;  // loaded one tile ahead
                 for (int j = 0; j < item.z && ok; ++j) {
                     int kblk = kblk_next;
                     if (j + 1 < item.z) kblk_next = __ldg(col_idx + item.y + j + 1);
@@ -312,55 +251,42 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                     mbar_wait_teardown(&bar->ring_full[st], (times - 1) & 1);
                 }
             }
-            if (qn > 0 && !(test_stall && blockIdx.x == 0 && slot == 0 && qn == 1))
-                mbar_wait_teardown(&bar->q_full, (qn - 1) & 1);
         }
-    } else {
+    } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             const uint32_t r0 = smem_addr(ring);
-            const uint32_t q0 = smem_addr(qtile);
-            uint32_t it = 0, rc = 0, tc = 0, qn = 0, on = 0;  // items, ring loads, tiles, Q tiles, outputs
+            uint32_t it = 0, rc = 0, tc = 0, qn = 0, on = 0;  // items, ring loads, tiles, Q loads, outputs
             bool ok = true;
             auto wait = [&](uint64_t *b, uint32_t parity) {
                 if (ok && !mbar_wait(b, parity, abort_flag, dev_status)) ok = false;
                 return ok;
             };
-            // S = Q K^T, Q from the Q tile, K from ring stage st (both K-major in shared memory)
-            // (descriptors of each k-step: one base descriptor plus the step's byte offset >> 4;
-            // shared-memory addresses stay below 2^18, so the 14-bit address field never carries)
-            // (kept as loops: the issue warpgroup runs on few registers)
-            const uint64_t qdesc = smem_desc_sw128(q0, 16, 1024);
-            auto issue_s = [&](uint32_t st) {
+            // S[scol] = Q[qcol] K^T: Q from TMEM, K of ring stage st (K-major in shared
+            // memory).  The descriptors of the k-steps are one base descriptor plus the
+            // step's byte offset >> 4 (shared-memory addresses stay below 2^18, so the
+            // 14-bit address field never carries).
+            auto issue_s = [&](uint32_t qcol, uint32_t scol, uint32_t st) {
                 const uint64_t kdesc = smem_desc_sw128(r0 + st * C::STAGE_BYTES, 16, 1024);
-#pragma unroll 1
-                for (int kb = 0; kb < C::KBLK; ++kb) {
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const uint64_t da = qdesc + ((kb * C::Q_CHUNK + k * 32) >> 4);
-                        const uint64_t db = kdesc + ((kb * BS * 128 + k * 32) >> 4);
-                        if (F8)
-                            mma_ss_f8_nc(tmem + C::T_S, da, db, C::IDESC_S, (kb | k) ? 1u : 0u);
-                        else
-                            mma_ss_nc(tmem + C::T_S, da, db, C::IDESC_S, (kb | k) ? 1u : 0u);
-                    }
+                for (int k = 0; k < D * C::EB / 32; ++k) {
+                    const uint64_t db = kdesc + (((k >> 2) * BS * 128 + (k & 3) * 32) >> 4);
+                    if (F8)
+                        mma_ts_f8_nc(tmem + scol, tmem + qcol + k * 8, db, C::IDESC_S, k > 0 ? 1u : 0u);
+                    else
+                        mma_ts_nc(tmem + scol, tmem + qcol + k * 8, db, C::IDESC_S, k > 0 ? 1u : 0u);
                 }
             };
-            // O (+)= P V, P from the S columns, V from ring stage st (MN-major)
-            auto issue_pv = [&](uint32_t st, bool first) {
+            // O (+)= P V, P from the S buffer at scol, V of ring stage st (MN-major)
+            auto issue_pv = [&](uint32_t scol, uint32_t st, bool first) {
                 const uint64_t vdesc = smem_desc_sw128(r0 + st * C::STAGE_BYTES, BS * 128, 1024);
-#pragma unroll 1
-                for (int k0 = 0; k0 < BS / C::KSTEP_PV; k0 += 2) {
 #pragma unroll
-                    for (int k = k0; k < k0 + 2; ++k) {
-                        const uint64_t dv = vdesc + ((k * C::KSTEP_PV * 128) >> 4);
-                        if (F8)
-                            mma_ts_f8_nc(tmem + C::T_O, tmem + C::T_S + k * 8, dv, C::IDESC_PV,
-                                         (!first || k > 0) ? 1u : 0u);
-                        else
-                            mma_ts_nc(tmem + C::T_O, tmem + C::T_S + k * 8, dv, C::IDESC_PV,
-                                      (!first || k > 0) ? 1u : 0u);
-                    }
+                for (int k = 0; k < BS / C::KSTEP; ++k) {
+                    const uint64_t dv = vdesc + ((k * C::KSTEP * 128) >> 4);
+                    if (F8)
+                        mma_ts_f8_nc(tmem + C::T_O, tmem + scol + k * 8, dv, C::IDESC_PV, (!first || k > 0) ? 1u : 0u);
+                    else
+                        mma_ts_nc(tmem + C::T_O, tmem + scol + k * 8, dv, C::IDESC_PV, (!first || k > 0) ? 1u : 0u);
                 }
             };
             while (ok) {
@@ -377,31 +303,34 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                     ++on;
                     continue;
                 }
-                if (!wait(&bar->q_full, qn & 1)) break;
-                // S of the first key block
-                if (!wait(&bar->ring_full[rc % NST], (rc / NST) & 1)) break;
+                if (!wait(&bar->q_full[qn & 1], (qn >> 1) & 1)) break;
                 tc_fence_after();
-                issue_s(rc % NST);
-                mma_commit(&bar->s_full);
-                mma_commit(&bar->ring_empty[rc % NST]);
-                if (count == 1) mma_commit(&bar->q_empty);
+                const uint32_t qcol = (qn & 1) ? C::T_Q1 : C::T_Q0;
+                // S of the first two key blocks, into both S buffers
+                for (int j = 0; j < 2 && j < count; ++j) {
+                    const uint32_t ki = rc + 2 * j;
+                    if (!wait(&bar->ring_full[ki % NST], (ki / NST) & 1)) break;
+                    const uint32_t sb = (tc + j) & 1;
+                    issue_s(qcol, sb ? C::T_S1 : C::T_S0, ki % NST);
+                    mma_commit(&bar->s_full[sb]);
+                    mma_commit(&bar->ring_empty[ki % NST]);
+                }
                 for (int j = 0; j < count && ok; ++j) {
-                    const uint32_t t = tc + j;
-                    if (!wait(&bar->p_full, t & 1)) break;
+                    const uint32_t t = tc + j, sb = t & 1, scol = sb ? C::T_S1 : C::T_S0;
+                    if (!wait(&bar->p_full[sb], (t >> 1) & 1)) break;
                     if (j == 0 && !wait(&bar->o_empty, (on & 1) ^ 1)) break;
                     const uint32_t vi = rc + 2 * j + 1;
                     if (!wait(&bar->ring_full[vi % NST], (vi / NST) & 1)) break;
                     tc_fence_after();
-                    issue_pv(vi % NST, j == 0);
+                    issue_pv(scol, vi % NST, j == 0);
                     mma_commit(&bar->ring_empty[vi % NST]);
-                    if (j + 1 < count) {  // S of the next block, behind the PV that reads P in its columns
-                        const uint32_t ki = rc + 2 * (j + 1);
+                    mma_commit(&bar->pv_done);
+                    if (j + 2 < count) {  // the S buffer just read by PV takes block j+2
+                        const uint32_t ki = rc + 2 * (j + 2);
                         if (!wait(&bar->ring_full[ki % NST], (ki / NST) & 1)) break;
-                        tc_fence_after();
-                        issue_s(ki % NST);
-                        mma_commit(&bar->s_full);
+                        issue_s(qcol, scol, ki % NST);
+                        mma_commit(&bar->s_full[sb]);
                         mma_commit(&bar->ring_empty[ki % NST]);
-                        if (j + 2 == count) mma_commit(&bar->q_empty);  // the item's last S has read Q
                     }
                 }
                 if (!ok) break;
@@ -415,15 +344,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             mma_commit(&bar->drain);
             mbar_wait_teardown(&bar->drain, 0);
         }
-    }
     } else {
-        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
-        // ------------------------------------------------ softmax / epilogue (warps 0-7)
-        const int r = threadIdx.x & (kRowsM - 1);                   // tile row = TMEM lane
-        const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-        const uint32_t tS = tmem + lane_base + C::T_S;
-        const uint32_t tO = tmem + lane_base + C::T_O;
-        uint32_t it = 0, tc = 0, on = 0;  // items read, tiles, outputs
+        // ------------------------------------------------ softmax / epilogue (warps 0-3)
+        const int r = threadIdx.x;                                  // tile row = TMEM lane
+        const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+        uint32_t it = 0, tc = 0, qn = 0, on = 0;  // items read, tiles, Q loads, outputs
+        bool ok = true;
         auto next_item = [&](int4 &out) {
             const uint32_t k = it & 1;
             if (!mbar_wait(&bar->sched_full[k], (it >> 1) & 1, abort_flag, dev_status)) return false;
@@ -433,163 +359,207 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             ++it;
             return true;
         };
-        int4 item;
-        bool ok = next_item(item);
-        while (ok && item.w) {
-            const int row = item.x, start = item.y, count = item.z;
-            const int64_t bh = row / nb;
-            const int qb = row % nb;
-            const int t_row = qb * BS + r;  // token index of this thread's row
-            float m = -CUDART_INF_F, l = 0.0f;
-            int prev = -1;
-            int kblk_next = count > 0 ? __ldg(col_idx + start) : 0;  // loaded one tile ahead
-            // e4m3 operands: the item's Q exponent, the running V reference exponent E
-            const int eq = F8 ? __ldg(q_exp + row) : 0;
-            int e_ref = 0;
-            bool have_ref = false;
-            for (int j = 0; j < count; ++j) {
-                const int kblk = kblk_next;
-                if (j + 1 < count) kblk_next = __ldg(col_idx + start + j + 1);
-                const bool valid = kblk >= 0 && kblk < nb && kblk > prev;
-                if (valid) prev = kblk;
-                // this tile's score scale (log2 units) and, for e4m3, its V exponent
-                float sc = scale_log2;
-                int ev = 0;
-                if (F8 && valid) {
-                    sc = pow2_scale(scale_log2, eq + __ldg(k_exp + bh * nb + kblk));
-                    ev = __ldg(v_exp + bh * nb + kblk);
+        // This thread's query row of `itm` (zeros past the block or past N) into the
+        // Q buffer of Q load number qn, as packed operands (bf16 pairs or e4m3 quads,
+        // in order).
+        auto load_q = [&](const int4 &itm) {
+            const int64_t bhq = itm.x / nb;
+            const int tq = (itm.x % nb) * BS + r;
+            const bool in = r < BS && tq < N;
+            const uint4 *src = reinterpret_cast<const uint4 *>(Qg + (bhq * N + (in ? tq : 0)) * (D * C::EB));
+            const uint32_t tQ = tmem + lane_base + ((qn & 1) ? C::T_Q1 : C::T_Q0);
+#pragma unroll
+            for (int c0 = 0; c0 < static_cast<int>(C::Q_COLS); c0 += 32) {
+                uint32_t q[32];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const uint4 x = in ? __ldg(src + c0 / 4 + i) : make_uint4(0, 0, 0, 0);
+                    q[4 * i] = x.x;
+                    q[4 * i + 1] = x.y;
+                    q[4 * i + 2] = x.z;
+                    q[4 * i + 3] = x.w;
                 }
-                const bool e_up = F8 && valid && (!have_ref || ev > e_ref);
-                const int e_new = e_up ? ev : e_ref;
-                const int key0 = kblk * BS;
-                // keys of this block that exist and are allowed for this row
-                int lim = valid ? min(BS, N - key0) : 0;
-                if (causal) lim = min(lim, t_row - key0 + 1);
-                if (!mbar_wait(&bar->s_full, tc & 1, abort_flag, dev_status)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                // the whole S row of this thread: BS fp32 values
-                uint32_t v[BS];
-#pragma unroll
-                for (int c0 = 0; c0 < BS; c0 += 32)
-                    tmem_ld32(tS + c0, *reinterpret_cast<uint32_t(*)[32]>(&v[c0]));
-                tmem_wait_ld();
-                if (lim < BS) {  // ragged last block, causal diagonal, or a skipped index
-#pragma unroll
-                    for (int c = 0; c < BS; ++c)
-                        if (c >= lim) v[c] = __float_as_uint(-CUDART_INF_F);
-                }
-                float mq[4] = {-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F};
-#pragma unroll
-                for (int c = 0; c < BS; c += 8) {
-#pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        mq[q] = max3f(mq[q], __uint_as_float(v[c + 2 * q]), __uint_as_float(v[c + 2 * q + 1]));
-                }
-                const float mxs = max3f(mq[0], mq[1], fmaxf(mq[2], mq[3])) * sc;
-                // The reference maximum only moves when the row maximum exceeds it by
-                // more than 2^8: P stays below 256 and the rescale of O is rare.  O and
-                // l always share the same reference, so the final O / l is exact.
-                const bool need = mxs > m + kRescaleLog2;
-                const float m_new = need ? mxs : m;
-                const float alpha_m = need ? ex2_approx(m - m_new) : 1.0f;  // rescale of l and O
-                float alpha = alpha_m;
-                const float neg_m = (m_new == -CUDART_INF_F) ? 0.0f : -m_new;
-                float rs[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-                if (!F8) {
-                    // P packed as bf16 pairs in place, v[c/2] <- (p[c], p[c+1]); one loop for
-                    // full and masked tiles (masked scores are -inf, and 2^-inf = 0)
-#pragma unroll
-                    for (int c = 0; c < BS; c += 2) {
-                        const float p0 = ex2_approx(fmaf(__uint_as_float(v[c]), sc, neg_m));
-                        const float p1 = ex2_approx(fmaf(__uint_as_float(v[c + 1]), sc, neg_m));
-                        rs[(c >> 1) & 3] += p0 + p1;
-                        v[c >> 1] = pack_bf16(p0, p1);
-                    }
-#pragma unroll
-                    for (int c0 = 0; c0 < BS / 2; c0 += 32)
-                        tmem_st32(tS + c0, *reinterpret_cast<const uint32_t(*)[32]>(&v[c0]));
-                } else {
-                    // P * 2^(e_v - E) as e4m3 quads in place, v[c/4] <- (p[c] .. p[c+3])
-                    const float fv = pow2_scale(1.0f, ev - e_new);
-#pragma unroll
-                    for (int c = 0; c < BS; c += 4) {
-                        const float p0 = ex2_approx(fmaf(__uint_as_float(v[c]), sc, neg_m));
-                        const float p1 = ex2_approx(fmaf(__uint_as_float(v[c + 1]), sc, neg_m));
-                        const float p2 = ex2_approx(fmaf(__uint_as_float(v[c + 2]), sc, neg_m));
-                        const float p3 = ex2_approx(fmaf(__uint_as_float(v[c + 3]), sc, neg_m));
-                        rs[(c >> 2) & 3] += (p0 + p1) + (p2 + p3);
-                        v[c >> 2] = pack_e4m3x4(p0 * fv, p1 * fv, p2 * fv, p3 * fv);
-                    }
-#pragma unroll
-                    for (int c0 = 0; c0 < BS / 4; c0 += 32)
-                        tmem_st32(tS + c0, *reinterpret_cast<const uint32_t(*)[32]>(&v[c0]));
-                    if (e_up && have_ref) alpha = pow2_scale(alpha_m, e_ref - e_new);  // O in units of 2^E
-                }
-                l = l * alpha_m + ((rs[0] + rs[1]) + (rs[2] + rs[3]));
-                // Rescale the running output.  S of this block completed after PV of the
-                // previous one (one issuing thread, in order), so O is complete here.
-                if (__any_sync(0xffffffffu, (need && j > 0) || (e_up && have_ref))) {
-#pragma unroll
-                    for (int c0 = 0; c0 < D; c0 += 32) {
-                        uint32_t o[32];
-                        tmem_ld32(tO + c0, o);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-                        tmem_st32(tO + c0, o);
-                    }
-                }
-                tmem_wait_st();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bar->p_full);
-                m = m_new;
-                e_ref = e_new;
-                have_ref = have_ref || e_up;
-                ++tc;
+                tmem_st32(tQ + c0, q);
             }
-            if (!ok) break;
-            // the next item from the queue, so that its Q tile and first K/V tiles load
-            // while this one finishes
-            int4 nxt;
-            if (!next_item(nxt)) break;
-            // epilogue
-            if (!mbar_wait(&bar->o_full, on & 1, abort_flag, dev_status)) break;
-            ++on;
-            tc_fence_after();
-            const bool row_ok = r < BS && t_row < N;
-            const float inv_l = (l > 0.0f) ? (F8 ? pow2_scale(1.0f / l, e_ref) : 1.0f / l) : 0.0f;
-            __nv_bfloat16 *orow = O + (bh * N + t_row) * D;
-#pragma unroll
-            for (int c0 = 0; c0 < D; c0 += 32) {
-                uint32_t o[32];
-                if (count > 0) {
-                    tmem_ld32(tO + c0, o);
-                    tmem_wait_ld();
-                } else {
-#pragma unroll
-                    for (int c = 0; c < 32; ++c) o[c] = 0u;
-                }
-                uint32_t pk[16];
-#pragma unroll
-                for (int c = 0; c < 32; c += 2)
-                    pk[c >> 1] = pack_bf16(__uint_as_float(o[c]) * inv_l, __uint_as_float(o[c + 1]) * inv_l);
-                if (row_ok) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(orow + c0);
-#pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-                }
-            }
-            if (row_ok)
-                LSE[bh * N + t_row] = (l > 0.0f) ? (m + __log2f(l)) * 0.69314718055994531f : -CUDART_INF_F;
+            tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bar->o_empty);
-            item = nxt;
+            // Test hook: the queue's first item never has its Q reported as loaded, so
+            // the MMA warp's bounded wait for it runs out (exercises the timeout path).
+            if (lane == 0 && !(test_stall && itm.w == 1)) mbar_arrive(&bar->q_full[qn & 1]);
+        };
+        int4 item;
+        if (next_item(item)) {
+            if (item.w && item.z > 0) load_q(item);
+            while (item.w) {
+                const int row = item.x, start = item.y, count = item.z;
+                const int64_t bh = row / nb;
+                const int qb = row % nb;
+                const int t_row = qb * BS + r;  // token index of this thread's row
+                float m = -CUDART_INF_F, l = 0.0f;
+                int prev = -1;
+                int kblk_next = count > 0 ? __ldg(col_idx + start) : 0;  // loaded one tile ahead
+                // e4m3 operands: the item's Q exponent, the running V reference exponent E
+                const int eq = F8 ? __ldg(q_exp + row) : 0;
+                int e_ref = 0;
+                bool have_ref = false;
+                for (int j = 0; j < count; ++j) {
+                    const int kblk = kblk_next;
+                    if (j + 1 < count) kblk_next = __ldg(col_idx + start + j + 1);
+                    const bool valid = kblk >= 0 && kblk < nb && kblk > prev;
+                    if (valid) prev = kblk;
+                    const int key0 = kblk * BS;
+                    // keys of this block that exist and are allowed for this row
+                    int lim = valid ? min(BS, N - key0) : 0;
+                    if (causal) lim = min(lim, t_row - key0 + 1);
+                    // this tile's score scale (log2 units) and, for e4m3, its V exponent
+                    float sc = scale_log2;
+                    int ev = 0;
+                    if (F8 && valid) {
+                        sc = pow2_scale(scale_log2, eq + __ldg(k_exp + bh * nb + kblk));
+                        ev = __ldg(v_exp + bh * nb + kblk);
+                    }
+                    const bool e_up = F8 && valid && (!have_ref || ev > e_ref);
+                    const int e_new = e_up ? ev : e_ref;
+                    const float fv = F8 ? pow2_scale(1.0f, ev - e_new) : 1.0f;
+                    const uint32_t sb = tc & 1;
+                    if (!mbar_wait(&bar->s_full[sb], (tc >> 1) & 1, abort_flag, dev_status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t tS = tmem + lane_base + (sb ? C::T_S1 : C::T_S0);
+                    // the whole S row of this thread: BS fp32 values
+                    uint32_t v[BS];
+#pragma unroll
+                    for (int c0 = 0; c0 < BS; c0 += 32)
+                        tmem_ld32(tS + c0, *reinterpret_cast<uint32_t(*)[32]>(&v[c0]));
+                    tmem_wait_ld();
+                    if (lim < BS) {  // ragged last block, causal diagonal, or a skipped index
+#pragma unroll
+                        for (int c = 0; c < BS; ++c)
+                            if (c >= lim) v[c] = __float_as_uint(-CUDART_INF_F);
+                    }
+                    float mq[4] = {-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F};
+#pragma unroll
+                    for (int c = 0; c < BS; c += 8) {
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            mq[q] = max3f(mq[q], __uint_as_float(v[c + 2 * q]), __uint_as_float(v[c + 2 * q + 1]));
+                    }
+                    const float mxs = max3f(mq[0], mq[1], fmaxf(mq[2], mq[3])) * sc;
+                    // The reference maximum only moves when the row maximum exceeds it by
+                    // more than 2^8: P stays below 256 and the rescale of O is rare.  O and
+                    // l always share the same reference, so the final O / l is exact.
+                    const bool need = mxs > m + kRescaleLog2;
+                    const float m_new = need ? mxs : m;
+                    const float alpha_m = need ? ex2_approx(m - m_new) : 1.0f;  // rescale of l and O
+                    const float neg_m = (m_new == -CUDART_INF_F) ? 0.0f : -m_new;
+                    float rs[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+                    if constexpr (!F8) {
+                        // P packed as bf16 pairs in place, v[c/2] <- (p[c], p[c+1]); one loop for
+                        // full and masked tiles (masked scores are -inf, and 2^-inf = 0)
+#pragma unroll
+                        for (int c = 0; c < BS; c += 2) {
+                            const float p0 = ex2_approx(fmaf(__uint_as_float(v[c]), sc, neg_m));
+                            const float p1 = ex2_approx(fmaf(__uint_as_float(v[c + 1]), sc, neg_m));
+                            rs[(c >> 1) & 3] += p0 + p1;
+                            v[c >> 1] = pack_bf16(p0, p1);
+                        }
+#pragma unroll
+                        for (int c0 = 0; c0 < BS / 2; c0 += 32)
+                            tmem_st32(tS + c0, *reinterpret_cast<const uint32_t(*)[32]>(&v[c0]));
+                    } else {
+                        // P * 2^(e_v - E) as e4m3 quads in place, v[c/4] <- (p[c] .. p[c+3])
+#pragma unroll
+                        for (int c = 0; c < BS; c += 4) {
+                            const float p0 = ex2_approx(fmaf(__uint_as_float(v[c]), sc, neg_m));
+                            const float p1 = ex2_approx(fmaf(__uint_as_float(v[c + 1]), sc, neg_m));
+                            const float p2 = ex2_approx(fmaf(__uint_as_float(v[c + 2]), sc, neg_m));
+                            const float p3 = ex2_approx(fmaf(__uint_as_float(v[c + 3]), sc, neg_m));
+                            rs[(c >> 2) & 3] += (p0 + p1) + (p2 + p3);
+                            v[c >> 2] = pack_e4m3x4(p0 * fv, p1 * fv, p2 * fv, p3 * fv);
+                        }
+                        if constexpr (BS / 4 >= 32)
+                            tmem_st32(tS, *reinterpret_cast<const uint32_t(*)[32]>(&v[0]));
+                        else
+                            tmem_st16(tS, *reinterpret_cast<const uint32_t(*)[16]>(&v[0]));
+                    }
+                    float alpha = alpha_m;
+                    if (F8 && e_up && have_ref) alpha = pow2_scale(alpha_m, e_ref - e_new);  // O in units of 2^E
+                    l = l * alpha_m + ((rs[0] + rs[1]) + (rs[2] + rs[3]));
+                    // Rescale the running output.  The PV of the previous block may still be
+                    // accumulating into O: wait for it first (its completion is phase tc-1
+                    // of pv_done; the PV of this block cannot start before P is published).
+                    if (__any_sync(0xffffffffu, (need && j > 0) || (e_up && have_ref))) {
+                        if (!mbar_wait(&bar->pv_done, (tc - 1) & 1, abort_flag, dev_status)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint32_t tO = tmem + lane_base + C::T_O;
+#pragma unroll
+                        for (int c0 = 0; c0 < D; c0 += 32) {
+                            uint32_t o[32];
+                            tmem_ld32(tO + c0, o);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+                            tmem_st32(tO + c0, o);
+                        }
+                    }
+                    tmem_wait_st();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&bar->p_full[sb]);
+                    m = m_new;
+                    e_ref = e_new;
+                    have_ref = have_ref || e_up;
+                    ++tc;
+                }
+                if (!ok) break;
+                if (count > 0) ++qn;
+                // the next item's Q goes into TMEM before this item's epilogue, so its first
+                // S tiles overlap the epilogue
+                int4 nxt;
+                if (!next_item(nxt)) break;
+                if (nxt.w && nxt.z > 0) load_q(nxt);
+                // epilogue
+                if (!mbar_wait(&bar->o_full, on & 1, abort_flag, dev_status)) break;
+                ++on;
+                tc_fence_after();
+                const bool row_ok = r < BS && t_row < N;
+                const float inv_l = (l > 0.0f) ? (F8 ? pow2_scale(1.0f / l, e_ref) : 1.0f / l) : 0.0f;
+                __nv_bfloat16 *orow = O + (bh * N + t_row) * D;
+                const uint32_t tO = tmem + lane_base + C::T_O;
+#pragma unroll
+                for (int c0 = 0; c0 < D; c0 += 32) {
+                    uint32_t o[32];
+                    if (count > 0) {
+                        tmem_ld32(tO + c0, o);
+                        tmem_wait_ld();
+                    } else {
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) o[c] = 0u;
+                    }
+                    uint32_t pkk[16];
+#pragma unroll
+                    for (int c = 0; c < 32; c += 2)
+                        pkk[c >> 1] = pack_bf16(__uint_as_float(o[c]) * inv_l, __uint_as_float(o[c + 1]) * inv_l);
+                    if (row_ok) {
+                        uint4 *dst = reinterpret_cast<uint4 *>(orow + c0);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            dst[q] = make_uint4(pkk[4 * q], pkk[4 * q + 1], pkk[4 * q + 2], pkk[4 * q + 3]);
+                    }
+                }
+                if (row_ok)
+                    LSE[bh * N + t_row] = (l > 0.0f) ? (m + __log2f(l)) * 0.69314718055994531f : -CUDART_INF_F;
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bar->o_empty);
+                item = nxt;
+            }
         }
     }
     tc_fence_before();
@@ -598,9 +568,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     if (cta_busy_ns && threadIdx.x == 0) {
         long long t_end;
         asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_end));
-        cta_busy_ns[blockIdx.x] = t_end - sh->t_start;
+        cta_busy_ns[blockIdx.x] = t_end - bar->t_start;
     }
-    if (warp == kMmaWarp) tmem_dealloc(sh->tmem_base, kTmemCols);
+    if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
 }
 
 // Natural order (rows by index), the comparison point for the load-imbalance factor.
@@ -721,25 +691,19 @@ cudaError_t launch_natural_order(int64_t n, int32_t *order, cudaStream_t stream)
 template <int D, int BS, bool F8>
 static cudaError_t launch_t(const AttnLaunch &a, cudaStream_t stream) {
     auto kern = sparse_attn_fwd_kernel<D, BS, F8>;
-    // Checked once per instantiation: the register hand-over waits until the pool
-    // holds the requested registers, so it must fit in what the launch allocates;
-    // the number of resident CTAs per SM sizes the persistent grid.
+    // Checked once per instantiation: the number of resident CTAs per SM sizes the
+    // persistent grid.
     static int per_sm = 0;  // 0 unknown, > 0 resident CTAs per SM, < 0 not launchable
     if (per_sm == 0) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<D, BS, F8>::SMEM_BYTES);
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
         if (e != cudaSuccess) return e;
-        cudaFuncAttributes fa{};
-        if ((e = cudaFuncGetAttributes(&fa, kern)) != cudaSuccess) return e;
         int occ = 0;
         if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kThreads, Cfg<D, BS, F8>::SMEM_BYTES)) !=
             cudaSuccess)
             return e;
-        if (2 * 128 * kSoftmaxRegs + 128 * kIssueRegs > fa.numRegs * kThreads) {
-            set_last_error("attention kernel: register hand-over exceeds the launch's registers");
-            per_sm = -1;
-        } else if (occ < 1) {
+        if (occ < 1) {
             set_last_error("attention kernel: no CTA fits on an SM");
             per_sm = -1;
         } else {
@@ -752,9 +716,9 @@ static cudaError_t launch_t(const AttnLaunch &a, cudaStream_t stream) {
     if (a.grid_out) *a.grid_out = grid;
     if (grid <= 0) return cudaSuccess;
     kern<<<grid, kThreads, Cfg<D, BS, F8>::SMEM_BYTES, stream>>>(
-        *a.tmap_q, *a.tmap_k, *a.tmap_v, a.row_ptr, a.col_idx, a.order, a.n_items, a.work_counter, a.N, a.nb,
-        a.causal, a.scale_log2, static_cast<__nv_bfloat16 *>(a.O), a.LSE, a.dev_status, a.test_stall,
-        a.cta_busy_ns, a.q_exp, a.k_exp, a.v_exp);
+        *a.tmap_k, *a.tmap_v, static_cast<const unsigned char *>(a.Q), a.row_ptr, a.col_idx, a.order, a.n_items,
+        a.work_counter, a.N, a.nb, a.causal, a.scale_log2, static_cast<__nv_bfloat16 *>(a.O), a.LSE, a.dev_status,
+        a.test_stall, a.cta_busy_ns, a.q_exp, a.k_exp, a.v_exp);
     return cudaGetLastError();
 }
 

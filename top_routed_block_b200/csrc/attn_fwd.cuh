@@ -8,7 +8,8 @@
 namespace fvattn {
 
 struct AttnLaunch {
-    const CUtensorMap *tmap_q, *tmap_k, *tmap_v;  // host copies, passed by value as kernel parameters
+    const CUtensorMap *tmap_k, *tmap_v;  // host copies, passed by value as kernel parameters
+    const void *Q;                       // [B,H,N,d] bf16 or e4m3 codes, read row by row into tensor memory
     const int32_t *row_ptr, *col_idx, *order;  // order: work items (CSR rows), head-major, longest first
     int n_items;
     int *work_counter;  // zeroed before the launch
