@@ -48,6 +48,9 @@ def _load():
         lib.oracle_attn_rows.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, P, P, P, i64, P, P, i32]
         lib.oracle_attn_tiled.argtypes = lib.oracle_attn_rows.argtypes
         lib.oracle_lpt_order.argtypes = [P, i64, P]
+        lib.oracle_route_cand.argtypes = [P, P, i32, i32, i32, i32, i32, dbl, P, P, i64, P, P, P, P, i32, i32]
+        lib.oracle_head_order.argtypes = [P, i64, i64, P]
+        lib.oracle_sasa.argtypes = [P, P, i64, P, P, i32, P, i32, P, P, P, P, i64]
         lib.oracle_attn_bwd.argtypes = [P, P, P, P, i32, i32, i32, i32, i32, i32, P, P, P, P, P, i32]
         lib.oracle_attn_bwd_sampled.argtypes = [P, P, P, P, i32, i32, i32, i32, i32, i32, P, P, P, i64, P, P, P,
                                                 i64, P, P, i32]
@@ -57,7 +60,8 @@ def _load():
         lib.oracle_e4m3_from_double.argtypes = [dbl]
         lib.oracle_e4m3_from_double.restype = ctypes.c_uint8
         for f in ("oracle_pool", "oracle_route", "oracle_attn_rows", "oracle_attn_tiled", "oracle_lpt_order",
-                  "oracle_attn_bwd", "oracle_attn_bwd_sampled", "oracle_quant_e4m3"):
+                  "oracle_attn_bwd", "oracle_attn_bwd_sampled", "oracle_quant_e4m3", "oracle_route_cand",
+                  "oracle_head_order", "oracle_sasa"):
             getattr(lib, f).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -238,6 +242,67 @@ def dequant_e4m3(codes, exps, bs):
     table = e4m3_decode_table()
     scale = np.ldexp(1.0, np.repeat(exps, bs, axis=2)[:, :, :N])
     return table[codes] * scale[..., None]
+
+
+def route_candidates(Q: np.ndarray, K: np.ndarray, p: float, bs: int, kc: int, nthreads: int | None = None):
+    """:func:`route` plus, per row, the kc key blocks that follow the cut in the
+    routing order (-1 past the last block) and their probabilities."""
+    Q, K = _bits(Q), _bits(K)
+    B, H, N, d = Q.shape
+    nb = -(-N // bs)
+    rows = B * H * nb
+    row_ptr = np.empty(rows + 1, dtype=np.int32)
+    cap = rows * nb
+    col_idx = np.empty(max(cap, 1), dtype=np.int32)
+    head_counts = np.empty(B * H, dtype=np.int32)
+    diag = np.empty((rows, 6), dtype=np.float64)
+    cand = np.empty((rows, max(kc, 1)), dtype=np.int32)
+    cand_p = np.empty((rows, max(kc, 1)), dtype=np.float64)
+    rc = _load().oracle_route_cand(_ptr(Q), _ptr(K), B, H, N, d, bs, float(p), _ptr(row_ptr), _ptr(col_idx), cap,
+                                   _ptr(head_counts), _ptr(diag), _ptr(cand), _ptr(cand_p), kc,
+                                   nthreads or default_threads())
+    if rc != 0:
+        raise ValueError(f"oracle_route_cand failed ({rc})")
+    return Route(row_ptr, col_idx[: row_ptr[-1]].copy(), head_counts, diag), cand[:, :kc], cand_p[:, :kc]
+
+
+def head_order(row_ptr: np.ndarray, BH: int, nb: int) -> np.ndarray:
+    """The attention queue: heads by total selected blocks (desc, ties lower head),
+    rows of a head by block count (desc, ties lower row)."""
+    row_ptr = np.ascontiguousarray(row_ptr, dtype=np.int32)
+    order = np.empty(BH * nb, dtype=np.int32)
+    if _load().oracle_head_order(_ptr(row_ptr), BH, nb, _ptr(order)) != 0:
+        raise ValueError("oracle_head_order failed")
+    return order
+
+
+class Sasa:
+    """Augmented CSR and, per row, the number and probability mass of the added blocks."""
+
+    def __init__(self, row_ptr, col_idx, added, added_mass):
+        self.row_ptr, self.col_idx, self.added, self.added_mass = row_ptr, col_idx, added, added_mass
+
+
+def sasa(row_ptr, col_idx, cand, cand_p, order, machines: int) -> Sasa:
+    """Slack-aware augmentation of a routed mask over `machines` SMs (see
+    oracle_sasa in fvattn_oracle.c)."""
+    row_ptr = np.ascontiguousarray(row_ptr, dtype=np.int32)
+    col_idx = np.ascontiguousarray(col_idx if len(col_idx) else np.zeros(1), dtype=np.int32)
+    cand = np.ascontiguousarray(cand, dtype=np.int32)
+    cand_p = np.ascontiguousarray(cand_p, dtype=np.float64)
+    order = np.ascontiguousarray(order, dtype=np.int32)
+    rows = row_ptr.size - 1
+    kc = cand.shape[1] if cand.ndim == 2 else 0
+    added = np.empty(max(rows, 1), dtype=np.int32)
+    mass = np.empty(max(rows, 1), dtype=np.float64)
+    rp = np.empty(rows + 1, dtype=np.int32)
+    cap = int(row_ptr[-1]) + rows * kc
+    ci = np.empty(max(cap, 1), dtype=np.int32)
+    rc = _load().oracle_sasa(_ptr(row_ptr), _ptr(col_idx), rows, _ptr(cand), _ptr(cand_p), kc, _ptr(order),
+                             int(machines), _ptr(added), _ptr(mass), _ptr(rp), _ptr(ci), cap)
+    if rc != 0:
+        raise ValueError(f"oracle_sasa failed ({rc})")
+    return Sasa(rp, ci[: rp[-1]].copy(), added[:rows], mass[:rows])
 
 
 def lpt_order(row_ptr: np.ndarray) -> np.ndarray:

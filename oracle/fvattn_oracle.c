@@ -43,6 +43,11 @@
  *   attn_bwd_sampled  equal, value for value, to attn_bwd at the sampled
  *               tokens, and to fp64 torch autograd of dense attention
  *   lpt_order   brute-force sort on small inputs
+ *   head_order  brute-force sort on small inputs
+ *   route candidates  the blocks right after the cut in the routing order:
+ *               exhaustive comparison with the selected set's complement
+ *   sasa        Graham's list-scheduling bound, loads within the makespan,
+ *               slack used up unless candidates run out, hand-worked examples
  *   e4m3 / quant_e4m3  the format's own values (known codes, ties to even,
  *               saturation, NaN), round trip of every finite code, monotone
  *               encoding, block scales putting the block maximum in (224, 448],
@@ -161,6 +166,9 @@ typedef struct {
     int32_t *counts;  /* [rows] */
     uint8_t *chosen;  /* [rows, nb] 0/1 */
     double *diag;     /* [rows, 6] or NULL */
+    int32_t *cand;    /* [rows, kc] or NULL: the next key blocks after the cut, in routing order */
+    double *cand_p;   /* [rows, kc] or NULL: their probabilities */
+    int kc;
 } route_ctx;
 
 /*
@@ -223,6 +231,13 @@ static void route_range(void *vctx, int64_t begin, int64_t end) {
         for (int64_t j = 0; j < nb; ++j) ch[j] = 0;
         for (int64_t r = 0; r <= k; ++r) ch[sb[r].j] = 1;
         c->counts[row] = (int32_t)(k + 1);
+        if (c->cand) {
+            for (int e = 0; e < c->kc; ++e) {
+                int64_t r = k + 1 + e;
+                c->cand[row * c->kc + e] = (r < nb) ? (int32_t)sb[r].j : -1;
+                if (c->cand_p) c->cand_p[row * c->kc + e] = (r < nb) ? prob[sb[r].j] : 0.0;
+            }
+        }
         if (c->diag) {
             double *g = c->diag + row * 6;
             g[0] = cum_at_k;                                     /* mass kept */
@@ -242,9 +257,9 @@ static void route_range(void *vctx, int64_t begin, int64_t end) {
  * ascending column indices inside each row, and per-head selected-block counts.
  * Returns 0, -1 on bad arguments, -4 when col_capacity is too small.
  */
-int oracle_route(const uint16_t *Q, const uint16_t *K, int B, int H, int N, int d, int bs, double p,
-                 int32_t *row_ptr, int32_t *col_idx, int64_t col_capacity, int32_t *head_counts,
-                 double *diag, int nthreads) {
+int oracle_route_cand(const uint16_t *Q, const uint16_t *K, int B, int H, int N, int d, int bs, double p,
+                      int32_t *row_ptr, int32_t *col_idx, int64_t col_capacity, int32_t *head_counts,
+                      double *diag, int32_t *cand, double *cand_p, int kc, int nthreads) {
     if (!Q || !K || !row_ptr || !head_counts || B < 1 || H < 1 || N < 1 || d < 1 || bs < 1) return -1;
     if (!(p > 0.0) || p > 1.0) return -1;
     int64_t BH = (int64_t)B * H, nb = num_blocks(N, bs), rows = BH * nb;
@@ -259,7 +274,7 @@ int oracle_route(const uint16_t *Q, const uint16_t *K, int B, int H, int N, int 
     }
     oracle_pool(Q, BH, N, d, bs, qbar, nthreads);
     oracle_pool(K, BH, N, d, bs, kbar, nthreads);
-    route_ctx c = {qbar, kbar, d, nb, p, 1.0 / sqrt((double)d), counts, chosen, diag};
+    route_ctx c = {qbar, kbar, d, nb, p, 1.0 / sqrt((double)d), counts, chosen, diag, cand, cand_p, kc};
     parallel_for(rows, nthreads, route_range, &c);
     /* CSR: exclusive prefix sum of the row counts, columns ascending */
     int64_t total = 0;
@@ -288,6 +303,13 @@ done:
     free(counts);
     free(chosen);
     return rc;
+}
+
+int oracle_route(const uint16_t *Q, const uint16_t *K, int B, int H, int N, int d, int bs, double p,
+                 int32_t *row_ptr, int32_t *col_idx, int64_t col_capacity, int32_t *head_counts,
+                 double *diag, int nthreads) {
+    return oracle_route_cand(Q, K, B, H, N, d, bs, p, row_ptr, col_idx, col_capacity, head_counts, diag, NULL,
+                             NULL, 0, nthreads);
 }
 
 /* ------------------------------------------------- attention, row by row */
@@ -841,4 +863,159 @@ int oracle_quant_e4m3(const uint16_t *X, int64_t BH, int N, int d, int bs, uint8
         }
     }
     return 0;
+}
+
+/* ------------------------------------------------ head-major work order */
+
+typedef struct {
+    int64_t key; /* selected blocks */
+    int64_t id;
+} keyed_id;
+
+static int by_key_desc_id_asc(const void *a, const void *b) {
+    const keyed_id *x = (const keyed_id *)a, *y = (const keyed_id *)b;
+    if (x->key != y->key) return (x->key < y->key) - (x->key > y->key);
+    return (x->id > y->id) - (x->id < y->id);
+}
+
+/*
+ * The order the attention kernel takes its work items in ([FVAttn] §1 RLB:
+ * per-head work balanced at run time; here over the SMs of one GPU): heads by
+ * their total selected blocks (descending, equal totals by lower head), then the
+ * rows of each head by block count (descending, equal counts by lower row).
+ */
+int oracle_head_order(const int32_t *row_ptr, int64_t BH, int64_t nb, int32_t *order) {
+    if (!row_ptr || !order || BH < 1 || nb < 1) return -1;
+    keyed_id *h = (keyed_id *)malloc(sizeof(keyed_id) * BH);
+    keyed_id *r = (keyed_id *)malloc(sizeof(keyed_id) * nb);
+    if (!h || !r) {
+        free(h);
+        free(r);
+        return -1;
+    }
+    for (int64_t b = 0; b < BH; ++b) {
+        h[b].key = (int64_t)row_ptr[(b + 1) * nb] - row_ptr[b * nb];
+        h[b].id = b;
+    }
+    qsort(h, (size_t)BH, sizeof(keyed_id), by_key_desc_id_asc);
+    int64_t w = 0;
+    for (int64_t x = 0; x < BH; ++x) {
+        int64_t b = h[x].id;
+        for (int64_t i = 0; i < nb; ++i) {
+            r[i].key = (int64_t)row_ptr[b * nb + i + 1] - row_ptr[b * nb + i];
+            r[i].id = b * nb + i;
+        }
+        qsort(r, (size_t)nb, sizeof(keyed_id), by_key_desc_id_asc);
+        for (int64_t i = 0; i < nb; ++i) order[w++] = (int32_t)r[i].id;
+    }
+    free(h);
+    free(r);
+    return 0;
+}
+
+/* ------------------------------------------- slack-aware augmentation (SASA) */
+
+/*
+ * [FVAttn] §1 Key Terms (SASA) and §3: after the work has been balanced, the
+ * ranks that still have idle time (slack) before the slowest one finishes
+ * compute additional high-value key blocks, raising quality at no cost in time.
+ * On one GPU the ranks are the `machines` SMs of the persistent attention grid:
+ *   1. schedule: the rows, taken in the attention's queue order `order`, each go
+ *      to the machine with the least load so far (equal loads: the lowest
+ *      machine), a row's load being its selected-block count; the makespan T is
+ *      the largest load;
+ *   2. augmentation: each machine m, with slack T - load_m, walks its rows in
+ *      the order they were assigned, round after round, giving each row its next
+ *      candidate block (the rows' unselected blocks in routing order, at most kc
+ *      of them, cand[row, e] < 0 marks the end) at a cost of one block each,
+ *      until the slack is used up or no row of m has a candidate left;
+ *   3. the augmented mask: each row's selected blocks plus its added ones, in
+ *      ascending order.
+ * added[row] receives the number of blocks added, added_mass[row] their
+ * probability (the sum of cand_p over them, in the order added).
+ * Returns 0, -1 on bad arguments, -4 when col_capacity is too small.
+ */
+int oracle_sasa(const int32_t *row_ptr, const int32_t *col_idx, int64_t rows, const int32_t *cand,
+                const double *cand_p, int kc, const int32_t *order, int machines, int32_t *added,
+                double *added_mass, int32_t *row_ptr_out, int32_t *col_idx_out, int64_t col_capacity) {
+    if (!row_ptr || !col_idx || !cand || !order || !added || !row_ptr_out || machines < 1 || kc < 0 ||
+        rows < 0)
+        return -1;
+    int64_t *load = (int64_t *)calloc((size_t)machines, sizeof(int64_t));
+    int32_t *mach = (int32_t *)malloc(sizeof(int32_t) * (rows > 0 ? rows : 1));
+    int64_t *seq = (int64_t *)malloc(sizeof(int64_t) * (rows > 0 ? rows : 1)); /* rows in assignment order */
+    if (!load || !mach || !seq) {
+        free(load);
+        free(mach);
+        free(seq);
+        return -1;
+    }
+    /* 1. list schedule in queue order */
+    for (int64_t x = 0; x < rows; ++x) {
+        int64_t row = order[x];
+        int best = 0;
+        for (int m = 1; m < machines; ++m)
+            if (load[m] < load[best]) best = m;
+        mach[row] = best;
+        load[best] += (int64_t)row_ptr[row + 1] - row_ptr[row];
+        seq[x] = row;
+    }
+    int64_t T = 0;
+    for (int m = 0; m < machines; ++m)
+        if (load[m] > T) T = load[m];
+    /* 2. fill each machine's slack with its rows' next candidates, round robin */
+    for (int64_t row = 0; row < rows; ++row) {
+        added[row] = 0;
+        if (added_mass) added_mass[row] = 0.0;
+    }
+    for (int m = 0; m < machines; ++m) {
+        int64_t slack = T - load[m];
+        while (slack > 0) {
+            int progress = 0;
+            for (int64_t x = 0; x < rows && slack > 0; ++x) {
+                int64_t row = seq[x];
+                if (mach[row] != m) continue;
+                int e = added[row];
+                if (e < kc && cand[row * kc + e] >= 0) {
+                    if (added_mass) added_mass[row] = added_mass[row] + (cand_p ? cand_p[row * kc + e] : 0.0);
+                    added[row] = e + 1;
+                    --slack;
+                    progress = 1;
+                }
+            }
+            if (!progress) break;
+        }
+    }
+    /* 3. augmented CSR, columns ascending */
+    int64_t total = 0;
+    for (int64_t row = 0; row < rows; ++row) {
+        row_ptr_out[row] = (int32_t)total;
+        total += (int64_t)row_ptr[row + 1] - row_ptr[row] + added[row];
+    }
+    row_ptr_out[rows] = (int32_t)total;
+    int rc = 0;
+    if (total > col_capacity || !col_idx_out) {
+        rc = -4;
+    } else {
+        for (int64_t row = 0; row < rows; ++row) {
+            int32_t *dst = col_idx_out + row_ptr_out[row];
+            int64_t n = 0;
+            for (int32_t e = row_ptr[row]; e < row_ptr[row + 1]; ++e) dst[n++] = col_idx[e];
+            for (int e = 0; e < added[row]; ++e) dst[n++] = cand[row * kc + e];
+            /* insertion sort: the row is short and almost sorted */
+            for (int64_t a = 1; a < n; ++a) {
+                int32_t v = dst[a];
+                int64_t b = a - 1;
+                while (b >= 0 && dst[b] > v) {
+                    dst[b + 1] = dst[b];
+                    --b;
+                }
+                dst[b + 1] = v;
+            }
+        }
+    }
+    free(load);
+    free(mach);
+    free(seq);
+    return rc;
 }

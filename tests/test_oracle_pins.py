@@ -23,6 +23,7 @@ from fractions import Fraction
 import numpy as np
 import pytest
 
+import workloads as W
 from workloads import bf16_bits_to_f32, f32_to_bf16_bits
 
 getcontext().prec = 60
@@ -667,3 +668,122 @@ def test_e4m3_input_rounding_against_the_attention_tolerances(oracle_mod):
     err = np.abs(O1 - O0)
     assert err.max() < 2e-2 and err.mean() < 2e-3
     assert np.abs(L1 - L0).max() > 1e-3
+
+
+# ------------------------------------------------------------------ SASA (NEXT-1)
+# FVAttn review §1 Key Terms "SASA" and §3: after balancing, ranks with slack compute
+# extra high-value blocks.  One GPU: ranks = SMs of the persistent grid (reading in
+# oracle_sasa).  Pinned to closed forms, a hand-worked schedule and Graham's bound.
+
+def test_route_candidates_uniform_scores_closed_form(oracle_mod):
+    # K = 0: every score is 0, every probability 1/nb; the cut takes the first
+    # ceil(p * nb) blocks by index and the candidates are the next ones by index.
+    B, H, N, d, bs, p, kc = 1, 2, 640, 64, 64, 0.35, 8
+    nb = N // bs
+    rng = np.random.default_rng(3)
+    Q = W.f32_to_bf16_bits(rng.standard_normal((B, H, N, d)).astype(np.float32))
+    K = np.zeros_like(Q)
+    r, cand, cand_p = oracle_mod.route_candidates(Q, K, p, bs, kc)
+    keep = int(np.ceil(p * nb))
+    for row in range(B * H * nb):
+        assert list(r.col_idx[r.row_ptr[row]:r.row_ptr[row + 1]]) == list(range(keep))
+        want = list(range(keep, min(nb, keep + kc))) + [-1] * max(0, keep + kc - nb)
+        assert list(cand[row]) == want
+        assert np.allclose(cand_p[row][: nb - keep], 1.0 / nb, rtol=0, atol=1e-15)
+
+
+def test_route_candidates_are_the_best_unselected_blocks(oracle_mod):
+    w = W.Workload("cand", B=1, H=3, N=1500, d=64, bs=64, p=0.6, dist="structured", grid=(6, 10, 25),
+                   head_scale=("uniform", 0.5, 4.0), seed=7)
+    Q, K, _ = W.generate(w)
+    r, cand, cand_p = oracle_mod.route_candidates(Q, K, w.p, w.bs, 8)
+    r0 = oracle_mod.route(Q, K, w.p, w.bs)
+    assert np.array_equal(r.row_ptr, r0.row_ptr) and np.array_equal(r.col_idx, r0.col_idx)
+    for row in range(w.rows):
+        sel = set(r.col_idx[r.row_ptr[row]:r.row_ptr[row + 1]].tolist())
+        c = [x for x in cand[row].tolist() if x >= 0]
+        assert not sel.intersection(c) and len(set(c)) == len(c)
+        assert len(c) == min(8, w.nb - len(sel))
+        pr = cand_p[row][: len(c)]
+        # non-increasing, below the last kept probability, the first equals the first dropped one
+        assert np.all(np.diff(pr) <= 0) and (len(c) == 0 or pr[0] <= r.diag[row, 4])
+        assert len(c) == 0 or pr[0] == r.diag[row, 5]
+
+
+@pytest.mark.parametrize("BH,nb,seed", [(1, 5, 0), (3, 7, 1), (8, 16, 2)])
+def test_head_order_brute_force(oracle_mod, BH, nb, seed):
+    rng = np.random.default_rng(seed)
+    counts = rng.integers(0, 5, size=(BH, nb))
+    if BH > 2:
+        counts[2] = counts[0]
+    rp = np.zeros(BH * nb + 1, np.int32)
+    rp[1:] = np.cumsum(counts.reshape(-1))
+    heads = sorted(range(BH), key=lambda h: (-int(counts[h].sum()), h))
+    want = [h * nb + i for h in heads for i in sorted(range(nb), key=lambda i: (-int(counts[h, i]), i))]
+    assert list(oracle_mod.head_order(rp, BH, nb)) == want
+
+
+def _csr(counts):
+    rp = np.zeros(len(counts) + 1, np.int32)
+    rp[1:] = np.cumsum(counts)
+    ci = np.concatenate([np.arange(c, dtype=np.int32) * 2 for c in counts]) if sum(counts) else np.zeros(0, np.int32)
+    return rp, ci
+
+
+def test_sasa_hand_worked_schedule(oracle_mod):
+    # rows 0, 1, 2 with 3, 2, 2 blocks, queue order 0, 1, 2, two machines:
+    # row 0 -> m0 (load 3), row 1 -> m1 (2), row 2 -> m1 (4); makespan 4, slack m0 = 1, m1 = 0,
+    # so row 0 (the only row of m0) gets its first candidate.
+    rp, ci = _csr([3, 2, 2])
+    cand = np.array([[1, 3, -1], [1, 3, 5], [1, -1, -1]], np.int32)
+    cand_p = np.array([[0.2, 0.1, 0.0], [0.3, 0.2, 0.1], [0.4, 0.0, 0.0]])
+    s = oracle_mod.sasa(rp, ci, cand, cand_p, np.array([0, 1, 2], np.int32), 2)
+    assert list(s.added) == [1, 0, 0]
+    assert list(s.row_ptr) == [0, 4, 6, 8]
+    assert list(s.col_idx[:4]) == [0, 1, 2, 4]
+    assert s.added_mass[0] == 0.2 and s.added_mass[1] == 0.0
+    # round robin: rows of 6, 1 and 2 blocks in that order on two machines: row 0 -> m0 (6),
+    # row 1 -> m1 (1), row 2 -> m1 (3); m1's slack of 3 goes row 1, row 2, row 1
+    rp, ci = _csr([6, 1, 2])
+    cand = np.array([[-1] * 4, [1, 3, 5, 7], [1, 5, 7, 9]], np.int32)
+    s = oracle_mod.sasa(rp, ci, cand, np.zeros((3, 4)), np.array([0, 1, 2], np.int32), 2)
+    assert list(s.added) == [0, 2, 1]
+    # one machine: no slack, nothing added
+    s = oracle_mod.sasa(rp, ci, cand, np.zeros((3, 4)), np.array([0, 1, 2], np.int32), 1)
+    assert not s.added.any() and np.array_equal(s.row_ptr, rp) and np.array_equal(s.col_idx, ci)
+
+
+@pytest.mark.parametrize("rows,machines,kc,seed", [(40, 3, 4, 0), (200, 16, 8, 1), (1000, 148, 8, 2), (10, 30, 2, 3)])
+def test_sasa_schedule_and_augmentation_invariants(oracle_mod, rows, machines, kc, seed):
+    rng = np.random.default_rng(seed)
+    counts = rng.integers(1, 60, size=rows)
+    rp, ci = _csr(counts.tolist())
+    cand = np.full((rows, kc), -1, np.int32)
+    avail = rng.integers(0, kc + 1, size=rows)
+    for r in range(rows):
+        cand[r, : avail[r]] = 2 * counts[r] + 1 + 2 * np.arange(avail[r])   # odd: never among the selected
+    cand_p = rng.random((rows, kc))
+    order = np.argsort(-counts, kind="stable").astype(np.int32)
+    s = oracle_mod.sasa(rp, ci, cand, cand_p, order, machines)
+    # replay the schedule (least-loaded machine, lowest index on ties) to get per-machine loads
+    load = np.zeros(machines, np.int64)
+    mach = np.zeros(rows, np.int64)
+    for r in order:
+        m = int(np.argmin(load))
+        mach[r] = m
+        load[m] += counts[r]
+    T = load.max()
+    # Graham's list-scheduling bound
+    assert T <= counts.sum() / machines + counts.max()
+    for m in range(machines):
+        rs = np.nonzero(mach == m)[0]
+        extra = int(s.added[rs].sum())
+        assert load[m] + extra <= T
+        # the slack is used up unless every row of the machine ran out of candidates
+        assert load[m] + extra == T or all(s.added[r] == avail[r] for r in rs)
+    assert np.all(s.added <= avail)
+    for r in range(rows):
+        row = s.col_idx[s.row_ptr[r]:s.row_ptr[r + 1]]
+        want = sorted(list(ci[rp[r]:rp[r + 1]]) + list(cand[r, : s.added[r]]))
+        assert list(row) == want
+        assert s.added_mass[r] == pytest.approx(cand_p[r, : s.added[r]].sum(), abs=1e-15)
