@@ -339,6 +339,44 @@ FVATTN_API int fvattn_sparse_fwd_fp8(const void *Q8, const void *K8, const void 
                                      void *O, float *LSE, void *workspace, size_t ws_bytes, int32_t *dev_status,
                                      fvattn_stream_t stream);
 
+/* Device workspace fvattn_route_sasa needs, in bytes (0 on bad arguments). */
+FVATTN_API size_t fvattn_sasa_workspace_bytes(int B, int H, int N, int d, int block);
+
+/*
+ * fvattn_route_sasa -- top-p routing followed by slack-aware augmentation (FVAttn
+ * review, §1 Key Terms "SASA" and §3: after the work is balanced, the ranks that
+ * would idle before the slowest one finishes compute extra high-value key
+ * blocks).  On one GPU the ranks are the SMs of the persistent attention grid:
+ *   1. the routed rows, in the attention's queue order (fvattn_attn_work_order),
+ *      are list-scheduled onto `machines` machines: each row to the machine with
+ *      the least load so far, the lowest machine on equal loads, a row's load
+ *      being its selected-block count; the makespan T is the largest load;
+ *   2. each machine walks its rows in the order they were assigned, round after
+ *      round, giving each row its next unselected key block in the routing order
+ *      (score descending, index ascending; at most 8 per row), one block each,
+ *      until T - (its load) blocks are added or no row has a candidate left;
+ *   3. the augmented mask is written as a CSR with ascending columns.
+ * The output is a mask for fvattn_sparse_fwd (a superset of fvattn_route's).
+ *   machines      1..256; the attention kernel runs one CTA per SM, so the SM count
+ *                 of the device is the natural choice.
+ *   row_ptr, col_idx, col_capacity, head_counts   as fvattn_route, for the
+ *                 augmented mask (col_capacity >= routed blocks + 8 per row is
+ *                 always enough; B*H*ceil(N/block)^2 too).
+ *   added         device int32[rows] (out): blocks added to each row.
+ *   added_mass    device fp64[rows] (out), 8-byte aligned: their routing probability.
+ *   cand, cand_p  optional (null: not written) device int32 / fp64 [rows, 8] (out):
+ *                 the routing candidates of every row (the key blocks past the cut
+ *                 in the routing order, -1 past the last) and their probabilities.
+ *   workspace     fvattn_sasa_workspace_bytes(B,H,N,d,block) bytes, 16-byte aligned.
+ * Other arguments and errors as fvattn_route; machines outside 1..256 give
+ * FVATTN_ERR_UNSUPPORTED.  Asynchronous on `stream`.
+ */
+FVATTN_API int fvattn_route_sasa(const void *Q, const void *K, int B, int H, int N, int d, int block, double p,
+                                 int machines, int32_t *row_ptr, int32_t *col_idx, int64_t col_capacity,
+                                 int32_t *head_counts, int32_t *added, double *added_mass, int32_t *cand,
+                                 double *cand_p, void *workspace, size_t ws_bytes, int32_t *dev_status,
+                                 fvattn_stream_t stream);
+
 /*
  * fvattn_attn_work_order -- the order in which fvattn_sparse_fwd takes its work
  * items (CSR rows, one query block of one head each), written to order[0 .. rows)

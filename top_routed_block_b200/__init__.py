@@ -78,6 +78,8 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         "fvattn_test_sparse_fwd_stall": (I, [P, P, P, P, P, I, I, I, I, I, I, P, P, P, SZ, P, P]),
         "fvattn_sparse_fwd_profiled": (I, [P, P, P, P, P, I, I, I, I, I, I, P, P, P, SZ, P, I, P, P, P]),
         "fvattn_attn_work_order": (I, [P, I, I, I, I, P, P, SZ, P]),
+        "fvattn_sasa_workspace_bytes": (SZ, [I, I, I, I, I]),
+        "fvattn_route_sasa": (I, [P, P, I, I, I, I, I, D, I, P, P, I64, P, P, P, P, P, P, SZ, P, P]),
         "fvattn_sparse_fwd_fp8": (I, [P, P, P, P, P, P, P, P, I, I, I, I, I, I, P, P, P, SZ, P, P]),
         "fvattn_bwd_workspace_bytes": (SZ, [I, I, I, I]),
         "fvattn_sparse_bwd": (I, [P, P, P, P, P, P, P, P, I, I, I, I, I, I, P, P, P, P, SZ, P, P]),
@@ -293,6 +295,47 @@ def fvattn_sparse_fwd_fp8(Q8: torch.Tensor, K8: torch.Tensor, V8: torch.Tensor, 
                                    _ptr(workspace), workspace.numel(), _ptr(dev_status), _stream_ptr(stream))
     _check(rc, "fvattn_sparse_fwd_fp8")
     return O, LSE, dev_status
+
+
+class SasaResult:
+    """Augmented CSR mask, per-head block counts, and per row the number and routing
+    probability of the blocks added."""
+
+    def __init__(self, row_ptr, col_idx, head_counts, added, added_mass, dev_status):
+        self.row_ptr, self.col_idx, self.head_counts = row_ptr, col_idx, head_counts
+        self.added, self.added_mass, self.dev_status = added, added_mass, dev_status
+
+
+def fvattn_route_sasa(Q: torch.Tensor, K: torch.Tensor, p: float, block: int, machines: int | None = None, *,
+                      stream=None, out: SasaResult | None = None, workspace: torch.Tensor | None = None,
+                      candidates: bool = False) -> SasaResult:
+    """Top-p routing plus slack-aware augmentation over `machines` SMs (default: the
+    device's SM count).  With ``candidates``, the result also carries the routing
+    candidates (``cand`` int32 and ``cand_p`` fp64, [rows, 8])."""
+    lib = load_library()
+    B, H, N, d = _shape(Q)
+    dev = Q.device
+    if machines is None:
+        machines = torch.cuda.get_device_properties(dev).multi_processor_count
+    rows = fvattn_num_rows(B, H, N, block)
+    if out is None:
+        cap = fvattn_route_max_nnz(B, H, N, block)
+        out = SasaResult(torch.empty(rows + 1, dtype=torch.int32, device=dev),
+                         torch.empty(max(cap, 1), dtype=torch.int32, device=dev),
+                         torch.empty(B * H, dtype=torch.int32, device=dev),
+                         torch.empty(rows, dtype=torch.int32, device=dev),
+                         torch.empty(rows, dtype=torch.float64, device=dev),
+                         torch.zeros(1, dtype=torch.int32, device=dev))
+    out.cand = torch.empty((rows, 8), dtype=torch.int32, device=dev) if candidates else None
+    out.cand_p = torch.empty((rows, 8), dtype=torch.float64, device=dev) if candidates else None
+    if workspace is None:
+        workspace = _empty_bytes(int(lib.fvattn_sasa_workspace_bytes(B, H, N, d, block)), dev)
+    rc = lib.fvattn_route_sasa(_ptr(Q), _ptr(K), B, H, N, d, block, float(p), int(machines), _ptr(out.row_ptr),
+                               _ptr(out.col_idx), out.col_idx.numel(), _ptr(out.head_counts), _ptr(out.added),
+                               _ptr(out.added_mass), _ptr(out.cand), _ptr(out.cand_p), _ptr(workspace),
+                               workspace.numel(), _ptr(out.dev_status), _stream_ptr(stream))
+    _check(rc, "fvattn_route_sasa")
+    return out
 
 
 def fvattn_attn_work_order(row_ptr: torch.Tensor, B: int, H: int, N: int, block: int, *, stream=None,

@@ -17,6 +17,7 @@
 #include "lpt.cuh"
 #include "quant.cuh"
 #include "route.cuh"
+#include "sasa.cuh"
 
 using namespace fvattn;
 
@@ -381,6 +382,87 @@ int fvattn_attn_work_order(const int32_t *row_ptr, int B, int H, int N, int bloc
     int32_t *head_rank = reinterpret_cast<int32_t *>(static_cast<char *>(workspace) + w.head_rank);
     return from_cuda(launch_item_order(row_ptr, BH, static_cast<int>(nb), head_rank, order,
                                        reinterpret_cast<cudaStream_t>(stream)));
+}
+
+namespace {
+struct SasaWorkspace {
+    size_t route, row_ptr, col_idx, head_counts, cand, cand_p, order, head_rank, mach, lists, list_off, counts, total;
+};
+SasaWorkspace sasa_layout(int64_t BH, int nb, int d) {
+    SasaWorkspace w{};
+    Carver c;
+    const int64_t rows = BH * nb;
+    w.route = c.take<char>(route_workspace_layout(BH, nb, d).total);
+    w.row_ptr = c.take<int32_t>(static_cast<size_t>(rows) + 1);
+    w.col_idx = c.take<int32_t>(static_cast<size_t>(rows) * nb);
+    w.head_counts = c.take<int32_t>(static_cast<size_t>(BH));
+    w.cand = c.take<int32_t>(static_cast<size_t>(rows) * kSasaCandidates);
+    w.cand_p = c.take<double>(static_cast<size_t>(rows) * kSasaCandidates);
+    w.order = c.take<int32_t>(static_cast<size_t>(rows));
+    w.head_rank = c.take<int32_t>(static_cast<size_t>(BH));
+    w.mach = c.take<uint8_t>(static_cast<size_t>(rows));
+    w.lists = c.take<int32_t>(static_cast<size_t>(rows));
+    w.list_off = c.take<int32_t>(kSasaMaxMachines + 1);
+    w.counts = c.take<int32_t>(static_cast<size_t>(rows));
+    w.total = align_up(c.off, 256);
+    return w;
+}
+}  // namespace
+
+size_t fvattn_sasa_workspace_bytes(int B, int H, int N, int d, int block) {
+    if (check_shape(B, H, N, d, block) != FVATTN_OK) return 0;
+    const int64_t nb = ceil_div(N, block);
+    const int64_t BH = static_cast<int64_t>(B) * H;
+    if (nb > kMaxRouteBlocks || BH > kMaxHeads) return 0;
+    return sasa_layout(BH, static_cast<int>(nb), d).total;
+}
+
+int fvattn_route_sasa(const void *Q, const void *K, int B, int H, int N, int d, int block, double p, int machines,
+                      int32_t *row_ptr, int32_t *col_idx, int64_t col_capacity, int32_t *head_counts,
+                      int32_t *added, double *added_mass, int32_t *cand, double *cand_p, void *workspace,
+                      size_t ws_bytes, int32_t *dev_status, fvattn_stream_t stream) {
+    int rc = check_shape(B, H, N, d, block);
+    if (rc != FVATTN_OK) return rc;
+    if (machines < 1 || machines > kSasaMaxMachines) return FVATTN_ERR_UNSUPPORTED;
+    if (!Q || !K || !row_ptr || !col_idx || !head_counts || !added || !added_mass || !workspace || !dev_status)
+        return FVATTN_ERR_INVALID_ARG;
+    if (!(p > 0.0) || p > 1.0 || std::isnan(p) || col_capacity < 0) return FVATTN_ERR_INVALID_ARG;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(workspace)) return FVATTN_ERR_ALIGNMENT;
+    if ((reinterpret_cast<uintptr_t>(row_ptr) | reinterpret_cast<uintptr_t>(col_idx) |
+         reinterpret_cast<uintptr_t>(head_counts) | reinterpret_cast<uintptr_t>(added) |
+         reinterpret_cast<uintptr_t>(dev_status) | reinterpret_cast<uintptr_t>(cand)) & 3u ||
+        ((reinterpret_cast<uintptr_t>(added_mass) | reinterpret_cast<uintptr_t>(cand_p)) & 7u))
+        return FVATTN_ERR_ALIGNMENT;
+    const int nb = static_cast<int>(ceil_div(N, block));
+    const int64_t BH = static_cast<int64_t>(B) * H;
+    if (nb > kMaxRouteBlocks || BH > kMaxHeads) return FVATTN_ERR_UNSUPPORTED;
+    if (ws_bytes < fvattn_sasa_workspace_bytes(B, H, N, d, block)) return FVATTN_ERR_CAPACITY;
+    if ((rc = check_device()) != FVATTN_OK) return rc;
+    const SasaWorkspace w = sasa_layout(BH, nb, d);
+    char *ws = static_cast<char *>(workspace);
+    auto i32 = [&](size_t off) { return reinterpret_cast<int32_t *>(ws + off); };
+    const int64_t rows = BH * nb;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if ((rc = from_cuda(cudaMemsetAsync(dev_status, 0, sizeof(int32_t), s))) != FVATTN_OK) return rc;
+    // the routed mask and its candidates, the attention's queue order, then the plan
+    rc = from_cuda(launch_route(Q, K, BH, N, d, block, nb, p, i32(w.row_ptr), i32(w.col_idx), rows * nb,
+                                i32(w.head_counts), ws + w.route, dev_status, s, i32(w.cand),
+                                reinterpret_cast<double *>(ws + w.cand_p)));
+    if (rc != FVATTN_OK) return rc;
+    if ((rc = from_cuda(launch_item_order(i32(w.row_ptr), BH, nb, i32(w.head_rank), i32(w.order), s))) != FVATTN_OK)
+        return rc;
+    rc = from_cuda(launch_sasa(i32(w.row_ptr), i32(w.col_idx), i32(w.order), rows, nb, BH, machines, i32(w.cand),
+                               reinterpret_cast<const double *>(ws + w.cand_p),
+                               reinterpret_cast<uint8_t *>(ws + w.mach), i32(w.lists),
+                               i32(w.list_off), i32(w.counts), added, added_mass, row_ptr, col_idx, col_capacity,
+                               head_counts, dev_status, s));
+    if (rc == FVATTN_OK && cand)
+        rc = from_cuda(cudaMemcpyAsync(cand, ws + w.cand, sizeof(int32_t) * rows * kSasaCandidates,
+                                       cudaMemcpyDeviceToDevice, s));
+    if (rc == FVATTN_OK && cand_p)
+        rc = from_cuda(cudaMemcpyAsync(cand_p, ws + w.cand_p, sizeof(double) * rows * kSasaCandidates,
+                                       cudaMemcpyDeviceToDevice, s));
+    return rc;
 }
 
 size_t fvattn_bwd_workspace_bytes(int B, int H, int N, int block) {

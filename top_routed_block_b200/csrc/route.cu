@@ -19,6 +19,9 @@
 //                         registers, prefix sum to p, a row bitmap.
 //   csr_scan_kernel       row_ptr = exclusive scan of the row counts; head counts.
 //   csr_scatter_kernel    col_idx from the row bitmaps, ascending.
+// With candidate outputs (the slack-aware augmentation of sasa.cu), the select
+// kernel also writes, per row, the kSasaCandidates key blocks that follow the cut
+// in the routing order and their probabilities.
 #include <cstdint>
 #include <math_constants.h>
 
@@ -122,7 +125,8 @@ template <int D, int MJ, int EPL>
 __global__ void __launch_bounds__(kSelThreads) route_select_kernel(const double *__restrict__ qbar,
                                                                    const double *__restrict__ kbarT, int nb, double p,
                                                                    double scale, int32_t *__restrict__ counts,
-                                                                   uint32_t *__restrict__ bitmap, int W) {
+                                                                   uint32_t *__restrict__ bitmap, int W,
+                                                                   int32_t *__restrict__ cand, double *__restrict__ cand_p) {
     constexpr int NP2 = 32 * EPL;
     extern __shared__ __align__(16) unsigned char smem_raw[];
     double *sq = reinterpret_cast<double *>(smem_raw);                 // [kSelRows][D] query means
@@ -175,6 +179,11 @@ __global__ void __launch_bounds__(kSelThreads) route_select_kernel(const double 
     uint32_t *bmw = bm + warp * 32;
     const int64_t row = bh * nb + i0 + warp;
     int count;
+    if (cand && lane < kSasaCandidates) {  // no candidate unless written below
+        cand[row * kSasaCandidates + lane] = -1;
+        cand_p[row * kSasaCandidates + lane] = 0.0;
+    }
+    __syncwarp();
     if (p >= 1.0) {
         count = nb;
         if (lane < W) {
@@ -281,6 +290,16 @@ __global__ void __launch_bounds__(kSelThreads) route_select_kernel(const double 
 #pragma unroll
         for (int q = 0; q < EPL; ++q)
             if (lane * EPL + q <= kcut) atomicOr(&bmw[idx[q] >> 5], 1u << (idx[q] & 31));
+        if (cand) {  // the blocks right after the cut, in routing order
+#pragma unroll
+            for (int q = 0; q < EPL; ++q) {
+                const int e = lane * EPL + q - kcut - 1;
+                if (e >= 0 && e < kSasaCandidates && idx[q] < nb) {
+                    cand[row * kSasaCandidates + e] = idx[q];
+                    cand_p[row * kSasaCandidates + e] = s[idx[q]];
+                }
+            }
+        }
     }
     __syncwarp();
     if (lane < W) bitmap[row * W + lane] = bmw[lane];
@@ -387,6 +406,8 @@ struct SelectArgs {
     uint32_t *bitmap;
     int W;
     int64_t BH;
+    int32_t *cand;
+    double *cand_p;
 };
 
 template <int D, int MJ, int EPL>
@@ -397,7 +418,7 @@ cudaError_t launch_select(const SelectArgs &a, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     const dim3 grid(static_cast<unsigned>(ceil_div(a.nb, kSelRows)), static_cast<unsigned>(a.BH));
     route_select_kernel<D, MJ, EPL><<<grid, kSelThreads, smem, stream>>>(a.qbar, a.kbarT, a.nb, a.p, a.scale,
-                                                                         a.counts, a.bitmap, a.W);
+                                                                         a.counts, a.bitmap, a.W, a.cand, a.cand_p);
     return cudaGetLastError();
 }
 
@@ -415,6 +436,13 @@ cudaError_t dispatch_select(const SelectArgs &a, cudaStream_t stream) {
 
 }  // namespace
 
+cudaError_t launch_csr_scan(const int32_t *counts, int64_t rows, int nb, int64_t BH, int32_t *row_ptr,
+                            int64_t capacity, int32_t *head_counts, int32_t *dev_status, cudaStream_t stream) {
+    csr_scan_kernel<<<1, kScanThreads, 0, stream>>>(counts, rows, nb, BH, row_ptr, capacity, head_counts,
+                                                    dev_status);
+    return cudaGetLastError();
+}
+
 RouteWorkspace route_workspace_layout(int64_t BH, int nb, int d) {
     RouteWorkspace w{};
     Carver c;
@@ -430,7 +458,7 @@ RouteWorkspace route_workspace_layout(int64_t BH, int nb, int d) {
 
 cudaError_t launch_route(const void *Q, const void *K, int64_t BH, int N, int d, int bs, int nb, double p,
                          int32_t *row_ptr, int32_t *col_idx, int64_t capacity, int32_t *head_counts,
-                         void *workspace, int32_t *dev_status, cudaStream_t stream) {
+                         void *workspace, int32_t *dev_status, cudaStream_t stream, int32_t *cand, double *cand_p) {
     const RouteWorkspace w = route_workspace_layout(BH, nb, d);
     char *ws = static_cast<char *>(workspace);
     double *qbar = reinterpret_cast<double *>(ws + w.qbar);
@@ -439,7 +467,7 @@ cudaError_t launch_route(const void *Q, const void *K, int64_t BH, int N, int d,
     uint32_t *bitmap = reinterpret_cast<uint32_t *>(ws + w.bitmap);
     const int64_t rows = BH * nb;
     const double scale = 1.0 / sqrt(static_cast<double>(d));
-    const SelectArgs sel{qbar, kbarT, nb, p, scale, counts, bitmap, w.W, BH};
+    const SelectArgs sel{qbar, kbarT, nb, p, scale, counts, bitmap, w.W, BH, cand, cand_p};
     const auto *q16 = static_cast<const uint16_t *>(Q);
     const auto *k16 = static_cast<const uint16_t *>(K);
     cudaError_t e;
@@ -453,8 +481,8 @@ cudaError_t launch_route(const void *Q, const void *K, int64_t BH, int N, int d,
         e = dispatch_select<64>(sel, stream);
     }
     if (e != cudaSuccess) return e;
-    csr_scan_kernel<<<1, kScanThreads, 0, stream>>>(counts, rows, nb, BH, row_ptr, capacity, head_counts,
-                                                    dev_status);
+    e = launch_csr_scan(counts, rows, nb, BH, row_ptr, capacity, head_counts, dev_status, stream);
+    if (e != cudaSuccess) return e;
     csr_scatter_kernel<<<static_cast<unsigned>(ceil_div(rows, 8)), 256, 0, stream>>>(bitmap, row_ptr, rows, w.W,
                                                                                      col_idx, capacity);
     return cudaGetLastError();
