@@ -51,6 +51,7 @@ def _load():
         lib.oracle_route_cand.argtypes = [P, P, i32, i32, i32, i32, i32, dbl, P, P, i64, P, P, P, P, i32, i32]
         lib.oracle_head_order.argtypes = [P, i64, i64, P]
         lib.oracle_sasa.argtypes = [P, P, i64, P, P, i32, P, i32, P, P, P, P, i64]
+        lib.oracle_rlb_plan.argtypes = [P, i32, i32, i32, P, P, P, P]
         lib.oracle_attn_bwd.argtypes = [P, P, P, P, i32, i32, i32, i32, i32, i32, P, P, P, P, P, i32]
         lib.oracle_attn_bwd_sampled.argtypes = [P, P, P, P, i32, i32, i32, i32, i32, i32, P, P, P, i64, P, P, P,
                                                 i64, P, P, i32]
@@ -61,7 +62,7 @@ def _load():
         lib.oracle_e4m3_from_double.restype = ctypes.c_uint8
         for f in ("oracle_pool", "oracle_route", "oracle_attn_rows", "oracle_attn_tiled", "oracle_lpt_order",
                   "oracle_attn_bwd", "oracle_attn_bwd_sampled", "oracle_quant_e4m3", "oracle_route_cand",
-                  "oracle_head_order", "oracle_sasa"):
+                  "oracle_head_order", "oracle_sasa", "oracle_rlb_plan"):
             getattr(lib, f).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -303,6 +304,21 @@ def sasa(row_ptr, col_idx, cand, cand_p, order, machines: int) -> Sasa:
     if rc != 0:
         raise ValueError(f"oracle_sasa failed ({rc})")
     return Sasa(rp, ci[: rp[-1]].copy(), added[:rows], mass[:rows])
+
+
+def rlb_plan(work: np.ndarray, max_moves: int | None = None):
+    """Head moves balancing per-rank work (work: int [ranks, units]); returns the
+    moves as an int32 array [n, 3] of (home unit r*units+i, source rank, destination)."""
+    work = np.ascontiguousarray(work, dtype=np.int64)
+    ranks, units = work.shape
+    cap = ranks * units * 4 if max_moves is None else max_moves
+    mu = np.empty(max(cap, 1), np.int32)
+    ms = np.empty(max(cap, 1), np.int32)
+    md = np.empty(max(cap, 1), np.int32)
+    n = ctypes.c_int32(0)
+    if _load().oracle_rlb_plan(_ptr(work), ranks, units, cap, _ptr(mu), _ptr(ms), _ptr(md), ctypes.byref(n)) != 0:
+        raise ValueError("oracle_rlb_plan failed")
+    return np.stack([mu[: n.value], ms[: n.value], md[: n.value]], axis=1)
 
 
 def lpt_order(row_ptr: np.ndarray) -> np.ndarray:

@@ -48,6 +48,9 @@
  *               exhaustive comparison with the selected set's complement
  *   sasa        Graham's list-scheduling bound, loads within the makespan,
  *               slack used up unless candidates run out, hand-worked examples
+ *   rlb_plan    hand-worked plans, every move lowers the sum of squared loads,
+ *               the final state admits no improving move, exhaustive optimum
+ *               never beaten on tiny instances
  *   e4m3 / quant_e4m3  the format's own values (known codes, ties to even,
  *               saturation, NaN), round trip of every finite code, monotone
  *               encoding, block scales putting the block maximum in (224, 448],
@@ -1018,4 +1021,62 @@ int oracle_sasa(const int32_t *row_ptr, const int32_t *col_idx, int64_t rows, co
     free(mach);
     free(seq);
     return rc;
+}
+
+/* ------------------------------------------ run-time load balancing (RLB) */
+
+/*
+ * [FVAttn] §1 Key Terms (RLB) and §3: once routing has fixed every head's amount
+ * of work, heads move between GPUs (P2P) so that the critical path shortens.
+ * Units are (batch, head) pairs; work[r * units + i] is the selected-block count
+ * of unit i of rank r (units per rank, all ranks alike).  The plan, step by step:
+ * the most loaded rank (lowest index on ties) gives the least loaded rank
+ * (lowest index on ties) the unit it holds with the largest work below their gap
+ * (among equal works the unit with the lowest home index r * units + i), as long
+ * as such a unit exists (the move then lowers both loads below the old maximum).
+ * A unit may move again later.  Writes the moves in
+ * order: move_unit[k] = r * units + i (the unit's home), move_src[k], move_dst[k];
+ * *n_moves their number (at most max_moves).  Returns 0, -1 on bad arguments.
+ */
+int oracle_rlb_plan(const int64_t *work, int ranks, int units, int max_moves, int32_t *move_unit, int32_t *move_src,
+                    int32_t *move_dst, int32_t *n_moves) {
+    if (!work || ranks < 1 || units < 0 || max_moves < 0 || !n_moves) return -1;
+    int64_t total = (int64_t)ranks * units;
+    int32_t *owner = (int32_t *)malloc(sizeof(int32_t) * (total > 0 ? total : 1));
+    int64_t *load = (int64_t *)calloc((size_t)ranks, sizeof(int64_t));
+    if (!owner || !load) {
+        free(owner);
+        free(load);
+        return -1;
+    }
+    for (int64_t u = 0; u < total; ++u) {
+        owner[u] = (int32_t)(u / units);
+        load[u / units] += work[u];
+    }
+    int k = 0;
+    while (k < max_moves) {
+        int src = 0, dst = 0;
+        for (int r = 1; r < ranks; ++r) {
+            if (load[r] > load[src]) src = r;
+            if (load[r] < load[dst]) dst = r;
+        }
+        int64_t gap = load[src] - load[dst];
+        int64_t best = -1;
+        for (int64_t u = 0; u < total; ++u) {
+            if (owner[u] != src || work[u] <= 0 || work[u] >= gap) continue;
+            if (best < 0 || work[u] > work[best]) best = u;
+        }
+        if (best < 0) break;
+        owner[best] = dst;
+        load[src] -= work[best];
+        load[dst] += work[best];
+        if (move_unit) move_unit[k] = (int32_t)best;
+        if (move_src) move_src[k] = src;
+        if (move_dst) move_dst[k] = dst;
+        ++k;
+    }
+    *n_moves = k;
+    free(owner);
+    free(load);
+    return 0;
 }

@@ -787,3 +787,64 @@ def test_sasa_schedule_and_augmentation_invariants(oracle_mod, rows, machines, k
         want = sorted(list(ci[rp[r]:rp[r + 1]]) + list(cand[r, : s.added[r]]))
         assert list(row) == want
         assert s.added_mass[r] == pytest.approx(cand_p[r, : s.added[r]].sum(), abs=1e-15)
+
+
+# ------------------------------------------------------------------ RLB (NEXT-2)
+# FVAttn review §1 Key Terms "RLB" and §3: heads move between GPUs once their work is
+# known.  Pinned to hand-worked plans, the sum-of-squares descent every move makes, the
+# absence of an improving move at the end, and an exhaustive optimum on tiny instances.
+
+def _rlb_apply(work, moves):
+    ranks, units = work.shape
+    owner = np.repeat(np.arange(ranks), units)
+    loads = work.sum(1).astype(np.int64)
+    flat = work.reshape(-1)
+    ss = [int((loads ** 2).sum())]
+    for u, s, d in moves:
+        assert owner[u] == s and s != d
+        owner[u] = d
+        loads[s] -= flat[u]
+        loads[d] += flat[u]
+        ss.append(int((loads ** 2).sum()))
+    return owner, loads, ss
+
+
+def test_rlb_hand_worked(oracle_mod):
+    assert oracle_mod.rlb_plan(np.array([[10, 1], [1, 1]])).tolist() == [[1, 0, 1]]
+    # loads 10 / 0: both 5s are below the gap; the lower home index moves, then the loads are equal
+    assert oracle_mod.rlb_plan(np.array([[5, 5], [0, 0]])).tolist() == [[0, 0, 1]]
+    assert oracle_mod.rlb_plan(np.array([[3, 4], [4, 3]])).size == 0          # already balanced
+    assert oracle_mod.rlb_plan(np.array([[7, 9, 1]])).size == 0               # one rank
+    # three ranks: 12 / 2 / 1 -> rank 0 gives 4 to rank 2 (gap 11) and 4 to rank 1 (gap 6): 4 / 6 / 5;
+    # then rank 1 gives its home unit 0 (work 1, below the gap 2) to rank 0: 5 / 5 / 5
+    moves = oracle_mod.rlb_plan(np.array([[4, 4, 4], [1, 1, 0], [1, 0, 0]]))
+    _, loads, _ = _rlb_apply(np.array([[4, 4, 4], [1, 1, 0], [1, 0, 0]]), moves)
+    assert moves.tolist() == [[0, 0, 2], [1, 0, 1], [3, 1, 0]] and loads.tolist() == [5, 5, 5]
+
+
+@pytest.mark.parametrize("ranks,units,seed", [(2, 4, 0), (3, 8, 1), (8, 5, 2), (8, 40, 3), (4, 1, 4)])
+def test_rlb_invariants(oracle_mod, ranks, units, seed):
+    rng = np.random.default_rng(seed)
+    work = rng.integers(0, 200, size=(ranks, units)) * (rng.random((ranks, 1)) * 3 + 0.2)
+    work = work.astype(np.int64)
+    moves = oracle_mod.rlb_plan(work)
+    owner, loads, ss = _rlb_apply(work, moves)
+    assert all(b < a for a, b in zip(ss, ss[1:]))               # every move lowers the sum of squares
+    assert loads.max() <= work.sum(1).max()
+    src, dst = int(np.argmax(loads)), int(np.argmin(loads))
+    gap = loads[src] - loads[dst]
+    flat = work.reshape(-1)
+    assert not any(owner[u] == src and 0 < flat[u] < gap for u in range(flat.size))
+
+
+def test_rlb_close_to_exhaustive_optimum_on_tiny_instances(oracle_mod):
+    import itertools as it
+    rng = np.random.default_rng(9)
+    for _ in range(40):
+        ranks, units = int(rng.integers(2, 4)), int(rng.integers(1, 4))
+        work = rng.integers(0, 30, size=(ranks, units)).astype(np.int64)
+        flat = work.reshape(-1)
+        best = min(max(sum(int(flat[u]) for u in range(flat.size) if a[u] == r) for r in range(ranks))
+                   for a in it.product(range(ranks), repeat=flat.size))
+        _, loads, _ = _rlb_apply(work, oracle_mod.rlb_plan(work))
+        assert best <= loads.max() <= best + flat.max()
