@@ -378,6 +378,26 @@ FVATTN_API int fvattn_route_sasa(const void *Q, const void *K, int B, int H, int
                                  fvattn_stream_t stream);
 
 /*
+ * fvattn_rlb_plan -- the head moves of run-time load balancing across ranks
+ * (FVAttn review, §1 Key Terms "RLB" and §3: once routing has fixed every head's
+ * amount of work, heads move between GPUs over P2P so the critical path shortens).
+ * Host code; no device work.
+ *   work       host int64[ranks * units]: work[r * units + i] = selected blocks of
+ *              unit i (a (batch, head) pair) that rank r holds; >= 0.
+ *   moves out  move_unit[k] = the unit's home index r * units + i, move_src[k] and
+ *              move_dst[k] its ranks, for k < *n_moves, in the order decided.
+ * Rule: while the most loaded rank holds a unit whose work lies strictly between 0
+ * and its gap to the least loaded rank, it hands the largest such unit (the lowest
+ * home index among equal works) to that rank; ranks tie by lower index.  Every
+ * move lowers the sum of squared loads, so the plan ends; a unit may move again.
+ * Errors: FVATTN_ERR_INVALID_ARG on null pointers or negative sizes or work;
+ * FVATTN_ERR_CAPACITY when the plan needs more than max_moves moves (the first
+ * max_moves are written).
+ */
+FVATTN_API int fvattn_rlb_plan(const int64_t *work, int ranks, int units, int max_moves, int32_t *move_unit,
+                               int32_t *move_src, int32_t *move_dst, int32_t *n_moves);
+
+/*
  * fvattn_attn_work_order -- the order in which fvattn_sparse_fwd takes its work
  * items (CSR rows, one query block of one head each), written to order[0 .. rows)
  * with rows = B*H*ceil(N/block).  FVAttn review §1 "RLB" balances per-head work at

@@ -123,3 +123,20 @@ def test_noalloc_rejects_shapes_beyond_its_scratch_without_a_gpu(lib):
     B, H, N, block = 16, 256, 65536, 128
     assert lib.fvattn_sparse_fwd_noalloc(None, None, None, None, None, B, H, N, 128, block, 0, None, None, None,
                                          None) == -4
+
+
+def test_rlb_plan_matches_the_oracle(lib, oracle_mod):
+    # host-only entry point: the library's plan equals the oracle's on random instances
+    import numpy as np
+    import top_routed_block_b200 as fv
+    rng = np.random.default_rng(11)
+    for ranks, units in [(1, 3), (2, 4), (3, 7), (8, 5), (8, 40), (16, 3)]:
+        for _ in range(5):
+            work = (rng.integers(0, 300, size=(ranks, units)) * (rng.random((ranks, 1)) * 3)).astype(np.int64)
+            want = oracle_mod.rlb_plan(work).tolist()
+            assert [list(m) for m in fv.fvattn_rlb_plan(work)] == want
+    assert fv.fvattn_rlb_plan(np.array([[3, 4], [4, 3]])) == []
+    with pytest.raises(fv.FvattnError):
+        fv.fvattn_rlb_plan(np.array([[1, -1]]))
+    with pytest.raises(fv.FvattnError):
+        fv.fvattn_rlb_plan(np.array([[4, 4, 4], [1, 1, 0], [1, 0, 0]]), max_moves=1)   # needs 3 moves

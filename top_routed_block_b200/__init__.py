@@ -79,6 +79,7 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         "fvattn_sparse_fwd_profiled": (I, [P, P, P, P, P, I, I, I, I, I, I, P, P, P, SZ, P, I, P, P, P]),
         "fvattn_attn_work_order": (I, [P, I, I, I, I, P, P, SZ, P]),
         "fvattn_sasa_workspace_bytes": (SZ, [I, I, I, I, I]),
+        "fvattn_rlb_plan": (I, [P, I, I, I, P, P, P, P]),
         "fvattn_route_sasa": (I, [P, P, I, I, I, I, I, D, I, P, P, I64, P, P, P, P, P, P, SZ, P, P]),
         "fvattn_sparse_fwd_fp8": (I, [P, P, P, P, P, P, P, P, I, I, I, I, I, I, P, P, P, SZ, P, P]),
         "fvattn_bwd_workspace_bytes": (SZ, [I, I, I, I]),
@@ -295,6 +296,23 @@ def fvattn_sparse_fwd_fp8(Q8: torch.Tensor, K8: torch.Tensor, V8: torch.Tensor, 
                                    _ptr(workspace), workspace.numel(), _ptr(dev_status), _stream_ptr(stream))
     _check(rc, "fvattn_sparse_fwd_fp8")
     return O, LSE, dev_status
+
+
+def fvattn_rlb_plan(work, max_moves: int | None = None):
+    """Run-time load balancing moves for per-rank unit work (int [ranks, units], host):
+    returns a list of (home unit index, source rank, destination rank)."""
+    import numpy as np
+    w = np.ascontiguousarray(np.asarray(work), dtype=np.int64)
+    ranks, units = (int(x) for x in w.shape)
+    cap = 4 * ranks * units + 16 if max_moves is None else int(max_moves)
+    mu = np.empty(max(cap, 1), np.int32)
+    ms = np.empty(max(cap, 1), np.int32)
+    md = np.empty(max(cap, 1), np.int32)
+    n = ctypes.c_int32(0)
+    rc = load_library().fvattn_rlb_plan(w.ctypes.data, ranks, units, cap, mu.ctypes.data, ms.ctypes.data,
+                                        md.ctypes.data, ctypes.byref(n))
+    _check(rc, "fvattn_rlb_plan")
+    return [(int(mu[k]), int(ms[k]), int(md[k])) for k in range(n.value)]
 
 
 class SasaResult:
