@@ -177,13 +177,18 @@ FVATTN_API int fvattn_quant_e4m3(const void *X, int B, int H, int N, int d, int 
  *   O           out, bf16 [B,H,N,d].   LSE  out, fp32 [B,H,N].
  *   workspace   >= fvattn_fwd_workspace_bytes(B,H,N,block).
  * Matmuls run on the tensor cores in bf16 with fp32 accumulation; softmax in
- * fp32.  A persistent grid takes work items (the CSR rows) from a queue
- * ordered head-major and longest-first: heads by total selected blocks
- * descending, the rows of a head by block count descending (ties by lower
- * index), so that the SMs share one head's K and V in L2 at a time and finish
- * on the shortest rows.  B*H <= 4096, else
- * FVATTN_ERR_UNSUPPORTED.  Out-of-range or non-ascending column indices are
- * skipped and set *dev_status = FVATTN_ERR_BAD_CSR.
+ * fp32.  A work item is 128 query tokens of one head: one CSR row at block 128;
+ * at block 64 the pair of rows 2i and 2i+1 (query blocks of the same head),
+ * which walks the union of the two rows' key blocks, each row masking the blocks
+ * it did not select (item size = the union's size; see fvattn_attn_work_order).
+ * A persistent grid takes the items from a queue ordered head-major and
+ * longest-first: heads by total work descending, the items of a head by size
+ * descending (ties by lower index), so that the SMs share one head's K and V in
+ * L2 at a time and finish on the shortest items.  B*H <= 4096, else
+ * FVATTN_ERR_UNSUPPORTED.  Malformed rows (a negative count, column indices out
+ * of range or not ascending) set *dev_status = FVATTN_ERR_BAD_CSR; at block 128
+ * the offending indices are skipped (an index not above the one before it), at
+ * block 64 each row uses the set of its in-range indices.
  */
 FVATTN_API int fvattn_sparse_fwd(const void *Q, const void *K, const void *V, const int32_t *row_ptr,
                       const int32_t *col_idx, int B, int H, int N, int d, int block, int causal, void *O,
@@ -233,7 +238,8 @@ FVATTN_API int fvattn_attention_host(const void *hQ, const void *hK, const void 
  * file-scope device array of FVATTN_NOALLOC_SCRATCH_BYTES (4 MiB) inside the
  * library, which every device that loads the library keeps until the process
  * exits.  Shapes that need more return FVATTN_ERR_CAPACITY without launching
- * anything (about 1M rows B*H*ceil(N/block) at most).
+ * anything (rows B*H*ceil(N/block) up to about 1M at block 128, about 700k at
+ * block 64, whose pairs also keep their union sizes and a scan of them).
  *
  * Each call made outside stream capture looks up the array's device address
  * (cudaGetSymbolAddress, with the call's device current; a lookup allocates
@@ -347,7 +353,9 @@ FVATTN_API size_t fvattn_sasa_workspace_bytes(int B, int H, int N, int d, int bl
  * review, §1 Key Terms "SASA" and §3: after the work is balanced, the ranks that
  * would idle before the slowest one finishes compute extra high-value key
  * blocks).  On one GPU the ranks are the SMs of the persistent attention grid:
- *   1. the routed rows, in the attention's queue order (fvattn_attn_work_order),
+ *   1. the routed rows, head-major and longest first (the attention's queue order
+ *      at block 128, fvattn_attn_work_order; at block 64 the attention takes pairs
+ *      of rows, and the plan still schedules single rows, a model of that queue),
  *      are list-scheduled onto `machines` machines: each row to the machine with
  *      the least load so far, the lowest machine on equal loads, a row's load
  *      being its selected-block count; the makespan T is the largest load;
@@ -397,24 +405,37 @@ FVATTN_API int fvattn_route_sasa(const void *Q, const void *K, int B, int H, int
 FVATTN_API int fvattn_rlb_plan(const int64_t *work, int ranks, int units, int max_moves, int32_t *move_unit,
                                int32_t *move_src, int32_t *move_dst, int32_t *n_moves);
 
+/* Work items of fvattn_sparse_fwd: B*H*nb at block 128, B*H*ceil(nb/2) at block
+ * 64 (nb = ceil(N/block)); 0 on bad arguments. */
+FVATTN_API int64_t fvattn_attn_num_items(int B, int H, int N, int block);
+
 /*
  * fvattn_attn_work_order -- the order in which fvattn_sparse_fwd takes its work
- * items (CSR rows, one query block of one head each), written to order[0 .. rows)
- * with rows = B*H*ceil(N/block).  FVAttn review §1 "RLB" balances per-head work at
- * run time once the mask is known; on one GPU the SMs pop the rows from this queue:
- * heads by their total selected blocks (descending, equal totals by lower head
- * index), and inside a head its rows by block count (descending, equal counts by
- * lower row index).  The same kernels run inside fvattn_sparse_fwd; this call
- * exposes their result (for checks and diagnostics).
- *   row_ptr    device int32[rows+1], the CSR of fvattn_route (or a caller's mask).
- *   order      device int32[rows] (out): global row ids r = (b*H+h)*nb + i.
+ * items, written to order[0 .. items), items = fvattn_attn_num_items(B,H,N,block).
+ * An item is 128 query tokens of one head: at block 128 one CSR row (item id =
+ * row id (b*H+h)*nb + i, size = its block count); at block 64 the pair of rows 2i
+ * and 2i+1 of head (b,h) (item id (b*H+h)*ceil(nb/2) + i, size = the number of
+ * key blocks either row selects; with nb odd the last pair has row 2i only).
+ * FVAttn review §1 "RLB" balances per-head work at run time once the mask is
+ * known; on one GPU the SMs pop the items from this queue: heads by their total
+ * item size (descending, equal totals by lower head index), and inside a head its
+ * items by size (descending, equal sizes by lower item id).  The same kernels run
+ * inside fvattn_sparse_fwd; this call exposes their result (for checks and
+ * diagnostics).
+ *   row_ptr    device int32[B*H*nb + 1], the CSR of fvattn_route (or a caller's mask).
+ *   col_idx    device int32, its column indices: read at block 64 (the pairs'
+ *              unions), ignored (may be null) at block 128.
+ *   order      device int32[items] (out): item ids.
  *   workspace  device, fvattn_fwd_workspace_bytes(B,H,N,block) bytes, 16-byte aligned.
+ *   dev_status device int32[1]: at block 64 cleared, then FVATTN_ERR_BAD_CSR for a
+ *              malformed row; ignored (may be null) at block 128.
  * Asynchronous on `stream`.  Errors: bad sizes or null pointers
  * FVATTN_ERR_INVALID_ARG; B*H > 4096 or ceil(N/block) > 4096
  * FVATTN_ERR_UNSUPPORTED; short workspace FVATTN_ERR_CAPACITY.
  */
-FVATTN_API int fvattn_attn_work_order(const int32_t *row_ptr, int B, int H, int N, int block, int32_t *order,
-                                      void *workspace, size_t ws_bytes, fvattn_stream_t stream);
+FVATTN_API int fvattn_attn_work_order(const int32_t *row_ptr, const int32_t *col_idx, int B, int H, int N, int block,
+                                      int32_t *order, void *workspace, size_t ws_bytes, int32_t *dev_status,
+                                      fvattn_stream_t stream);
 
 /* Compiled-in build description (architecture, version), static string. */
 FVATTN_API const char *fvattn_build_info(void);

@@ -50,6 +50,7 @@ def _load():
         lib.oracle_lpt_order.argtypes = [P, i64, P]
         lib.oracle_route_cand.argtypes = [P, P, i32, i32, i32, i32, i32, dbl, P, P, i64, P, P, P, P, i32, i32]
         lib.oracle_head_order.argtypes = [P, i64, i64, P]
+        lib.oracle_pair_items.argtypes = [P, P, i64, i64, P, P, P]
         lib.oracle_sasa.argtypes = [P, P, i64, P, P, i32, P, i32, P, P, P, P, i64]
         lib.oracle_rlb_plan.argtypes = [P, i32, i32, i32, P, P, P, P]
         lib.oracle_attn_bwd.argtypes = [P, P, P, P, i32, i32, i32, i32, i32, i32, P, P, P, P, P, i32]
@@ -275,6 +276,24 @@ def head_order(row_ptr: np.ndarray, BH: int, nb: int) -> np.ndarray:
     if _load().oracle_head_order(_ptr(row_ptr), BH, nb, _ptr(order)) != 0:
         raise ValueError("oracle_head_order failed")
     return order
+
+
+def pair_items(row_ptr: np.ndarray, col_idx: np.ndarray, BH: int, nb: int):
+    """Work items at block 64: pairs of query blocks (2i, 2i+1) of a head, each the
+    union of the two rows' key blocks.  Returns (pair_ptr, pair_col, pair_bits), a CSR
+    over the BH * ceil(nb/2) pairs; bits 1: row 2i selected the block, 2: row 2i+1."""
+    row_ptr = np.ascontiguousarray(row_ptr, dtype=np.int32)
+    col_idx = np.ascontiguousarray(col_idx if len(col_idx) else np.zeros(1), dtype=np.int32)
+    np_ = (nb + 1) // 2
+    pair_ptr = np.empty(BH * np_ + 1, dtype=np.int32)
+    cap = max(int(row_ptr[-1]), 1)
+    pair_col = np.empty(cap, dtype=np.int32)
+    pair_bits = np.empty(cap, dtype=np.int32)
+    if _load().oracle_pair_items(_ptr(row_ptr), _ptr(col_idx), BH, nb, _ptr(pair_ptr), _ptr(pair_col),
+                                 _ptr(pair_bits)) != 0:
+        raise ValueError("oracle_pair_items failed")
+    n = int(pair_ptr[-1])
+    return pair_ptr, pair_col[:n].copy(), pair_bits[:n].copy()
 
 
 class Sasa:

@@ -44,6 +44,9 @@
  *               tokens, and to fp64 torch autograd of dense attention
  *   lpt_order   brute-force sort on small inputs
  *   head_order  brute-force sort on small inputs
+ *   pair_items  a hand-worked example (odd nb, empty rows, shared and single
+ *               blocks); on random rows, set unions and each row recovered from
+ *               its bits
  *   route candidates  the blocks right after the cut in the routing order:
  *               exhaustive comparison with the selected set's complement
  *   sasa        Graham's list-scheduling bound, loads within the makespan,
@@ -913,6 +916,55 @@ int oracle_head_order(const int32_t *row_ptr, int64_t BH, int64_t nb, int32_t *o
     }
     free(h);
     free(r);
+    return 0;
+}
+
+/*
+ * The attention's work items at a block of 64 tokens.  A tensor-core tile holds
+ * 128 query rows, two query blocks; the kernel gives it query blocks 2i and
+ * 2i+1 of one head (the last one alone when the head has an odd number of
+ * blocks), and the tile visits every key block either of the two selected
+ * ([FVAttn] §1 Key Terms, top-p routing: each query block keeps its own set).
+ * For pair i of head b (np = ceil(nb / 2) pairs per head, item id b * np + i)
+ * this writes the union of the two rows' key blocks, ascending, as a CSR
+ * (pair_ptr [BH*np + 1], pair_col), and pair_bits[e] = 1 if row 2i selected
+ * block pair_col[e], + 2 if row 2i+1 did.  The rows must hold ascending, in-range
+ * indices; the union is their two-way merge.  The work of an item (what the
+ * queue of oracle_head_order sorts by) is its union size.
+ */
+int oracle_pair_items(const int32_t *row_ptr, const int32_t *col_idx, int64_t BH, int64_t nb, int32_t *pair_ptr,
+                      int32_t *pair_col, int32_t *pair_bits) {
+    if (!row_ptr || !pair_ptr || BH < 1 || nb < 1) return -1;
+    const int64_t np = (nb + 1) / 2;
+    int64_t w = 0;
+    pair_ptr[0] = 0;
+    for (int64_t b = 0; b < BH; ++b) {
+        for (int64_t i = 0; i < np; ++i) {
+            const int64_t ra = b * nb + 2 * i;
+            int64_t ia = row_ptr[ra], ea = row_ptr[ra + 1];
+            int64_t ib = 0, eb = 0;
+            if (2 * i + 1 < nb) {
+                ib = row_ptr[ra + 1];
+                eb = row_ptr[ra + 2];
+            }
+            while (ia < ea || ib < eb) {
+                if (ib >= eb || (ia < ea && col_idx[ia] < col_idx[ib])) {
+                    pair_col[w] = col_idx[ia++];
+                    pair_bits[w] = 1;
+                } else if (ia >= ea || col_idx[ib] < col_idx[ia]) {
+                    pair_col[w] = col_idx[ib++];
+                    pair_bits[w] = 2;
+                } else {
+                    pair_col[w] = col_idx[ia];
+                    pair_bits[w] = 3;
+                    ++ia;
+                    ++ib;
+                }
+                ++w;
+            }
+            pair_ptr[b * np + i + 1] = (int32_t)w;
+        }
+    }
     return 0;
 }
 

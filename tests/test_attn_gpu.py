@@ -27,6 +27,11 @@ SMALL = [
     (W.Workload("p_one_small", B=2, H=2, N=700, d=128, bs=128, p=1.0, seed=36), False),
     (W.Workload("p_one_small_causal", B=2, H=2, N=700, d=128, bs=128, p=1.0, seed=36), True),
     (W.Workload("p_one_bs64_d64_causal", B=1, H=2, N=500, d=64, bs=64, p=1.0, seed=38), True),
+    # block 64, an odd number of query blocks (the last pair holds one row) and a
+    # ragged last block of 4 tokens
+    (W.Workload("bs64_odd_nb_causal", B=1, H=2, N=900, d=128, bs=64, p=1.0, seed=47), True),
+    (W.Workload("bs64_odd_nb_routed", B=2, H=2, N=900, d=64, bs=64, p=0.7, dist="structured", grid=(4, 15, 15),
+                head_scale=("uniform", 0.5, 4.0), seed=48), False),
     (W.Workload("large_scores", B=1, H=2, N=600, d=128, bs=128, p=0.8, dist="structured", grid=(6, 10, 10),
                 head_scale=("const", 6.0), seed=39), False),
 ]
@@ -84,6 +89,68 @@ def test_attention_custom_mask_with_empty_rows(oracle_mod):
     assert empty_tok.size > 0
 
 
+@pytest.mark.parametrize("N,causal", [(900, False), (1024, False), (900, True)])
+def test_block64_pairs_with_every_pattern(N, causal, oracle_mod):
+    """Block 64 runs neighbouring query blocks 2i and 2i+1 as one tile over the union of
+    their key blocks.  Pairs cycle through: both rows empty (O = 0, LSE = -inf), only
+    the second row non-empty, equal lists, disjoint lists, and independent lists; an
+    odd block count leaves the last row alone."""
+    rng = np.random.default_rng(49 + N)
+    w = W.Workload("pairs", B=1, H=3, N=N, d=128, bs=64, p=1.0, seed=49)
+    Q, K, V = W.generate(w)
+    nb = w.nb
+    sets = []
+    for h in range(w.H):
+        for i in range(0, nb, 2):
+            kind = (i // 2 + h) % 5
+            rand = lambda: sorted(rng.choice(nb, size=int(rng.integers(1, nb + 1)), replace=False).tolist())
+            if kind == 0:
+                a, b = [], []
+            elif kind == 1:
+                a, b = [], rand()
+            elif kind == 2:
+                a = rand()
+                b = list(a)
+            elif kind == 3:
+                perm = rng.permutation(nb)
+                a, b = sorted(perm[: nb // 2].tolist()), sorted(perm[nb // 2:].tolist())
+            else:
+                a, b = rand(), rand()
+            sets.append(a)
+            if i + 1 < nb:
+                sets.append(b)
+    rp = np.zeros(len(sets) + 1, np.int32)
+    rp[1:] = np.cumsum([len(x) for x in sets])
+    ci = np.asarray([j for x in sets for j in x], np.int32)
+    O, LSE = run_fwd(to_dev(Q), to_dev(K), to_dev(V), rp, ci, w.bs, causal)
+    tokens = np.arange(w.B * w.H * w.N, dtype=np.int64)
+    Oref, Lref = oracle_mod.attn_rows(Q, K, V, w.bs, causal, rp, ci, tokens)
+    compare_attention(O, LSE, Oref, Lref, tokens, w.d, "pairs")
+    # head 0, pair 0: both rows empty
+    assert torch.all(O.reshape(-1, w.d)[: 2 * w.bs].float() == 0)
+    assert torch.all(torch.isinf(LSE.reshape(-1)[: 2 * w.bs]))
+
+
+def test_block64_bad_csr_is_reported_and_in_range_entries_are_computed(oracle_mod):
+    """Block 64: an out-of-range index and a repeated one are reported as
+    FVATTN_ERR_BAD_CSR; every row is computed over its in-range entries."""
+    import top_routed_block_b200 as fv
+    w = W.Workload("badcsr64", B=1, H=1, N=256, d=64, bs=64, p=1.0, seed=50)
+    Q, K, V = W.generate(w)
+    rp = np.array([0, 2, 4, 6, 8], np.int32)
+    ci = np.array([0, 1, 1, 9, 2, 2, 0, 3], np.int32)   # row 1: index 9 out of range; row 2: repeat
+    good_rp = np.array([0, 2, 3, 4, 6], np.int32)
+    good_ci = np.array([0, 1, 1, 2, 0, 3], np.int32)
+    dQ, dK, dV = to_dev(Q), to_dev(K), to_dev(V)
+    O, LSE, st = fv.fvattn_sparse_fwd(dQ, dK, dV, torch.from_numpy(rp).cuda(), torch.from_numpy(ci).cuda(),
+                                      w.bs, False)
+    torch.cuda.synchronize()
+    assert int(st.item()) == fv.FVATTN_ERR_BAD_CSR
+    tokens = np.arange(w.N, dtype=np.int64)
+    Oref, Lref = oracle_mod.attn_rows(Q, K, V, w.bs, False, good_rp, good_ci, tokens)
+    compare_attention(O, LSE, Oref, Lref, tokens, w.d, "badcsr64")
+
+
 def test_attention_uniform_probabilities_give_mean_of_values(oracle_mod):
     """K = 0 makes every probability equal: O is the mean of the selected V rows.
     This isolates the P.V product (P layout in tensor memory, V descriptor)."""
@@ -114,7 +181,7 @@ def test_attention_one_hot_values_expose_probabilities(oracle_mod):
     compare_attention(O, LSE, Oref, Lref, tokens, w.d, "onehot")
 
 
-FULL = [(W.VIDEO, False), (W.DENSE, False), (W.DENSE_CAUSAL, True), (W.LONG, False)]
+FULL = [(W.VIDEO, False), (W.DENSE, False), (W.DENSE_CAUSAL, True), (W.LONG, False), (W.VIDEO_BS64, False)]
 
 
 @pytest.mark.parametrize("w,causal", FULL, ids=lambda x: x.name if hasattr(x, "name") else str(x))

@@ -723,6 +723,47 @@ def test_head_order_brute_force(oracle_mod, BH, nb, seed):
     assert list(oracle_mod.head_order(rp, BH, nb)) == want
 
 
+def test_pair_items_hand_worked(oracle_mod):
+    # one head, nb = 5 (three pairs, the last holding row 4 alone):
+    # rows 0: {0, 2}, 1: {1, 2, 4}, 2: {3}, 3: {}, 4: {0, 4}
+    rp = np.array([0, 2, 5, 6, 6, 8], np.int32)
+    ci = np.array([0, 2, 1, 2, 4, 3, 0, 4], np.int32)
+    pp, pc, pb = oracle_mod.pair_items(rp, ci, 1, 5)
+    assert list(pp) == [0, 4, 5, 7]
+    assert list(pc) == [0, 1, 2, 4, 3, 0, 4]
+    assert list(pb) == [1, 2, 3, 2, 1, 1, 1]
+
+
+@pytest.mark.parametrize("BH,nb,seed", [(1, 1, 0), (2, 7, 1), (3, 16, 2), (2, 33, 3)])
+def test_pair_items_are_set_unions(oracle_mod, BH, nb, seed):
+    rng = np.random.default_rng(seed)
+    sets = []
+    for r in range(BH * nb):
+        kind = r % 4
+        if kind == 0:
+            sets.append([])
+        elif kind == 1 and sets[-1]:
+            sets.append(list(sets[-1]))         # the same list as the row before
+        else:
+            sets.append(sorted(rng.choice(nb, size=int(rng.integers(1, nb + 1)), replace=False).tolist()))
+    rp = np.zeros(BH * nb + 1, np.int32)
+    rp[1:] = np.cumsum([len(x) for x in sets])
+    ci = np.asarray([j for x in sets for j in x], np.int32)
+    pp, pc, pb = oracle_mod.pair_items(rp, ci, BH, nb)
+    np_ = (nb + 1) // 2
+    assert pp.size == BH * np_ + 1
+    for b in range(BH):
+        for i in range(np_):
+            e0, e1 = pp[b * np_ + i], pp[b * np_ + i + 1]
+            a = set(sets[b * nb + 2 * i])
+            bb = set(sets[b * nb + 2 * i + 1]) if 2 * i + 1 < nb else set()
+            cols = list(pc[e0:e1])
+            assert cols == sorted(a | bb)
+            assert [c for c, x in zip(cols, pb[e0:e1]) if x & 1] == sorted(a)
+            assert [c for c, x in zip(cols, pb[e0:e1]) if x & 2] == sorted(bb)
+            assert all(x in (1, 2, 3) for x in pb[e0:e1])
+
+
 def _csr(counts):
     rp = np.zeros(len(counts) + 1, np.int32)
     rp[1:] = np.cumsum(counts)

@@ -77,7 +77,8 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         "fvattn_sparse_fwd_noalloc": (I, [P, P, P, P, P, I, I, I, I, I, I, P, P, P, P]),
         "fvattn_test_sparse_fwd_stall": (I, [P, P, P, P, P, I, I, I, I, I, I, P, P, P, SZ, P, P]),
         "fvattn_sparse_fwd_profiled": (I, [P, P, P, P, P, I, I, I, I, I, I, P, P, P, SZ, P, I, P, P, P]),
-        "fvattn_attn_work_order": (I, [P, I, I, I, I, P, P, SZ, P]),
+        "fvattn_attn_num_items": (I64, [I, I, I, I]),
+        "fvattn_attn_work_order": (I, [P, P, I, I, I, I, P, P, SZ, P, P]),
         "fvattn_sasa_workspace_bytes": (SZ, [I, I, I, I, I]),
         "fvattn_rlb_plan": (I, [P, I, I, I, P, P, P, P]),
         "fvattn_route_sasa": (I, [P, P, I, I, I, I, I, D, I, P, P, I64, P, P, P, P, P, P, SZ, P, P]),
@@ -356,20 +357,30 @@ def fvattn_route_sasa(Q: torch.Tensor, K: torch.Tensor, p: float, block: int, ma
     return out
 
 
-def fvattn_attn_work_order(row_ptr: torch.Tensor, B: int, H: int, N: int, block: int, *, stream=None,
-                           order: torch.Tensor | None = None, workspace: torch.Tensor | None = None) -> torch.Tensor:
-    """The queue order of fvattn_sparse_fwd's work items (global CSR row ids)."""
+def fvattn_attn_num_items(B: int, H: int, N: int, block: int) -> int:
+    """Work items of fvattn_sparse_fwd: query blocks at block 128, pairs of them at 64."""
+    return int(load_library().fvattn_attn_num_items(B, H, N, block))
+
+
+def fvattn_attn_work_order(row_ptr: torch.Tensor, B: int, H: int, N: int, block: int,
+                           col_idx: torch.Tensor | None = None, *, stream=None, order: torch.Tensor | None = None,
+                           workspace: torch.Tensor | None = None, dev_status: torch.Tensor | None = None):
+    """The queue order of fvattn_sparse_fwd's work items (item ids: CSR rows at block
+    128, pairs of rows 2i, 2i+1 at block 64, which needs col_idx).  Returns the order
+    and the device status (FVATTN_ERR_BAD_CSR for a malformed row at block 64)."""
     lib = load_library()
     dev = row_ptr.device
-    rows = fvattn_num_rows(B, H, N, block)
+    items = fvattn_attn_num_items(B, H, N, block)
     if order is None:
-        order = torch.empty(rows, dtype=torch.int32, device=dev)
+        order = torch.empty(items, dtype=torch.int32, device=dev)
     if workspace is None:
         workspace = _empty_bytes(fvattn_fwd_workspace_bytes(B, H, N, block), dev)
-    rc = lib.fvattn_attn_work_order(_ptr(row_ptr), B, H, N, block, _ptr(order), _ptr(workspace), workspace.numel(),
-                                    _stream_ptr(stream))
+    if dev_status is None:
+        dev_status = torch.zeros(1, dtype=torch.int32, device=dev)
+    rc = lib.fvattn_attn_work_order(_ptr(row_ptr), _ptr(col_idx), B, H, N, block, _ptr(order), _ptr(workspace),
+                                    workspace.numel(), _ptr(dev_status), _stream_ptr(stream))
     _check(rc, "fvattn_attn_work_order")
-    return order
+    return order, dev_status
 
 
 def fvattn_bwd_workspace_bytes(B: int, H: int, N: int, block: int) -> int:

@@ -108,25 +108,56 @@ bool make_map(CUtensorMap *m, const void *base, int64_t BH, int N, int d, int ro
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-struct FwdWorkspace {
-    size_t order, head_rank, counter, total;
-};
-
-// items: work items of the attention kernel; BH: heads.
-FwdWorkspace fwd_layout(int64_t items, int64_t BH) {
-    FwdWorkspace w{};
-    Carver c;
-    w.order = c.take<int32_t>(static_cast<size_t>(items));
-    w.head_rank = c.take<int32_t>(static_cast<size_t>(BH));
-    w.counter = c.take<int32_t>(64);
-    w.total = align_up(c.off, 256);
-    return w;
-}
-
 int from_cuda(cudaError_t e) {
     if (e == cudaSuccess) return FVATTN_OK;
     set_last_error(cudaGetErrorName(e));
     return FVATTN_ERR_CUDA;
+}
+
+struct FwdWorkspace {
+    size_t order, head_rank, counter, pair_count, pair_ptr, pair_head, total;
+};
+
+// The forward's scratch for BH heads of nb query blocks at block bs: the queue order
+// of the work items, the ordering kernels' head ranks and the queue counter; at block
+// 64 also the pairs' union sizes, their scan and per-head sums.
+FwdWorkspace fwd_layout(int64_t BH, int nb, int bs) {
+    FwdWorkspace w{};
+    Carver c;
+    const int64_t items = attn_num_items(BH, nb, bs);
+    w.order = c.take<int32_t>(static_cast<size_t>(items));
+    w.head_rank = c.take<int32_t>(static_cast<size_t>(BH));
+    w.counter = c.take<int32_t>(64);
+    if (bs == 64) {
+        w.pair_count = c.take<int32_t>(static_cast<size_t>(items));
+        w.pair_ptr = c.take<int32_t>(static_cast<size_t>(items) + 1);
+        w.pair_head = c.take<int32_t>(static_cast<size_t>(BH));
+    }
+    w.total = align_up(c.off, 256);
+    return w;
+}
+
+// The queue order of the forward's work items into ws + w.order (head-major, longest
+// first; order_mode 1: items by index).  Block 64 first sizes the pairs (their key-block
+// unions, which also checks the CSR) and orders them by those sizes.
+int enqueue_work_order(const int32_t *row_ptr, const int32_t *col_idx, int64_t BH, int nb, int bs, int order_mode,
+                       char *ws, const FwdWorkspace &w, int32_t *dev_status, cudaStream_t s) {
+    const int64_t items = attn_num_items(BH, nb, bs);
+    auto i32 = [&](size_t off) { return reinterpret_cast<int32_t *>(ws + off); };
+    const int32_t *item_ptr = row_ptr;
+    int per_head = nb;
+    if (bs == 64) {
+        const int np = (nb + 1) / 2;
+        cudaError_t e = launch_pair_counts(row_ptr, col_idx, BH, nb, i32(w.pair_count), dev_status, s);
+        if (e == cudaSuccess)
+            e = launch_csr_scan(i32(w.pair_count), items, np, BH, i32(w.pair_ptr), items * nb, i32(w.pair_head),
+                                dev_status, s);
+        if (e != cudaSuccess) return from_cuda(e);
+        item_ptr = i32(w.pair_ptr);
+        per_head = np;
+    }
+    return from_cuda(order_mode == 1 ? launch_natural_order(items, i32(w.order), s)
+                                     : launch_item_order(item_ptr, BH, per_head, i32(w.head_rank), i32(w.order), s));
 }
 
 struct BwdWorkspace {
@@ -204,7 +235,7 @@ size_t fvattn_fwd_workspace_bytes(int B, int H, int N, int block) {
     if (nb > kMaxCount) return 0;
     const int64_t BH = static_cast<int64_t>(B) * H;
     if (BH > kMaxHeads) return 0;
-    return fwd_layout(attn_num_items(BH, static_cast<int>(nb)), BH).total;
+    return fwd_layout(BH, static_cast<int>(nb), block).total;
 }
 
 int fvattn_route(const void *Q, const void *K, int B, int H, int N, int d, int block, double p, int32_t *row_ptr,
@@ -283,11 +314,10 @@ static int sparse_fwd_impl(const void *Q, const void *K, const void *V, const in
     const int64_t BH = static_cast<int64_t>(B) * H;
     const int nb = static_cast<int>(ceil_div(N, block));
     if (BH > kMaxHeads) return FVATTN_ERR_UNSUPPORTED;
-    const int64_t items = attn_num_items(BH, nb);
-    const FwdWorkspace w = fwd_layout(items, BH);
+    const int64_t items = attn_num_items(BH, nb, block);
+    const FwdWorkspace w = fwd_layout(BH, nb, block);
     char *ws = static_cast<char *>(workspace);
     int32_t *order = reinterpret_cast<int32_t *>(ws + w.order);
-    int32_t *head_rank = reinterpret_cast<int32_t *>(ws + w.head_rank);
     int *counter = reinterpret_cast<int *>(ws + w.counter);
 
     // K and V are read one key block per TMA box
@@ -297,10 +327,10 @@ static int sparse_fwd_impl(const void *Q, const void *K, const void *V, const in
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if ((rc = from_cuda(cudaMemsetAsync(dev_status, 0, sizeof(int32_t), s))) != FVATTN_OK) return rc;
-    // work items (CSR rows): head-major, longest first (or rows by index, for comparison)
-    rc = from_cuda(order_mode == 1 ? launch_natural_order(items, order, s)
-                                   : launch_item_order(row_ptr, BH, nb, head_rank, order, s));
-    if (rc != FVATTN_OK) return rc;
+    // work items (rows, or pairs of rows at block 64): head-major, longest first (or by
+    // index, for comparison)
+    if ((rc = enqueue_work_order(row_ptr, col_idx, BH, nb, block, order_mode, ws, w, dev_status, s)) != FVATTN_OK)
+        return rc;
     if ((rc = from_cuda(cudaMemsetAsync(counter, 0, sizeof(int), s))) != FVATTN_OK) return rc;
 
     AttnLaunch a{};
@@ -366,22 +396,36 @@ int fvattn_sparse_fwd_profiled(const void *Q, const void *K, const void *V, cons
                            dev_status, stream, 0, order_mode, cta_busy_ns, grid);
 }
 
-int fvattn_attn_work_order(const int32_t *row_ptr, int B, int H, int N, int block, int32_t *order, void *workspace,
-                           size_t ws_bytes, fvattn_stream_t stream) {
+int64_t fvattn_attn_num_items(int B, int H, int N, int block) {
+    if (B < 1 || H < 1 || N < 1 || (block != 64 && block != 128)) return 0;
+    return attn_num_items(static_cast<int64_t>(B) * H, static_cast<int>(ceil_div(N, block)), block);
+}
+
+int fvattn_attn_work_order(const int32_t *row_ptr, const int32_t *col_idx, int B, int H, int N, int block,
+                           int32_t *order, void *workspace, size_t ws_bytes, int32_t *dev_status,
+                           fvattn_stream_t stream) {
     if (B < 1 || H < 1 || N < 1 || !row_ptr || !order || !workspace) return FVATTN_ERR_INVALID_ARG;
     if (block != 64 && block != 128) return FVATTN_ERR_UNSUPPORTED;
+    if (block == 64 && (!col_idx || !dev_status)) return FVATTN_ERR_INVALID_ARG;
     const int64_t BH = static_cast<int64_t>(B) * H;
     const int64_t nb = ceil_div(N, block);
     if (BH > kMaxHeads || nb > kMaxCount) return FVATTN_ERR_UNSUPPORTED;
     if (!aligned16(workspace)) return FVATTN_ERR_ALIGNMENT;
-    if ((reinterpret_cast<uintptr_t>(row_ptr) | reinterpret_cast<uintptr_t>(order)) & 3u) return FVATTN_ERR_ALIGNMENT;
+    if ((reinterpret_cast<uintptr_t>(row_ptr) | reinterpret_cast<uintptr_t>(order) |
+         reinterpret_cast<uintptr_t>(col_idx) | reinterpret_cast<uintptr_t>(dev_status)) & 3u)
+        return FVATTN_ERR_ALIGNMENT;
     if (ws_bytes < fvattn_fwd_workspace_bytes(B, H, N, block)) return FVATTN_ERR_CAPACITY;
     int rc = check_device();
     if (rc != FVATTN_OK) return rc;
-    const FwdWorkspace w = fwd_layout(attn_num_items(BH, static_cast<int>(nb)), BH);
-    int32_t *head_rank = reinterpret_cast<int32_t *>(static_cast<char *>(workspace) + w.head_rank);
-    return from_cuda(launch_item_order(row_ptr, BH, static_cast<int>(nb), head_rank, order,
-                                       reinterpret_cast<cudaStream_t>(stream)));
+    const FwdWorkspace w = fwd_layout(BH, static_cast<int>(nb), block);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (dev_status && (rc = from_cuda(cudaMemsetAsync(dev_status, 0, sizeof(int32_t), s))) != FVATTN_OK) return rc;
+    char *ws = static_cast<char *>(workspace);
+    if ((rc = enqueue_work_order(row_ptr, col_idx, BH, static_cast<int>(nb), block, 0, ws, w, dev_status, s)) !=
+        FVATTN_OK)
+        return rc;
+    const int64_t items = attn_num_items(BH, static_cast<int>(nb), block);
+    return from_cuda(cudaMemcpyAsync(order, ws + w.order, sizeof(int32_t) * items, cudaMemcpyDeviceToDevice, s));
 }
 
 namespace {

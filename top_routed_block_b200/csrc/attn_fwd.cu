@@ -8,11 +8,22 @@
 // partial output rescaled by exp(m_old - m_new) whenever the maximum grows.
 //
 // B200 design:
-//   * One work item = one query block of one head (a CSR row).  A persistent
-//     grid of one CTA per SM pops items from a queue ordered head-major and
-//     longest-first (FVAttn §1 "RLB" balances per-head work at run time; here
-//     the SMs are balanced instead, and the head order keeps one or two heads'
-//     K and V in L2 while all SMs work on them).
+//   * One work item = 128 query rows of one head: at block 128 one query block
+//     (a CSR row), at block 64 two neighbouring query blocks 2i and 2i+1 (a
+//     pair).  A pair walks the union of its two rows' key-block lists; each
+//     half of the tile masks the key blocks its own row did not select, which
+//     leaves its m, l and O exactly as they were, so every row gets the result
+//     of its own list and the M = 128 MMAs carry no zero rows.  The TMA warp
+//     builds a pair's union in shared memory (per-row bitmaps, then a warp
+//     scan) when it takes the item.  A tile is always 128 key columns: at
+//     block 64, two consecutive entries of the union (two 64-row TMA boxes in
+//     one ring stage; an odd union's last tile reads rows past N, zero-filled,
+//     for its second half), so the MMAs and the softmax have the same shapes,
+//     and the same per-tile overheads, at both block sizes.  A persistent grid of one CTA per SM pops
+//     items from a queue ordered head-major and longest-first (FVAttn §1 "RLB"
+//     balances per-head work at run time; here the SMs are balanced instead,
+//     and the head order keeps one or two heads' K and V in L2 while all SMs
+//     work on them).
 //   * Warps 0-3 run the softmax and the epilogue (thread = query row = TMEM
 //     lane); warp 4 issues TMA loads of K and V tiles into a ring of shared
 //     memory stages; warp 5 issues the tcgen05 MMAs.
@@ -65,6 +76,7 @@ namespace {
 using namespace ptx;
 
 constexpr int kRowsM = 128;           // query rows per tile (tcgen05 M)
+constexpr int kKT = 128;              // key columns per tile (tcgen05 N of S, K of PV)
 constexpr int kThreads = 192;         // softmax warpgroup + TMA warp + MMA warp
 constexpr int kCtasPerSm = 1;         // kernels that hold tensor memory are resident one CTA per SM
 constexpr int kTmaWarp = 4;
@@ -72,6 +84,8 @@ constexpr int kMmaWarp = 5;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kMaxStages = 12;
 constexpr int kRingBytes = 192 * 1024;
+constexpr int kUnionCap = kMaxCount;           // entries of one pair's key-block union
+constexpr int kBitmapWords = kMaxCount / 32;   // one row's key-block bitmap
 
 template <int D, int BS, bool F8>
 struct Cfg {
@@ -80,16 +94,25 @@ struct Cfg {
     static constexpr int KBLK = D * EB / 128;             // 128-byte column blocks along d
     static constexpr int X_CHUNK = 128 / EB;              // elements per 128-byte column block
     static constexpr int KSTEP = 32 / EB;                 // K of one MMA (32 bytes of operand)
-    static constexpr int STAGE_BYTES = KBLK * BS * 128;   // one K or V tile
+    // A tile is kKT = 128 key columns: one key block at block 128, two key blocks
+    // (two entries of a pair's union, 64 rows each) at block 64.
+    static constexpr int HALVES = kKT / BS;               // key blocks per tile
+    static constexpr int STAGE_BYTES = KBLK * kKT * 128;  // one K or V tile
     static constexpr int NST = kRingBytes / STAGE_BYTES < kMaxStages ? kRingBytes / STAGE_BYTES : kMaxStages;
     static constexpr int TILE_BYTES = NST * STAGE_BYTES;
-    static constexpr int SMEM_BYTES = TILE_BYTES + 1024 /*alignment slack*/ + 512 /*barriers*/;
+    // block 64: an item is a pair of query blocks; its key-block union lives in
+    // shared memory, two slots of uint16 entries (block << 2 | row bits), plus the
+    // two rows' bitmaps the union is built from
+    static constexpr bool PAIR = BS == 64;
+    static constexpr int UNION_BYTES = PAIR ? 2 * kUnionCap * 2 + 2 * kBitmapWords * 4 : 0;
+    static constexpr int SMEM_BYTES = TILE_BYTES + 1024 /*alignment slack*/ + 512 /*barriers*/ + UNION_BYTES;
+    static_assert(!PAIR || 2 * BS == kRowsM, "a pair fills the M = 128 tile");
     // TMEM columns: Q buffers (packed operands), S buffers (fp32; P as bf16 pairs or
     // e4m3 quads in their first columns), O (fp32)
     static constexpr uint32_t Q_COLS = D * EB / 4;
-    static constexpr uint32_t T_Q0 = 0, T_Q1 = Q_COLS, T_S0 = 128, T_S1 = 128 + BS, T_O = 128 + 2 * BS;
+    static constexpr uint32_t T_Q0 = 0, T_Q1 = Q_COLS, T_S0 = 128, T_S1 = 128 + kKT, T_O = 128 + 2 * kKT;
     static_assert(2 * Q_COLS <= 128 && T_O + D <= kTmemCols, "TMEM layout exceeds 512 columns");
-    static constexpr uint32_t IDESC_S = F8 ? idesc_e4m3_f32(kRowsM, BS, 0, 0) : idesc_bf16_f32(kRowsM, BS, 0, 0);
+    static constexpr uint32_t IDESC_S = F8 ? idesc_e4m3_f32(kRowsM, kKT, 0, 0) : idesc_bf16_f32(kRowsM, kKT, 0, 0);
     static constexpr uint32_t IDESC_PV = F8 ? idesc_e4m3_f32(kRowsM, D, 0, 1) : idesc_bf16_f32(kRowsM, D, 0, 1);
 };
 
@@ -139,6 +162,69 @@ __device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float
 // sums of degenerate blocks finite).
 __device__ __forceinline__ float pow2_scale(float x, int e) { return ldexpf(x, max(-200, min(e, 126))); }
 
+// ------------------------------------------------------------- block-64 pairs
+// Pair i of head bh: query blocks 2i (row A) and 2i+1 (row B, absent when nb is
+// odd and i is the last pair).  The 32 lanes of a warp set one bit per selected
+// key block in two bitmaps bm[0, nw) (A) and bm[nw, 2 nw) (B), nw = ceil(nb / 32);
+// entries outside [0, nb) are left out.  With CHECK, also whether a row is
+// malformed (a negative count, an entry outside [0, nb), or one not above the
+// entry before it).
+template <bool CHECK>
+__device__ bool pair_bitmaps(const int32_t *__restrict__ row_ptr, const int32_t *__restrict__ col_idx, int64_t bh,
+                             int pair, int nb, uint32_t *bm, int lane) {
+    const int nw = (nb + 31) >> 5;
+    for (int w = lane; w < 2 * nw; w += 32) bm[w] = 0u;
+    __syncwarp();
+    const int64_t ra = bh * nb + 2 * pair;
+    const bool has_b = 2 * pair + 1 < nb;
+    const int a0 = __ldg(row_ptr + ra), a1 = __ldg(row_ptr + ra + 1);
+    const int b1 = has_b ? __ldg(row_ptr + ra + 2) : a1;
+    bool bad = CHECK && (a1 < a0 || b1 < a1);
+    for (int h = 0; h < 2; ++h) {
+        const int s0 = h ? a1 : a0, s1 = h ? b1 : a1;
+        for (int k = s0 + lane; k < s1; k += 32) {
+            const int x = __ldg(col_idx + k);
+            if (x >= 0 && x < nb) atomicOr(bm + h * nw + (x >> 5), 1u << (x & 31));
+            else if (CHECK) bad = true;
+            if (CHECK && k > s0 && __ldg(col_idx + k - 1) >= x) bad = true;
+        }
+    }
+    __syncwarp();
+    return __any_sync(0xffffffffu, bad);
+}
+
+// The pair's union from its bitmaps, ascending, as entries (block << 2) | (1 if row
+// A selected it) | (2 if row B did), written to out[0, count) by the 32 lanes (each
+// lane takes a run of words; a warp scan of their bit counts places the runs).
+// Returns count (<= nb) on every lane.
+__device__ int pair_union(const uint32_t *bm, int nb, uint16_t *out, int lane) {
+    const int nw = (nb + 31) >> 5;
+    const int wpl = (nw + 31) >> 5;  // words per lane (<= kBitmapWords / 32)
+    const int w0 = lane * wpl;
+    int cnt = 0;
+    for (int q = 0; q < wpl; ++q)
+        if (w0 + q < nw) cnt += __popc(bm[w0 + q] | bm[nw + w0 + q]);
+    int inc = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += t;
+    }
+    int pos = inc - cnt;
+    for (int q = 0; q < wpl; ++q) {
+        const int w = w0 + q;
+        if (w >= nw) break;
+        const uint32_t a = bm[w], b = bm[nw + w];
+        uint32_t u = a | b;
+        while (u) {
+            const int bit = __ffs(u) - 1;
+            u &= u - 1;
+            out[pos++] = static_cast<uint16_t>(((w * 32 + bit) << 2) | ((a >> bit) & 1u) | (((b >> bit) & 1u) << 1));
+        }
+    }
+    return __shfl_sync(0xffffffffu, inc, 31);
+}
+
 template <int D, int BS, bool F8>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
@@ -155,6 +241,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     const uint32_t base_addr = smem_addr(smem_raw);
     unsigned char *ring = smem_raw + ((1024 - (base_addr & 1023)) & 1023);  // stage s at s * STAGE_BYTES
     Barriers *bar = reinterpret_cast<Barriers *>(ring + C::TILE_BYTES);
+    // pairs only: the two union slots and the bitmaps
+    uint16_t *uni = reinterpret_cast<uint16_t *>(ring + C::TILE_BYTES + 512);
+    uint32_t *bmap = reinterpret_cast<uint32_t *>(ring + C::TILE_BYTES + 512 + 2 * kUnionCap * 2);
+    const int ipb = C::PAIR ? (nb + 1) >> 1 : nb;  // items per head
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -193,7 +283,81 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         bar->t_start = t0;
     }
 
-    if (warp == kTmaWarp) {
+    if (warp == kTmaWarp && C::PAIR) {
+        // ------------------------------------------------- producer (pairs)
+        // The whole warp builds each pair's union into the item's slot; lane 0
+        // pops items, publishes them and issues the loads.
+        if (lane == 0) {
+            prefetch_tensormap(&tmap_k);
+            prefetch_tensormap(&tmap_v);
+        }
+        uint32_t it = 0, rc = 0;  // items published, ring loads issued (lane 0)
+        while (true) {
+            int idx = 0, pr = -1;
+            if (lane == 0) {
+                idx = atomicAdd(work_counter, 1);
+                pr = (idx < n_items) ? order[idx] : -1;
+            }
+            idx = __shfl_sync(0xffffffffu, idx, 0);
+            pr = __shfl_sync(0xffffffffu, pr, 0);
+            const uint32_t k = it & 1;
+            // the slot is free once the previous item in it has been consumed
+            int free_ok = 1;
+            if (lane == 0) free_ok = mbar_wait(&bar->sched_empty[k], ((it >> 1) & 1) ^ 1, abort_flag, dev_status);
+            if (!__shfl_sync(0xffffffffu, free_ok, 0)) break;
+            uint16_t *ul = uni + k * kUnionCap;
+            int count = 0;
+            if (pr >= 0) {
+                pair_bitmaps<false>(row_ptr, col_idx, pr / ipb, pr % ipb, nb, bmap, lane);
+                count = pair_union(bmap, nb, ul, lane);
+            }
+            __threadfence_block();  // the union entries before lane 0 publishes the item
+            __syncwarp();
+            int ok = 1;
+            if (lane == 0) {
+                // item: {pair, union entries, tiles (two entries each), queue index + 1}
+                const int tiles = (count + 1) >> 1;
+                bar->sched_item[k] = make_int4(pr, count, tiles, pr >= 0 ? idx + 1 : 0);
+                mbar_arrive(&bar->sched_full[k]);
+                if (pr >= 0) {
+                    const int bh = pr / ipb;
+                    for (int j = 0; j < tiles && ok; ++j) {
+                        // the two key blocks of the tile (the union is ascending and in
+                        // range); an odd union's last tile loads rows past N for its
+                        // second half, which the TMA unit fills with zeros
+                        const int row0 = (ul[2 * j] >> 2) * BS;
+                        const int row1 = (2 * j + 1 < count) ? (ul[2 * j + 1] >> 2) * BS : nb * BS;
+                        for (int kv = 0; kv < 2; ++kv) {
+                            const uint32_t st = rc % NST;
+                            if (!mbar_wait(&bar->ring_empty[st], ((rc / NST) & 1) ^ 1, abort_flag, dev_status)) {
+                                ok = 0;
+                                break;
+                            }
+                            mbar_arrive_expect_tx(&bar->ring_full[st], C::STAGE_BYTES);
+                            for (int kb = 0; kb < C::KBLK; ++kb) {
+                                unsigned char *dst = ring + st * C::STAGE_BYTES + kb * kKT * 128;
+                                const CUtensorMap *map = kv == 0 ? &tmap_k : &tmap_v;
+                                tma_load_3d(dst, map, &bar->ring_full[st], kb * C::X_CHUNK, row0, bh);
+                                tma_load_3d(dst + BS * 128, map, &bar->ring_full[st], kb * C::X_CHUNK, row1, bh);
+                            }
+                            ++rc;
+                        }
+                    }
+                }
+            }
+            ++it;
+            if (pr < 0 || !__shfl_sync(0xffffffffu, ok, 0)) break;
+        }
+        // every load lane 0 issued lands before the CTA exits
+        if (lane == 0) {
+            for (uint32_t st = 0; st < static_cast<uint32_t>(NST); ++st) {
+                if (rc > st) {
+                    const uint32_t times = (rc - st + NST - 1) / NST;
+                    mbar_wait_teardown(&bar->ring_full[st], (times - 1) & 1);
+                }
+            }
+        }
+    } else if (warp == kTmaWarp) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             prefetch_tensormap(&tmap_k);
@@ -238,7 +402,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                         }
                         mbar_arrive_expect_tx(&bar->ring_full[st], C::STAGE_BYTES);
                         for (int kb = 0; kb < C::KBLK; ++kb)
-                            tma_load_3d(ring + st * C::STAGE_BYTES + kb * BS * 128, kv == 0 ? &tmap_k : &tmap_v,
+                            tma_load_3d(ring + st * C::STAGE_BYTES + kb * kKT * 128, kv == 0 ? &tmap_k : &tmap_v,
                                         &bar->ring_full[st], kb * C::X_CHUNK, kblk * BS, bh);
                         ++rc;
                     }
@@ -270,7 +434,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                 const uint64_t kdesc = smem_desc_sw128(r0 + st * C::STAGE_BYTES, 16, 1024);
 #pragma unroll
                 for (int k = 0; k < D * C::EB / 32; ++k) {
-                    const uint64_t db = kdesc + (((k >> 2) * BS * 128 + (k & 3) * 32) >> 4);
+                    const uint64_t db = kdesc + (((k >> 2) * kKT * 128 + (k & 3) * 32) >> 4);
                     if (F8)
                         mma_ts_f8_nc(tmem + scol, tmem + qcol + k * 8, db, C::IDESC_S, k > 0 ? 1u : 0u);
                     else
@@ -279,9 +443,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             };
             // O (+)= P V, P from the S buffer at scol, V of ring stage st (MN-major)
             auto issue_pv = [&](uint32_t scol, uint32_t st, bool first) {
-                const uint64_t vdesc = smem_desc_sw128(r0 + st * C::STAGE_BYTES, BS * 128, 1024);
+                const uint64_t vdesc = smem_desc_sw128(r0 + st * C::STAGE_BYTES, kKT * 128, 1024);
 #pragma unroll
-                for (int k = 0; k < BS / C::KSTEP; ++k) {
+                for (int k = 0; k < kKT / C::KSTEP; ++k) {
                     const uint64_t dv = vdesc + ((k * C::KSTEP * 128) >> 4);
                     if (F8)
                         mma_ts_f8_nc(tmem + C::T_O, tmem + scol + k * 8, dv, C::IDESC_PV, (!first || k > 0) ? 1u : 0u);
@@ -350,22 +514,31 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
         uint32_t it = 0, tc = 0, qn = 0, on = 0;  // items read, tiles, Q loads, outputs
         bool ok = true;
+        // Items are read in queue order; item number n sits in slot n & 1.  A pair's
+        // slot also holds its key-block union, so the slot is released only after the
+        // item's last tile (release_item); a row's slot is released at once.
         auto next_item = [&](int4 &out) {
             const uint32_t k = it & 1;
             if (!mbar_wait(&bar->sched_full[k], (it >> 1) & 1, abort_flag, dev_status)) return false;
             out = bar->sched_item[k];
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bar->sched_empty[k]);
+            if (!C::PAIR && lane == 0) mbar_arrive(&bar->sched_empty[k]);
             ++it;
             return true;
+        };
+        auto release_item = [&](uint32_t n) {
+            if (C::PAIR) {
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bar->sched_empty[n & 1]);
+            }
         };
         // This thread's query row of `itm` (zeros past the block or past N) into the
         // Q buffer of Q load number qn, as packed operands (bf16 pairs or e4m3 quads,
         // in order).
         auto load_q = [&](const int4 &itm) {
-            const int64_t bhq = itm.x / nb;
-            const int tq = (itm.x % nb) * BS + r;
-            const bool in = r < BS && tq < N;
+            const int64_t bhq = itm.x / ipb;
+            const int tq = (itm.x % ipb) * kRowsM + r;
+            const bool in = tq < N;
             const uint4 *src = reinterpret_cast<const uint4 *>(Qg + (bhq * N + (in ? tq : 0)) * (D * C::EB));
             const uint32_t tQ = tmem + lane_base + ((qn & 1) ? C::T_Q1 : C::T_Q0);
 #pragma unroll
@@ -392,36 +565,67 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         if (next_item(item)) {
             if (item.w && item.z > 0) load_q(item);
             while (item.w) {
-                const int row = item.x, start = item.y, count = item.z;
-                const int64_t bh = row / nb;
-                const int qb = row % nb;
-                const int t_row = qb * BS + r;  // token index of this thread's row
+                // rows: item.y = CSR start, item.z = key blocks (tiles); pairs: item.y =
+                // union entries, item.z = tiles (two entries each)
+                const int start = item.y, count = item.z;
+                const uint32_t slot_n = it - 1;  // queue number of this item (its slot: & 1)
+                const int64_t bh = item.x / ipb;
+                const int t_row = (item.x % ipb) * kRowsM + r;  // token index of this thread's row
+                const int qb = t_row / BS;                     // this row's query block
+                const int half = C::PAIR ? (r >> 6) : 0;       // pairs: row A (0) or row B (1) of the item
+                const uint16_t *ul = uni + (slot_n & 1) * kUnionCap;
                 float m = -CUDART_INF_F, l = 0.0f;
                 int prev = -1;
-                int kblk_next = count > 0 ? __ldg(col_idx + start) : 0;  // loaded one tile ahead
-                // e4m3 operands: the item's Q exponent, the running V reference exponent E
-                const int eq = F8 ? __ldg(q_exp + row) : 0;
+                // rows: the next tile's key block, loaded one tile ahead
+                int kblk_next = (!C::PAIR && count > 0) ? __ldg(col_idx + start) : 0;
+                // e4m3 operands: the row's Q exponent, the running V reference exponent E
+                const int eq = (F8 && qb < nb) ? __ldg(q_exp + bh * nb + qb) : 0;
                 int e_ref = 0;
                 bool have_ref = false;
                 for (int j = 0; j < count; ++j) {
-                    const int kblk = kblk_next;
-                    if (j + 1 < count) kblk_next = __ldg(col_idx + start + j + 1);
-                    const bool valid = kblk >= 0 && kblk < nb && kblk > prev;
-                    if (valid) prev = kblk;
-                    const int key0 = kblk * BS;
-                    // keys of this block that exist and are allowed for this row
-                    int lim = valid ? min(BS, N - key0) : 0;
-                    if (causal) lim = min(lim, t_row - key0 + 1);
-                    // this tile's score scale (log2 units) and, for e4m3, its V exponent
-                    float sc = scale_log2;
-                    int ev = 0;
-                    if (F8 && valid) {
-                        sc = pow2_scale(scale_log2, eq + __ldg(k_exp + bh * nb + kblk));
-                        ev = __ldg(v_exp + bh * nb + kblk);
+                    // the tile's key blocks (-1: none) and whether this row takes each
+                    int kb[C::HALVES];
+                    bool mine[C::HALVES];
+                    if constexpr (C::PAIR) {
+#pragma unroll
+                        for (int h = 0; h < C::HALVES; ++h) {
+                            const int e = (C::HALVES * j + h < start) ? static_cast<int>(ul[C::HALVES * j + h]) : -1;
+                            kb[h] = e >= 0 ? (e >> 2) : -1;
+                            mine[h] = e >= 0 && ((e >> half) & 1);
+                        }
+                    } else {
+                        kb[0] = kblk_next;
+                        if (j + 1 < count) kblk_next = __ldg(col_idx + start + j + 1);
+                        mine[0] = true;
                     }
-                    const bool e_up = F8 && valid && (!have_ref || ev > e_ref);
-                    const int e_new = e_up ? ev : e_ref;
-                    const float fv = F8 ? pow2_scale(1.0f, ev - e_new) : 1.0f;
+                    // per key block: the keys that exist and are allowed for this row, the
+                    // score scale (log2 units) and, for e4m3, the V exponent; E moves up to
+                    // the largest V exponent this row has taken
+                    int lim[C::HALVES], ev[C::HALVES];
+                    float sc[C::HALVES], fv[C::HALVES];
+                    int e_new = e_ref;
+                    bool e_up = false;
+#pragma unroll
+                    for (int h = 0; h < C::HALVES; ++h) {
+                        const bool valid = kb[h] >= 0 && kb[h] < nb && kb[h] > prev;
+                        if (valid) prev = kb[h];
+                        mine[h] = mine[h] && valid;
+                        const int key0 = kb[h] * BS;
+                        lim[h] = mine[h] ? min(BS, N - key0) : 0;
+                        if (causal) lim[h] = min(lim[h], t_row - key0 + 1);
+                        sc[h] = scale_log2;
+                        ev[h] = 0;
+                        if (F8 && mine[h]) {
+                            sc[h] = pow2_scale(scale_log2, eq + __ldg(k_exp + bh * nb + kb[h]));
+                            ev[h] = __ldg(v_exp + bh * nb + kb[h]);
+                            if (!(have_ref || e_up) || ev[h] > e_new) {
+                                e_new = ev[h];
+                                e_up = true;
+                            }
+                        }
+                    }
+#pragma unroll
+                    for (int h = 0; h < C::HALVES; ++h) fv[h] = F8 ? pow2_scale(1.0f, ev[h] - e_new) : 1.0f;
                     const uint32_t sb = tc & 1;
                     if (!mbar_wait(&bar->s_full[sb], (tc >> 1) & 1, abort_flag, dev_status)) {
                         ok = false;
@@ -429,25 +633,32 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                     }
                     tc_fence_after();
                     const uint32_t tS = tmem + lane_base + (sb ? C::T_S1 : C::T_S0);
-                    // the whole S row of this thread: BS fp32 values
-                    uint32_t v[BS];
+                    // the whole S row of this thread: kKT fp32 values
+                    uint32_t v[kKT];
 #pragma unroll
-                    for (int c0 = 0; c0 < BS; c0 += 32)
+                    for (int c0 = 0; c0 < kKT; c0 += 32)
                         tmem_ld32(tS + c0, *reinterpret_cast<uint32_t(*)[32]>(&v[c0]));
                     tmem_wait_ld();
-                    if (lim < BS) {  // ragged last block, causal diagonal, or a skipped index
 #pragma unroll
-                        for (int c = 0; c < BS; ++c)
-                            if (c >= lim) v[c] = __float_as_uint(-CUDART_INF_F);
+                    for (int h = 0; h < C::HALVES; ++h) {
+                        if (lim[h] < BS) {  // ragged last block, causal diagonal, a skipped index or none
+#pragma unroll
+                            for (int c = 0; c < BS; ++c)
+                                if (c >= lim[h]) v[h * BS + c] = __float_as_uint(-CUDART_INF_F);
+                        }
                     }
-                    float mq[4] = {-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F};
+                    float mxs = -CUDART_INF_F;
 #pragma unroll
-                    for (int c = 0; c < BS; c += 8) {
+                    for (int h = 0; h < C::HALVES; ++h) {
+                        float mq[4] = {-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F};
 #pragma unroll
-                        for (int q = 0; q < 4; ++q)
-                            mq[q] = max3f(mq[q], __uint_as_float(v[c + 2 * q]), __uint_as_float(v[c + 2 * q + 1]));
+                        for (int c = h * BS; c < (h + 1) * BS; c += 8) {
+#pragma unroll
+                            for (int q = 0; q < 4; ++q)
+                                mq[q] = max3f(mq[q], __uint_as_float(v[c + 2 * q]), __uint_as_float(v[c + 2 * q + 1]));
+                        }
+                        mxs = fmaxf(mxs, max3f(mq[0], mq[1], fmaxf(mq[2], mq[3])) * sc[h]);
                     }
-                    const float mxs = max3f(mq[0], mq[1], fmaxf(mq[2], mq[3])) * sc;
                     // The reference maximum only moves when the row maximum exceeds it by
                     // more than 2^8: P stays below 256 and the rescale of O is rare.  O and
                     // l always share the same reference, so the final O / l is exact.
@@ -460,30 +671,28 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                         // P packed as bf16 pairs in place, v[c/2] <- (p[c], p[c+1]); one loop for
                         // full and masked tiles (masked scores are -inf, and 2^-inf = 0)
 #pragma unroll
-                        for (int c = 0; c < BS; c += 2) {
-                            const float p0 = ex2_approx(fmaf(__uint_as_float(v[c]), sc, neg_m));
-                            const float p1 = ex2_approx(fmaf(__uint_as_float(v[c + 1]), sc, neg_m));
+                        for (int c = 0; c < kKT; c += 2) {
+                            const float p0 = ex2_approx(fmaf(__uint_as_float(v[c]), sc[c / BS], neg_m));
+                            const float p1 = ex2_approx(fmaf(__uint_as_float(v[c + 1]), sc[c / BS], neg_m));
                             rs[(c >> 1) & 3] += p0 + p1;
                             v[c >> 1] = pack_bf16(p0, p1);
                         }
 #pragma unroll
-                        for (int c0 = 0; c0 < BS / 2; c0 += 32)
+                        for (int c0 = 0; c0 < kKT / 2; c0 += 32)
                             tmem_st32(tS + c0, *reinterpret_cast<const uint32_t(*)[32]>(&v[c0]));
                     } else {
                         // P * 2^(e_v - E) as e4m3 quads in place, v[c/4] <- (p[c] .. p[c+3])
 #pragma unroll
-                        for (int c = 0; c < BS; c += 4) {
-                            const float p0 = ex2_approx(fmaf(__uint_as_float(v[c]), sc, neg_m));
-                            const float p1 = ex2_approx(fmaf(__uint_as_float(v[c + 1]), sc, neg_m));
-                            const float p2 = ex2_approx(fmaf(__uint_as_float(v[c + 2]), sc, neg_m));
-                            const float p3 = ex2_approx(fmaf(__uint_as_float(v[c + 3]), sc, neg_m));
+                        for (int c = 0; c < kKT; c += 4) {
+                            const float s4 = sc[c / BS], f4 = fv[c / BS];
+                            const float p0 = ex2_approx(fmaf(__uint_as_float(v[c]), s4, neg_m));
+                            const float p1 = ex2_approx(fmaf(__uint_as_float(v[c + 1]), s4, neg_m));
+                            const float p2 = ex2_approx(fmaf(__uint_as_float(v[c + 2]), s4, neg_m));
+                            const float p3 = ex2_approx(fmaf(__uint_as_float(v[c + 3]), s4, neg_m));
                             rs[(c >> 2) & 3] += (p0 + p1) + (p2 + p3);
-                            v[c >> 2] = pack_e4m3x4(p0 * fv, p1 * fv, p2 * fv, p3 * fv);
+                            v[c >> 2] = pack_e4m3x4(p0 * f4, p1 * f4, p2 * f4, p3 * f4);
                         }
-                        if constexpr (BS / 4 >= 32)
-                            tmem_st32(tS, *reinterpret_cast<const uint32_t(*)[32]>(&v[0]));
-                        else
-                            tmem_st16(tS, *reinterpret_cast<const uint32_t(*)[16]>(&v[0]));
+                        tmem_st32(tS, *reinterpret_cast<const uint32_t(*)[32]>(&v[0]));
                     }
                     float alpha = alpha_m;
                     if (F8 && e_up && have_ref) alpha = pow2_scale(alpha_m, e_ref - e_new);  // O in units of 2^E
@@ -491,7 +700,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                     // Rescale the running output.  The PV of the previous block may still be
                     // accumulating into O: wait for it first (its completion is phase tc-1
                     // of pv_done; the PV of this block cannot start before P is published).
-                    if (__any_sync(0xffffffffu, (need && j > 0) || (e_up && have_ref))) {
+                    // (a row without an earlier block, m = -inf, has O = 0: nothing to rescale)
+                    if (__any_sync(0xffffffffu, (need && m != -CUDART_INF_F) || (e_up && have_ref))) {
                         if (!mbar_wait(&bar->pv_done, (tc - 1) & 1, abort_flag, dev_status)) {
                             ok = false;
                             break;
@@ -518,6 +728,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                     ++tc;
                 }
                 if (!ok) break;
+                release_item(slot_n);
                 if (count > 0) ++qn;
                 // the next item's Q goes into TMEM before this item's epilogue, so its first
                 // S tiles overlap the epilogue
@@ -528,7 +739,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                 if (!mbar_wait(&bar->o_full, on & 1, abort_flag, dev_status)) break;
                 ++on;
                 tc_fence_after();
-                const bool row_ok = r < BS && t_row < N;
+                const bool row_ok = t_row < N;
                 const float inv_l = (l > 0.0f) ? (F8 ? pow2_scale(1.0f / l, e_ref) : 1.0f / l) : 0.0f;
                 __nv_bfloat16 *orow = O + (bh * N + t_row) * D;
                 const uint32_t tO = tmem + lane_base + C::T_O;
@@ -571,6 +782,30 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         cta_busy_ns[blockIdx.x] = t_end - bar->t_start;
     }
     if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
+}
+
+// Block 64: the key-block union size of every pair (one warp per pair), the work
+// of its item; also checks the two rows and records FVATTN_ERR_BAD_CSR for a
+// malformed one (the attention kernel then uses each row's in-range entries).
+constexpr int kPairWarps = 8;
+__global__ void __launch_bounds__(kPairWarps * 32)
+    pair_count_kernel(const int32_t *__restrict__ row_ptr, const int32_t *__restrict__ col_idx, int64_t BH, int nb,
+                      int32_t *__restrict__ counts, int32_t *dev_status) {
+    __shared__ uint32_t bm_s[kPairWarps][2 * kBitmapWords];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int np = (nb + 1) >> 1;
+    const int nw = (nb + 31) >> 5;
+    uint32_t *bm = bm_s[warp];
+    for (int64_t pr = static_cast<int64_t>(blockIdx.x) * kPairWarps + warp; pr < BH * np;
+         pr += static_cast<int64_t>(gridDim.x) * kPairWarps) {
+        const bool bad = pair_bitmaps<true>(row_ptr, col_idx, pr / np, static_cast<int>(pr % np), nb, bm, lane);
+        if (bad && lane == 0) record_error(dev_status, FVATTN_ERR_BAD_CSR);
+        int c = 0;
+        for (int w = lane; w < nw; w += 32) c += __popc(bm[w] | bm[nw + w]);
+        c = __reduce_add_sync(0xffffffffu, c);
+        if (lane == 0) counts[pr] = c;
+        __syncwarp();  // the bitmaps are reused by the next pair
+    }
 }
 
 // Natural order (rows by index), the comparison point for the load-imbalance factor.
@@ -663,7 +898,16 @@ int attn_smem_bytes(int d, int bs) {
 
 int attn_ctas_per_sm() { return kCtasPerSm; }
 
-int64_t attn_num_items(int64_t BH, int nb) { return BH * nb; }
+int64_t attn_num_items(int64_t BH, int nb, int bs) { return BH * (bs == 64 ? (nb + 1) / 2 : nb); }
+
+cudaError_t launch_pair_counts(const int32_t *row_ptr, const int32_t *col_idx, int64_t BH, int nb, int32_t *counts,
+                               int32_t *dev_status, cudaStream_t stream) {
+    const int64_t pairs = BH * ((nb + 1) / 2);
+    const int64_t need = (pairs + kPairWarps - 1) / kPairWarps;
+    const int grid = static_cast<int>(need < 4096 ? (need > 0 ? need : 1) : 4096);
+    pair_count_kernel<<<grid, kPairWarps * 32, 0, stream>>>(row_ptr, col_idx, BH, nb, counts, dev_status);
+    return cudaGetLastError();
+}
 
 static int pow2_at_least(int n) {
     int p = 1;

@@ -10,7 +10,10 @@ namespace fvattn {
 struct AttnLaunch {
     const CUtensorMap *tmap_k, *tmap_v;  // host copies, passed by value as kernel parameters
     const void *Q;                       // [B,H,N,d] bf16 or e4m3 codes, read row by row into tensor memory
-    const int32_t *row_ptr, *col_idx, *order;  // order: work items (CSR rows), head-major, longest first
+    // order: work items, head-major, longest first; an item is a CSR row at block 128,
+    // a pair of neighbouring rows (query blocks 2i, 2i+1; item id bh * ceil(nb/2) + i)
+    // at block 64
+    const int32_t *row_ptr, *col_idx, *order;
     int n_items;
     int *work_counter;  // zeroed before the launch
     int N, nb, causal;
@@ -27,8 +30,13 @@ struct AttnLaunch {
 };
 
 int attn_smem_bytes(int d, int bs);
-// Work items of the attention kernel: the CSR rows (query blocks of every head).
-int64_t attn_num_items(int64_t BH, int nb);
+// Work items of the attention kernel: the CSR rows (query blocks of every head) at
+// block 128, the pairs of neighbouring rows at block 64.
+int64_t attn_num_items(int64_t BH, int nb, int bs);
+// Block 64: counts[bh * ceil(nb/2) + i] = size of the union of the key-block lists of
+// rows 2i and 2i+1 of head bh; a malformed row records FVATTN_ERR_BAD_CSR.
+cudaError_t launch_pair_counts(const int32_t *row_ptr, const int32_t *col_idx, int64_t BH, int nb, int32_t *counts,
+                               int32_t *dev_status, cudaStream_t stream);
 // order[] = rows head-major, longest first (heads by total selected blocks, rows of
 // a head by block count); head_rank[BH] is scratch.  B*H <= 4096, nb <= 4096.
 cudaError_t launch_item_order(const int32_t *row_ptr, int64_t BH, int nb, int32_t *head_rank, int32_t *order,

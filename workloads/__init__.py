@@ -65,6 +65,10 @@ DENSE_CAUSAL = dataclasses.replace(DENSE, name="dense_causal", causal=True)
 LONG = Workload("long_video", B=1, H=24, N=33 * 45 * 80, d=128, bs=128, p=0.8, dist="structured",
                 grid=(33, 45, 80), head_scale=("uniform", 0.5, 4.0), seed=3)
 
+# Block 64 on the video shape (a measurement case beside the named configs: the
+# pages' video workload, routed and attended in blocks of 64 tokens).
+VIDEO_BS64 = dataclasses.replace(VIDEO, name="video_dit_bs64", bs=64)
+
 
 def sweep() -> list[Workload]:
     """B1 H8 N32768 on a 16x32x64 grid; d x p x head-scale spread (20 runs)."""
@@ -80,7 +84,7 @@ def sweep() -> list[Workload]:
     return out
 
 
-ALL = {w.name: w for w in [TINY, VIDEO, DENSE, DENSE_CAUSAL, LONG] + sweep()}
+ALL = {w.name: w for w in [TINY, VIDEO, DENSE, DENSE_CAUSAL, LONG, VIDEO_BS64] + sweep()}
 
 
 def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
