@@ -291,8 +291,8 @@ def run_reference(args, w, rank, world):
 # ------------------------------------------------------------ GPU (ours)
 
 # Workloads timed beside the headline one, each for a few steps in the same run.
-CONFIG_SET = ("tiny", "dense", "dense_causal", "long_video", "sweep_d64_s1_p0.9", "sweep_d64_s05_8_p0.9",
-              "sweep_d128_s1_p0.9", "sweep_d128_s05_8_p0.9")
+CONFIG_SET = ("tiny", "dense", "dense_causal", "long_video", "video_dit_bs64", "sweep_d64_s1_p0.9",
+              "sweep_d64_s05_8_p0.9", "sweep_d128_s1_p0.9", "sweep_d128_s05_8_p0.9")
 
 
 def causal_block_csr(w: W.Workload, dev):
