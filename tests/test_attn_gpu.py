@@ -32,6 +32,10 @@ SMALL = [
     (W.Workload("bs64_odd_nb_causal", B=1, H=2, N=900, d=128, bs=64, p=1.0, seed=47), True),
     (W.Workload("bs64_odd_nb_routed", B=2, H=2, N=900, d=64, bs=64, p=0.7, dist="structured", grid=(4, 15, 15),
                 head_scale=("uniform", 0.5, 4.0), seed=48), False),
+    # d = 64 at block 128: many items, ragged tails, causal and routed
+    (W.Workload("d64_bs128_routed", B=1, H=4, N=3000, d=64, bs=128, p=0.7, dist="structured",
+                grid=(5, 20, 30), head_scale=("uniform", 0.5, 4.0), seed=51), False),
+    (W.Workload("d64_bs128_causal", B=2, H=3, N=1500, d=64, bs=128, p=1.0, seed=52), True),
     (W.Workload("large_scores", B=1, H=2, N=600, d=128, bs=128, p=0.8, dist="structured", grid=(6, 10, 10),
                 head_scale=("const", 6.0), seed=39), False),
 ]
@@ -64,10 +68,11 @@ def test_attention_small_every_token(w, causal, oracle_mod):
     print(w.name, compare_attention(O, LSE, Oref, Lref, tokens, w.d, w.name))
 
 
-def test_attention_custom_mask_with_empty_rows(oracle_mod):
+@pytest.mark.parametrize("d", [128, 64])
+def test_attention_custom_mask_with_empty_rows(d, oracle_mod):
     """Arbitrary ascending key-block sets, empty rows included (O = 0, LSE = -inf)."""
     rng = np.random.default_rng(40)
-    w = W.Workload("custom", B=1, H=2, N=900, d=128, bs=128, p=1.0, seed=40)
+    w = W.Workload("custom", B=1, H=2, N=900, d=d, bs=128, p=1.0, seed=40)
     Q, K, V = W.generate(w)
     rows, nb = w.rows, w.nb
     sets = []
@@ -266,11 +271,12 @@ def test_host_buffer_path_matches_device_path(w):
         assert torch.equal(hL, L_dev.cpu())
 
 
-def test_profiled_forward_reports_busy_time_and_matches():
+@pytest.mark.parametrize("d,bs", [(128, 128), (64, 128), (128, 64)])
+def test_profiled_forward_reports_busy_time_and_matches(d, bs):
     """fvattn_sparse_fwd_profiled returns exactly what fvattn_sparse_fwd returns, in
     either work order (rows are independent), plus a positive busy time per CTA."""
     import top_routed_block_b200 as fv
-    w = W.Workload("profiled", B=1, H=6, N=3000, d=128, bs=128, p=0.8, dist="structured", grid=(5, 20, 30),
+    w = W.Workload("profiled", B=1, H=6, N=3000, d=d, bs=bs, p=0.8, dist="structured", grid=(5, 20, 30),
                    head_scale=("uniform", 0.5, 4.0), seed=45)
     Q, K, V = W.generate(w)
     dQ, dK, dV = to_dev(Q), to_dev(K), to_dev(V)

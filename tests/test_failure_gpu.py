@@ -12,9 +12,11 @@ from tests.gpu_util import compare_attention, gpu_route, to_dev
 pytestmark = pytest.mark.gpu
 
 
-def test_bounded_wait_times_out_and_context_survives(oracle_mod):
+@pytest.mark.parametrize("d,bs", [(128, 128), (64, 128), (128, 64)],
+                         ids=["d128_bs128", "d64_bs128", "paired_blocks_bs64"])
+def test_bounded_wait_times_out_and_context_survives(d, bs, oracle_mod):
     import top_routed_block_b200 as fv
-    w = W.Workload("stall", B=1, H=2, N=1024, d=128, bs=128, p=0.9, dist="structured", grid=(4, 16, 16),
+    w = W.Workload("stall", B=1, H=2, N=1024, d=d, bs=bs, p=0.9, dist="structured", grid=(4, 16, 16),
                    head_scale=("uniform", 0.5, 4.0), seed=61)
     Q, K, V = W.generate(w)
     dQ, dK, dV = to_dev(Q), to_dev(K), to_dev(V)
