@@ -889,3 +889,19 @@ def test_rlb_close_to_exhaustive_optimum_on_tiny_instances(oracle_mod):
                    for a in it.product(range(ranks), repeat=flat.size))
         _, loads, _ = _rlb_apply(work, oracle_mod.rlb_plan(work))
         assert best <= loads.max() <= best + flat.max()
+
+
+def test_near_tie_report_flags_exact_ties_at_the_cut(oracle_mod):
+    """The GPU routing tests report rows whose cut separates two blocks of (almost)
+    equal probability.  With K = 0 every score ties, so every row cut short of all
+    blocks is such a row; on structured inputs none is expected."""
+    from tests.gpu_util import near_tie_rows
+    w = W.Workload("ties", B=1, H=2, N=1000, d=64, bs=64, p=0.5, seed=5)
+    Q, K, _ = W.generate(w)
+    r = oracle_mod.route(Q, np.zeros_like(K), w.p, w.bs)
+    cut = np.diff(r.row_ptr) < w.nb
+    assert cut.all() and np.array_equal(near_tie_rows(r, w.p), cut)
+    w2 = W.Workload("no_ties", B=1, H=2, N=1000, d=64, bs=64, p=0.7, dist="structured", grid=(4, 10, 25),
+                    head_scale=("uniform", 0.5, 4.0), seed=6)
+    Q2, K2, _ = W.generate(w2)
+    assert not near_tie_rows(oracle_mod.route(Q2, K2, w2.p, w2.bs), w2.p).any()

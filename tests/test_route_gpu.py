@@ -36,7 +36,8 @@ def run_case(w, oracle_mod):
     ora = oracle_mod.route(Q, K, w.p, w.bs)
     gpu = gpu_route(to_dev(Q), to_dev(K), w.p, w.bs)
     excluded = compare_routes(gpu, ora, w.p, w.nb, w.B * w.H)
-    print(f"{w.name}: rows {w.rows} nnz {gpu[0][-1]} excluded(near p) {excluded}")
+    print(f"{w.name}: rows {w.rows} nnz {gpu[0][-1]} excluded(near p) {excluded} "
+          f"near-tie cuts (checked bit-exact) {compare_routes.last_near_ties}")
     return gpu, ora
 
 
