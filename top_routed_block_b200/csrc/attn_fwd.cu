@@ -602,7 +602,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                     // score scale (log2 units) and, for e4m3, the V exponent; E moves up to
                     // the largest V exponent this row has taken
                     int lim[C::HALVES], ev[C::HALVES];
-                    float sc[C::HALVES], fv[C::HALVES];
+                    float sc[C::HALVES];
                     int e_new = e_ref;
                     bool e_up = false;
 #pragma unroll
@@ -624,8 +624,6 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                             }
                         }
                     }
-#pragma unroll
-                    for (int h = 0; h < C::HALVES; ++h) fv[h] = F8 ? pow2_scale(1.0f, ev[h] - e_new) : 1.0f;
                     const uint32_t sb = tc & 1;
                     if (!mbar_wait(&bar->s_full[sb], (tc >> 1) & 1, abort_flag, dev_status)) {
                         ok = false;
@@ -681,18 +679,30 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                         for (int c0 = 0; c0 < kKT / 2; c0 += 32)
                             tmem_st32(tS + c0, *reinterpret_cast<const uint32_t(*)[32]>(&v[c0]));
                     } else {
-                        // P * 2^(e_v - E) as e4m3 quads in place, v[c/4] <- (p[c] .. p[c+3])
+                        // P * 2^(e_v - E) as e4m3 quads in place, v[c/4] <- (p[c] .. p[c+3]).  The
+                        // power of two goes into the exponent, 2^(s sc - m + e_v - E), and the
+                        // row sum takes the scaled values back by 2^(E - e_v) once per key block
+                        // (exact: a power of two).
+                        float nm[C::HALVES], rh[C::HALVES][2];
+#pragma unroll
+                        for (int h = 0; h < C::HALVES; ++h) {
+                            nm[h] = neg_m + static_cast<float>(ev[h] - e_new);
+                            rh[h][0] = rh[h][1] = 0.0f;
+                        }
 #pragma unroll
                         for (int c = 0; c < kKT; c += 4) {
-                            const float s4 = sc[c / BS], f4 = fv[c / BS];
-                            const float p0 = ex2_approx(fmaf(__uint_as_float(v[c]), s4, neg_m));
-                            const float p1 = ex2_approx(fmaf(__uint_as_float(v[c + 1]), s4, neg_m));
-                            const float p2 = ex2_approx(fmaf(__uint_as_float(v[c + 2]), s4, neg_m));
-                            const float p3 = ex2_approx(fmaf(__uint_as_float(v[c + 3]), s4, neg_m));
-                            rs[(c >> 2) & 3] += (p0 + p1) + (p2 + p3);
-                            v[c >> 2] = pack_e4m3x4(p0 * f4, p1 * f4, p2 * f4, p3 * f4);
+                            const float s4 = sc[c / BS], n4 = nm[c / BS];
+                            const float p0 = ex2_approx(fmaf(__uint_as_float(v[c]), s4, n4));
+                            const float p1 = ex2_approx(fmaf(__uint_as_float(v[c + 1]), s4, n4));
+                            const float p2 = ex2_approx(fmaf(__uint_as_float(v[c + 2]), s4, n4));
+                            const float p3 = ex2_approx(fmaf(__uint_as_float(v[c + 3]), s4, n4));
+                            rh[c / BS][(c >> 2) & 1] += (p0 + p1) + (p2 + p3);
+                            v[c >> 2] = pack_e4m3x4(p0, p1, p2, p3);
                         }
                         tmem_st32(tS, *reinterpret_cast<const uint32_t(*)[32]>(&v[0]));
+#pragma unroll
+                        for (int h = 0; h < C::HALVES; ++h)
+                            rs[h] = pow2_scale(rh[h][0] + rh[h][1], e_new - ev[h]);
                     }
                     float alpha = alpha_m;
                     if (F8 && e_up && have_ref) alpha = pow2_scale(alpha_m, e_ref - e_new);  // O in units of 2^E
