@@ -667,14 +667,26 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                     float rs[4] = {0.0f, 0.0f, 0.0f, 0.0f};
                     if constexpr (!F8) {
                         // P packed as bf16 pairs in place, v[c/2] <- (p[c], p[c+1]); one loop for
-                        // full and masked tiles (masked scores are -inf, and 2^-inf = 0)
+                        // full and masked tiles (masked scores are -inf, and 2^-inf = 0).  The
+                        // scaling and the row sums run on fp32 pairs (one instruction per two
+                        // columns).
+                        uint64_t sc2[C::HALVES];
+#pragma unroll
+                        for (int h = 0; h < C::HALVES; ++h) sc2[h] = f32x2_pack(sc[h], sc[h]);
+                        const uint64_t nm2 = f32x2_pack(neg_m, neg_m);
+                        uint64_t acc2[2] = {0ull, 0ull};
 #pragma unroll
                         for (int c = 0; c < kKT; c += 2) {
-                            const float p0 = ex2_approx(fmaf(__uint_as_float(v[c]), sc[c / BS], neg_m));
-                            const float p1 = ex2_approx(fmaf(__uint_as_float(v[c + 1]), sc[c / BS], neg_m));
-                            rs[(c >> 1) & 3] += p0 + p1;
+                            float x0, x1;
+                            f32x2_unpack(f32x2_fma(f32x2_pack(__uint_as_float(v[c]), __uint_as_float(v[c + 1])),
+                                                   sc2[c / BS], nm2),
+                                         x0, x1);
+                            const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+                            acc2[(c >> 1) & 1] = f32x2_add(acc2[(c >> 1) & 1], f32x2_pack(p0, p1));
                             v[c >> 1] = pack_bf16(p0, p1);
                         }
+                        f32x2_unpack(acc2[0], rs[0], rs[1]);
+                        f32x2_unpack(acc2[1], rs[2], rs[3]);
 #pragma unroll
                         for (int c0 = 0; c0 < kKT / 2; c0 += 32)
                             tmem_st32(tS + c0, *reinterpret_cast<const uint32_t(*)[32]>(&v[c0]));
@@ -683,26 +695,36 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                         // power of two goes into the exponent, 2^(s sc - m + e_v - E), and the
                         // row sum takes the scaled values back by 2^(E - e_v) once per key block
                         // (exact: a power of two).
-                        float nm[C::HALVES], rh[C::HALVES][2];
+                        // (scaling and row sums on fp32 pairs, one instruction per two columns)
+                        uint64_t sc2[C::HALVES], nm2[C::HALVES], rh2[C::HALVES];
 #pragma unroll
                         for (int h = 0; h < C::HALVES; ++h) {
-                            nm[h] = neg_m + static_cast<float>(ev[h] - e_new);
-                            rh[h][0] = rh[h][1] = 0.0f;
+                            const float nmh = neg_m + static_cast<float>(ev[h] - e_new);
+                            sc2[h] = f32x2_pack(sc[h], sc[h]);
+                            nm2[h] = f32x2_pack(nmh, nmh);
+                            rh2[h] = 0ull;
                         }
 #pragma unroll
                         for (int c = 0; c < kKT; c += 4) {
-                            const float s4 = sc[c / BS], n4 = nm[c / BS];
-                            const float p0 = ex2_approx(fmaf(__uint_as_float(v[c]), s4, n4));
-                            const float p1 = ex2_approx(fmaf(__uint_as_float(v[c + 1]), s4, n4));
-                            const float p2 = ex2_approx(fmaf(__uint_as_float(v[c + 2]), s4, n4));
-                            const float p3 = ex2_approx(fmaf(__uint_as_float(v[c + 3]), s4, n4));
-                            rh[c / BS][(c >> 2) & 1] += (p0 + p1) + (p2 + p3);
+                            float x0, x1, x2, x3;
+                            f32x2_unpack(f32x2_fma(f32x2_pack(__uint_as_float(v[c]), __uint_as_float(v[c + 1])),
+                                                   sc2[c / BS], nm2[c / BS]),
+                                         x0, x1);
+                            f32x2_unpack(f32x2_fma(f32x2_pack(__uint_as_float(v[c + 2]), __uint_as_float(v[c + 3])),
+                                                   sc2[c / BS], nm2[c / BS]),
+                                         x2, x3);
+                            const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+                            const float p2 = ex2_approx(x2), p3 = ex2_approx(x3);
+                            rh2[c / BS] = f32x2_add(f32x2_add(rh2[c / BS], f32x2_pack(p0, p1)), f32x2_pack(p2, p3));
                             v[c >> 2] = pack_e4m3x4(p0, p1, p2, p3);
                         }
                         tmem_st32(tS, *reinterpret_cast<const uint32_t(*)[32]>(&v[0]));
 #pragma unroll
-                        for (int h = 0; h < C::HALVES; ++h)
-                            rs[h] = pow2_scale(rh[h][0] + rh[h][1], e_new - ev[h]);
+                        for (int h = 0; h < C::HALVES; ++h) {
+                            float a0, a1;
+                            f32x2_unpack(rh2[h], a0, a1);
+                            rs[h] = pow2_scale(a0 + a1, e_new - ev[h]);
+                        }
                     }
                     float alpha = alpha_m;
                     if (F8 && e_up && have_ref) alpha = pow2_scale(alpha_m, e_ref - e_new);  // O in units of 2^E

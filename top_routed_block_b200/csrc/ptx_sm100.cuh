@@ -313,5 +313,27 @@ __host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N, int a_mn_maj
            | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// ------------------------------------------------------- packed fp32 pairs (sm_100)
+// Two fp32 values in one 64-bit register pair; fma/add on both lanes in one
+// instruction (each lane rounds as its scalar counterpart, round to nearest even).
+__device__ __forceinline__ uint64_t f32x2_pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f32x2_unpack(uint64_t x, float &lo, float &hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(x));
+}
+__device__ __forceinline__ uint64_t f32x2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t f32x2_add(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
 }  // namespace ptx
 }  // namespace fvattn
