@@ -421,9 +421,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bar->s_free);  // S may be overwritten by the next block
                 if (__all_sync(0xffffffffu, lim >= BS)) {
+                    // scale-and-shift on fp32 pairs (one instruction per two columns)
+                    const uint64_t sc2 = f32x2_pack(scale_log2, scale_log2), nl2 = f32x2_pack(-lse2, -lse2);
 #pragma unroll
-                    for (int c = 0; c < BS; ++c)
-                        v[c] = __float_as_uint(ex2_approx(fmaf(__uint_as_float(v[c]), scale_log2, -lse2)));
+                    for (int c = 0; c < BS; c += 2) {
+                        float x0, x1;
+                        f32x2_unpack(f32x2_fma(f32x2_pack(__uint_as_float(v[c]), __uint_as_float(v[c + 1])), sc2, nl2),
+                                     x0, x1);
+                        v[c] = __float_as_uint(ex2_approx(x0));
+                        v[c + 1] = __float_as_uint(ex2_approx(x1));
+                    }
                 } else {
 #pragma unroll
                     for (int c = 0; c < BS; ++c)
@@ -443,10 +450,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tmem_ld32(tmem + lane_base + C::T_DP + h0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&g[32]));
                     tmem_wait_ld();
                     uint32_t w[32];
+                    const uint64_t d2 = f32x2_pack(Dt, Dt);
 #pragma unroll
-                    for (int c = 0; c < 64; c += 2)
-                        w[c >> 1] = pack_bf16(__uint_as_float(v[h0 + c]) * (__uint_as_float(g[c]) - Dt),
-                                              __uint_as_float(v[h0 + c + 1]) * (__uint_as_float(g[c + 1]) - Dt));
+                    for (int c = 0; c < 64; c += 2) {
+                        // on fp32 pairs: (dP - D) and the product with P, one instruction each per two columns
+                        float y0, y1;
+                        f32x2_unpack(f32x2_mul(f32x2_pack(__uint_as_float(v[h0 + c]), __uint_as_float(v[h0 + c + 1])),
+                                               f32x2_sub(f32x2_pack(__uint_as_float(g[c]), __uint_as_float(g[c + 1])),
+                                                         d2)),
+                                     y0, y1);
+                        w[c >> 1] = pack_bf16(y0, y1);
+                    }
                     tmem_st32(tmem + lane_base + C::T_DP + h0 / 2, w);
                 }
                 tmem_wait_st();
@@ -742,7 +756,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int ku = (cl % nb) * BS + r;  // this thread's key token
             const bool key_in = ku < N;
             bool ok = true;
-            // The LSE (log2 units, +inf past N) and D of the item's query block jj, the
+            // The negated LSE (log2 units, -inf past N) and D of the item's query block jj, the
             // CTA's tile number tt, go into shared copy tt % 3 one tile ahead, shared by
             // the four warps (three copies: a warp can run one tile ahead of the others).
             auto stage_meta = [&](int jj, uint32_t tt) {
@@ -751,7 +765,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int tq = qb * BS + r;
                 const bool qin = qb >= 0 && qb < nb && tq < N;
                 const float lse = qin ? __ldg(LSE + bh * N + tq) : CUDART_INF_F;
-                mt[r] = (lse == -CUDART_INF_F) ? CUDART_INF_F : lse * kLog2e;
+                mt[r] = (lse == -CUDART_INF_F) ? -CUDART_INF_F : -(lse * kLog2e);  // -LSE, log2 units
                 mt[BS + r] = qin ? __ldg(Dg + bh * N + tq) : 0.0f;
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bar->meta[tt % 3]);
@@ -781,23 +795,28 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_wait_ld();
                 // P^T = exp(S^T / sqrt(d) - LSE), packed in place as bf16 pairs: v[c/2] <- (p[c], p[c+1])
                 if (__all_sync(0xffffffffu, lo == 0 && hi == BS)) {
+                    // scale-and-shift on fp32 pairs (one instruction per two columns)
+                    const uint64_t sc2 = f32x2_pack(scale_log2, scale_log2);
 #pragma unroll
                     for (int c = 0; c < BS; c += 4) {
                         const float4 l4 = *reinterpret_cast<const float4 *>(mt + c);
-                        const float p0 = ex2_approx(fmaf(__uint_as_float(v[c]), scale_log2, -l4.x));
-                        const float p1 = ex2_approx(fmaf(__uint_as_float(v[c + 1]), scale_log2, -l4.y));
-                        const float p2 = ex2_approx(fmaf(__uint_as_float(v[c + 2]), scale_log2, -l4.z));
-                        const float p3 = ex2_approx(fmaf(__uint_as_float(v[c + 3]), scale_log2, -l4.w));
-                        v[c >> 1] = pack_bf16(p0, p1);
-                        v[(c >> 1) + 1] = pack_bf16(p2, p3);
+                        float x0, x1, x2, x3;
+                        f32x2_unpack(f32x2_fma(f32x2_pack(__uint_as_float(v[c]), __uint_as_float(v[c + 1])), sc2,
+                                               f32x2_pack(l4.x, l4.y)),
+                                     x0, x1);
+                        f32x2_unpack(f32x2_fma(f32x2_pack(__uint_as_float(v[c + 2]), __uint_as_float(v[c + 3])), sc2,
+                                               f32x2_pack(l4.z, l4.w)),
+                                     x2, x3);
+                        v[c >> 1] = pack_bf16(ex2_approx(x0), ex2_approx(x1));
+                        v[(c >> 1) + 1] = pack_bf16(ex2_approx(x2), ex2_approx(x3));
                     }
                 } else {
 #pragma unroll
                     for (int c = 0; c < BS; c += 2) {
                         const float p0 = (c >= lo && c < hi)
-                                             ? ex2_approx(fmaf(__uint_as_float(v[c]), scale_log2, -mt[c])) : 0.0f;
+                                             ? ex2_approx(fmaf(__uint_as_float(v[c]), scale_log2, mt[c])) : 0.0f;
                         const float p1 = (c + 1 >= lo && c + 1 < hi)
-                                             ? ex2_approx(fmaf(__uint_as_float(v[c + 1]), scale_log2, -mt[c + 1]))
+                                             ? ex2_approx(fmaf(__uint_as_float(v[c + 1]), scale_log2, mt[c + 1]))
                                              : 0.0f;
                         v[c >> 1] = pack_bf16(p0, p1);
                     }
@@ -825,12 +844,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_wait_ld();
 #pragma unroll
                 for (int c = 0; c < BS; c += 4) {
+                    // on fp32 pairs: (dP^T - D) and the product with P^T, one instruction each per two columns
                     const float4 d4 = *reinterpret_cast<const float4 *>(mt + BS + c);
                     const uint32_t pa = v[c >> 1], pb = v[(c >> 1) + 1];
-                    g[c >> 1] = pack_bf16(__uint_as_float(pa << 16) * (__uint_as_float(g[c]) - d4.x),
-                                          __uint_as_float(pa & 0xFFFF0000u) * (__uint_as_float(g[c + 1]) - d4.y));
-                    g[(c >> 1) + 1] = pack_bf16(__uint_as_float(pb << 16) * (__uint_as_float(g[c + 2]) - d4.z),
-                                                __uint_as_float(pb & 0xFFFF0000u) * (__uint_as_float(g[c + 3]) - d4.w));
+                    float y0, y1, y2, y3;
+                    f32x2_unpack(f32x2_mul(f32x2_pack(__uint_as_float(pa << 16), __uint_as_float(pa & 0xFFFF0000u)),
+                                           f32x2_sub(f32x2_pack(__uint_as_float(g[c]), __uint_as_float(g[c + 1])),
+                                                     f32x2_pack(d4.x, d4.y))),
+                                 y0, y1);
+                    f32x2_unpack(f32x2_mul(f32x2_pack(__uint_as_float(pb << 16), __uint_as_float(pb & 0xFFFF0000u)),
+                                           f32x2_sub(f32x2_pack(__uint_as_float(g[c + 2]), __uint_as_float(g[c + 3])),
+                                                     f32x2_pack(d4.z, d4.w))),
+                                 y2, y3);
+                    g[c >> 1] = pack_bf16(y0, y1);
+                    g[(c >> 1) + 1] = pack_bf16(y2, y3);
                 }
 #pragma unroll
                 for (int c0 = 0; c0 < BS / 2; c0 += 32)
