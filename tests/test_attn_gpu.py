@@ -136,6 +136,43 @@ def test_block64_pairs_with_every_pattern(N, causal, oracle_mod):
     assert torch.all(torch.isinf(LSE.reshape(-1)[: 2 * w.bs]))
 
 
+@pytest.mark.parametrize("N,causal", [(50, False), (50, True), (100, False), (128, True)])
+def test_block64_one_pair(N, causal, oracle_mod):
+    """Block 64 with one or two query blocks: a single pair, its second row absent
+    (N <= 64) or present; every token."""
+    w = W.Workload("one_pair", B=2, H=2, N=N, d=64, bs=64, p=1.0, seed=53)
+    Q, K, V = W.generate(w)
+    rp, ci = oracle_mod.dense_csr(w.B, w.H, w.N, w.bs, causal=causal)
+    O, LSE = run_fwd(to_dev(Q), to_dev(K), to_dev(V), rp, ci, w.bs, causal)
+    tokens = np.arange(w.B * w.H * w.N, dtype=np.int64)
+    Oref, Lref = oracle_mod.attn_rows(Q, K, V, w.bs, causal, rp, ci, tokens)
+    compare_attention(O, LSE, Oref, Lref, tokens, w.d, "one_pair")
+
+
+@pytest.mark.slow
+def test_block64_largest_block_count(oracle_mod):
+    """Block 64 at the largest supported block count (4096 query blocks, a ragged last
+    block): the first pair's rows select every key block, so its union fills the
+    whole union slot; the other rows hold a few blocks, the last one included.
+    Sampled tokens: the first pair, the last pair and random pairs."""
+    rng = np.random.default_rng(54)
+    nb = 4096
+    w = W.Workload("nb4096", B=1, H=1, N=nb * 64 - 5, d=64, bs=64, p=1.0, seed=54)
+    Q, K, V = W.generate(w)
+    sets = [list(range(nb)), list(range(nb))]
+    for r in range(2, nb):
+        k = int(rng.integers(1, 9))
+        sets.append(sorted(set(rng.choice(nb, size=k, replace=False).tolist()) | {nb - 1}))
+    rp = np.zeros(nb + 1, np.int32)
+    rp[1:] = np.cumsum([len(x) for x in sets])
+    ci = np.asarray([j for x in sets for j in x], np.int32)
+    O, LSE = run_fwd(to_dev(Q), to_dev(K), to_dev(V), rp, ci, w.bs, False)
+    pairs = [0, nb // 2 - 1] + rng.choice(np.arange(1, nb // 2 - 1), size=6, replace=False).tolist()
+    tokens = np.concatenate([np.arange(p * 128, min(w.N, p * 128 + 128)) for p in sorted(pairs)]).astype(np.int64)
+    Oref, Lref = oracle_mod.attn_rows(Q, K, V, w.bs, False, rp, ci, tokens)
+    compare_attention(O, LSE, Oref, Lref, tokens, w.d, "nb4096")
+
+
 def test_block64_bad_csr_is_reported_and_in_range_entries_are_computed(oracle_mod):
     """Block 64: an out-of-range index and a repeated one are reported as
     FVATTN_ERR_BAD_CSR; every row is computed over its in-range entries."""
