@@ -28,18 +28,20 @@
 //     lane); warp 4 issues TMA loads of K and V tiles into a ring of shared
 //     memory stages; warp 5 issues the tcgen05 MMAs.
 //   * Tensor memory (512 columns) holds Q twice (the current and the next
-//     item), S twice and O once (fp32): S = Q K^T of key block j+2 is computed
-//     while the softmax works on block j+1 and the tensor cores run
-//     O += P_j V_j, so the tensor cores never wait for the softmax of the block
+//     item), S twice and O once (fp32): S = Q K^T of tile j+2 is computed
+//     while the softmax works on tile j+1 and the tensor cores run
+//     O += P_j V_j, so the tensor cores never wait for the softmax of the tile
 //     they need next.  Q comes from TMEM (TS MMA: only K is read from shared
 //     memory for S), P is written into the columns of its S buffer and read
 //     from there by the PV MMA (V from shared memory, MN-major).
-//   * tcgen05 MMAs of one thread execute in issue order: S of block j+2 is
-//     issued after PV of block j, which reads the P in the same columns.
+//   * tcgen05 MMAs of one thread execute in issue order: S of tile j+2 is
+//     issued after PV of tile j, which reads the P in the same columns.
 //   * The softmax reads the whole S row of its thread (tcgen05.ld), takes the
 //     row maximum, and writes P in place; the running reference maximum moves
 //     only when a row's maximum exceeds it by more than 2^8, so the rescale of
-//     O in tensor memory is rare.
+//     O in tensor memory is rare.  The scale-and-shift of the scores and the
+//     row sums run on packed fp32 pairs (one instruction per two columns): the
+//     softmax warp, not a pipe, is the critical path, so instructions count.
 //   * O stays in TMEM for the whole item; the epilogue divides by l, converts
 //     to bf16 and stores; LSE = (m + log2 l) ln 2.  The softmax warps load the
 //     next item's Q into TMEM before the epilogue, so the next item's first two
@@ -54,10 +56,11 @@
 // kind::f8f6f4 MMAs (e4m3 x e4m3, fp32 accumulation; twice the bf16 rate).
 //   * S: the codes' dot products are exact products summed in fp32; the tile's
 //     scale 2^(e_q + e_k) is folded into the softmax scale of that tile.
-//   * PV: P is rounded to e4m3 (one scale for all rows of a tile: the key block's
-//     2^(e_v - E), E the largest e_v of the item's blocks so far, so that P <= 256
-//     stays in range) and written four codes per TMEM column; the row sum l uses
-//     the unrounded P.  When a later block has a larger e_v, O is rescaled by the
+//   * PV: P is rounded to e4m3 (one scale for all rows of a key block: its
+//     2^(e_v - E), E the largest e_v the row has taken so far, so that P <= 256
+//     stays in range; the power of two rides in the exponent argument) and
+//     written four codes per TMEM column; the row sum l uses the unrounded P
+//     (the scaled values summed, then scaled back exactly by 2^(E - e_v)).  When a later block has a larger e_v, O is rescaled by the
 //     exact power of two 2^(E_old - E_new) (together with the maximum rescale).
 //     The epilogue multiplies by 2^E / l.
 #include <cuda.h>
@@ -122,7 +125,8 @@ struct Barriers {
     uint64_t pv_done, o_full, o_empty;
     uint64_t sched_full[2], sched_empty[2];
     uint64_t drain;
-    int4 sched_item[2];  // {row, col start, count, queue index + 1 (0: no more items)}
+    // {item (row, or pair of rows), CSR start (pairs: union entries), tiles, queue index + 1 (0: no more items)}
+    int4 sched_item[2];
     long long t_start;   // diagnostic: global timer at the start of the CTA's work
     uint32_t tmem_base;
     int abort_flag;
