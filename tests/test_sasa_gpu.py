@@ -29,6 +29,9 @@ SMALL = [
     W.Workload("sasa_bs64", B=2, H=3, N=2000, d=64, bs=64, p=0.8, dist="structured", grid=(5, 20, 20),
                head_scale=("uniform", 0.5, 4.0), seed=82),
     W.Workload("sasa_iid", B=1, H=2, N=1024, d=64, bs=64, p=0.6, seed=83),
+    # more than 256 key blocks: the shared-memory selection kernel writes the candidates
+    W.Workload("sasa_wide", B=1, H=2, N=20000, d=64, bs=64, p=0.8, dist="structured", grid=(5, 40, 100),
+               head_scale=("uniform", 0.5, 4.0), seed=84),
 ]
 
 
