@@ -70,6 +70,15 @@ def test_size_helpers(lib):
     assert fw >= 40 * 256 * 4 + 40 * 4
     assert fv.fvattn_fwd_workspace_bytes(1, 4097, 128, 128) == 0           # head limit 4096
     assert fv.fvattn_lpt_workspace_bytes(10, 5000) == 0                  # count limit 4096
+    # work items: query blocks at block 128, pairs of query blocks (2i, 2i+1) at block 64
+    assert fv.fvattn_attn_num_items(1, 40, 32760, 128) == 40 * 256
+    assert fv.fvattn_attn_num_items(1, 40, 32760, 64) == 40 * 256          # 512 blocks per head, 256 pairs
+    assert fv.fvattn_attn_num_items(2, 3, 900, 64) == 6 * 8                # 15 blocks: 7 pairs and one alone
+    assert fv.fvattn_attn_num_items(1, 1, 50, 64) == 1
+    assert fv.fvattn_attn_num_items(1, 1, 100, 32) == 0                    # block unsupported
+    # block 64 also keeps the pairs' union sizes, their scan and per-head sums
+    f64 = fv.fvattn_fwd_workspace_bytes(1, 40, 32760, 64)
+    assert f64 >= 40 * 256 * 4 * 3 + 40 * 4 * 2
 
 
 def test_invalid_arguments_rejected_before_any_device_work(lib):
@@ -101,6 +110,10 @@ def test_invalid_arguments_rejected_before_any_device_work(lib):
     assert lib.fvattn_quant_e4m3(fake, 1, 1, 128, 64, 64, fake, None, None) == -1
     assert lib.fvattn_quant_e4m3(P(18), 1, 1, 128, 64, 64, fake, fake, None) == -3
     assert lib.fvattn_quant_e4m3(fake, 0, 1, 128, 64, 64, fake, fake, None) == -1
+    # the block-64 work order reads the column indices and writes a status word
+    assert lib.fvattn_attn_work_order(fake, None, 1, 1, 256, 64, fake, fake, 1 << 20, fake, None) == -1
+    assert lib.fvattn_attn_work_order(fake, fake, 1, 1, 256, 64, fake, fake, 1 << 20, None, None) == -1
+    assert lib.fvattn_attn_work_order(fake, None, 1, 1, 256, 32, fake, fake, 1 << 20, None, None) == -2
     # routing supports at most 1024 blocks per sequence
     assert lib.fvattn_route(fake, fake, 1, 1, 1025 * 64, 64, 64, 0.5, fake, fake, 4, fake, fake, 1 << 30, fake,
                             None) == -2
