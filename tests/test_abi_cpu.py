@@ -46,6 +46,25 @@ def test_only_declared_symbols_are_exported(lib):
     assert exported == set(declared_functions())
 
 
+def test_header_is_plain_c(tmp_path):
+    """The boundary is a C ABI: the header compiles as strict C99 (and as C++), and
+    a C program that calls a host-only entry point links against the library."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "use.c"
+    src.write_text('#include "fvattn.h"\n'
+                   'int main(void) { return fvattn_attn_num_items(1, 40, 32760, 64) == 40 * 256 ? 0 : 1; }\n')
+    inc = os.path.join(ROOT, "include")
+    for cmd in (["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", inc, "-c", str(src),
+                 "-o", str(tmp_path / "c.o")],
+                ["g++", "-std=c++17", "-Wall", "-Wextra", "-Werror", "-I", inc, "-x", "c++", "-c", str(src),
+                 "-o", str(tmp_path / "cpp.o")]):
+        r = subprocess.run(cmd, capture_output=True, text=True)
+        assert r.returncode == 0, r.stderr
+
+
 def test_status_strings(lib):
     import top_routed_block_b200 as fv
     assert fv.status_string(0) == "ok"
