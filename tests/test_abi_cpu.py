@@ -46,7 +46,7 @@ def test_only_declared_symbols_are_exported(lib):
     assert exported == set(declared_functions())
 
 
-def test_header_is_plain_c(tmp_path):
+def test_header_is_plain_c(lib, tmp_path):
     """The boundary is a C ABI: the header compiles as strict C99 (and as C++), and
     a C program that calls a host-only entry point links against the library."""
     import shutil
@@ -63,6 +63,13 @@ def test_header_is_plain_c(tmp_path):
                  "-o", str(tmp_path / "cpp.o")]):
         r = subprocess.run(cmd, capture_output=True, text=True)
         assert r.returncode == 0, r.stderr
+    from top_routed_block_b200 import LIB_PATH
+    libdir = os.path.dirname(LIB_PATH)
+    exe = tmp_path / "use"
+    r = subprocess.run(["gcc", str(tmp_path / "c.o"), "-o", str(exe), "-L", libdir, "-lfvattn",
+                        "-Wl,-rpath," + libdir], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    assert subprocess.run([str(exe)]).returncode == 0
 
 
 def test_status_strings(lib):
