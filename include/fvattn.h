@@ -184,11 +184,12 @@ FVATTN_API int fvattn_quant_e4m3(const void *X, int B, int H, int N, int d, int 
  * A persistent grid takes the items from a queue ordered head-major and
  * longest-first: heads by total work descending, the items of a head by size
  * descending (ties by lower index), so that the SMs share one head's K and V in
- * L2 at a time and finish on the shortest items.  B*H <= 4096, else
- * FVATTN_ERR_UNSUPPORTED.  Malformed rows (a negative count, column indices out
- * of range or not ascending) set *dev_status = FVATTN_ERR_BAD_CSR; at block 128
- * the offending indices are skipped (an index not above the one before it), at
- * block 64 each row uses the set of its in-range indices.
+ * L2 at a time and finish on the shortest items.  B*H <= 4096 and
+ * ceil(N/block) <= 4096, else FVATTN_ERR_UNSUPPORTED (before any device work).
+ * Malformed rows (a negative count, column indices out of range or not
+ * ascending) set *dev_status = FVATTN_ERR_BAD_CSR; at block 128 the offending
+ * indices are skipped (an index not above the one before it), at block 64 each
+ * row uses the set of its in-range indices.
  */
 FVATTN_API int fvattn_sparse_fwd(const void *Q, const void *K, const void *V, const int32_t *row_ptr,
                       const int32_t *col_idx, int B, int H, int N, int d, int block, int causal, void *O,
@@ -289,7 +290,8 @@ FVATTN_API size_t fvattn_bwd_workspace_bytes(int B, int H, int N, int block);
  *   row_ptr, col_idx  the CSR block mask of the forward (ascending columns).
  *   dQ, dK, dV      out, bf16 [B,H,N,d] (fp32 accumulation in tensor memory).
  *   workspace       >= fvattn_bwd_workspace_bytes(B,H,N,block).
- * block must be 128 and d 64 or 128 (else FVATTN_ERR_UNSUPPORTED); B*H <= 4096.
+ * block must be 128 and d 64 or 128 (else FVATTN_ERR_UNSUPPORTED); B*H <= 4096 and
+ * ceil(N/block) <= 4096 (else FVATTN_ERR_UNSUPPORTED, before any device work).
  * Work: D; the transpose of the mask (key block -> the query blocks that
  * selected it); a dQ pass over the CSR rows and a dK/dV pass over the key
  * blocks, both on tcgen05 with accumulators in tensor memory and longest-first

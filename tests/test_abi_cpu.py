@@ -136,6 +136,14 @@ def test_invalid_arguments_rejected_before_any_device_work(lib):
     assert lib.fvattn_quant_e4m3(fake, 1, 1, 128, 64, 64, fake, None, None) == -1
     assert lib.fvattn_quant_e4m3(P(18), 1, 1, 128, 64, 64, fake, fake, None) == -3
     assert lib.fvattn_quant_e4m3(fake, 0, 1, 128, 64, 64, fake, fake, None) == -1
+    # at most 4096 query blocks per sequence and 4096 heads, refused before any device work
+    for block in (64, 128):
+        assert lib.fvattn_sparse_fwd(fake, fake, fake, fake, fake, 1, 1, 4097 * block, 64, block, 0, fake, fake,
+                                     fake, 1 << 30, fake, None) == -2
+    assert lib.fvattn_sparse_fwd(fake, fake, fake, fake, fake, 1, 4097, 128, 64, 64, 0, fake, fake, fake, 1 << 30,
+                                 fake, None) == -2
+    assert lib.fvattn_sparse_bwd(fake, fake, fake, fake, fake, fake, fake, fake, 1, 1, 4097 * 128, 64, 128, 0,
+                                 fake, fake, fake, fake, 1 << 30, fake, None) == -2
     # the block-64 work order reads the column indices and writes a status word
     assert lib.fvattn_attn_work_order(fake, None, 1, 1, 256, 64, fake, fake, 1 << 20, fake, None) == -1
     assert lib.fvattn_attn_work_order(fake, fake, 1, 1, 256, 64, fake, fake, 1 << 20, None, None) == -1

@@ -307,6 +307,9 @@ static int sparse_fwd_impl(const void *Q, const void *K, const void *V, const in
     if ((reinterpret_cast<uintptr_t>(row_ptr) | reinterpret_cast<uintptr_t>(col_idx) |
          reinterpret_cast<uintptr_t>(LSE) | reinterpret_cast<uintptr_t>(dev_status)) & 3u)
         return FVATTN_ERR_ALIGNMENT;
+    // at most kMaxCount query blocks per sequence (the ordering kernels' shared arrays, and
+    // at block 64 the pairs' bitmaps and union slots); the workspace query returns 0 beyond
+    if (ceil_div(N, block) > kMaxCount || static_cast<int64_t>(B) * H > kMaxHeads) return FVATTN_ERR_UNSUPPORTED;
     if (ws_bytes < fvattn_fwd_workspace_bytes(B, H, N, block)) return FVATTN_ERR_CAPACITY;
     if ((rc = check_device()) != FVATTN_OK) return rc;
     DeviceInfo info;
@@ -536,6 +539,8 @@ int fvattn_sparse_bwd(const void *Q, const void *K, const void *V, const void *O
         return FVATTN_ERR_ALIGNMENT;
     const int64_t BH = static_cast<int64_t>(B) * H;
     if (BH > kMaxHeads) return FVATTN_ERR_UNSUPPORTED;
+    // at most kMaxCount blocks per sequence (the workspace query returns 0 beyond)
+    if (ceil_div(N, block) > kMaxCount) return FVATTN_ERR_UNSUPPORTED;
     const int nb = static_cast<int>(ceil_div(N, block));
     if (ws_bytes < fvattn_bwd_workspace_bytes(B, H, N, block)) return FVATTN_ERR_CAPACITY;
     if ((rc = check_device()) != FVATTN_OK) return rc;
