@@ -172,7 +172,11 @@ FVATTN_API int fvattn_quant_e4m3(const void *X, int B, int H, int N, int d, int 
  * An empty keys(t) gives O[t] = 0 and LSE[t] = -inf.
  *
  *   Q, K, V     bf16 [B,H,N,d], read only.
- *   row_ptr, col_idx  CSR as above (e.g. from fvattn_route), read only.
+ *   row_ptr, col_idx  CSR as above (e.g. from fvattn_route), read only.  The
+ *               library reads col_idx[row_ptr[r] .. row_ptr[r+1]) for every row and
+ *               cannot check that this lies inside the caller's col_idx buffer:
+ *               row_ptr[B*H*nb] must not exceed its length (a row with a negative
+ *               count is reported as FVATTN_ERR_BAD_CSR and read as empty).
  *   causal      0 or 1.
  *   O           out, bf16 [B,H,N,d].   LSE  out, fp32 [B,H,N].
  *   workspace   >= fvattn_fwd_workspace_bytes(B,H,N,block).
