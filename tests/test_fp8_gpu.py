@@ -42,6 +42,8 @@ SMALL = [
                 head_scale=("uniform", 0.5, 4.0), seed=64), False),
     (W.Workload("fp8_large_scores", B=1, H=2, N=600, d=128, bs=128, p=0.8, dist="structured", grid=(6, 10, 10),
                 head_scale=("const", 6.0), seed=65), False),
+    # block 64, causal, an odd block count (the last pair holds one row) and a ragged last block
+    (W.Workload("fp8_bs64_causal_odd", B=1, H=2, N=900, d=128, bs=64, p=1.0, seed=66), True),
 ]
 
 

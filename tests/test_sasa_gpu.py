@@ -29,7 +29,7 @@ SMALL = [
     W.Workload("sasa_bs64", B=2, H=3, N=2000, d=64, bs=64, p=0.8, dist="structured", grid=(5, 20, 20),
                head_scale=("uniform", 0.5, 4.0), seed=82),
     W.Workload("sasa_iid", B=1, H=2, N=1024, d=64, bs=64, p=0.6, seed=83),
-    # more than 256 key blocks: the shared-memory selection kernel writes the candidates
+    # more than 256 key blocks per row (the selection sorts 512 positions per row)
     W.Workload("sasa_wide", B=1, H=2, N=20000, d=64, bs=64, p=0.8, dist="structured", grid=(5, 40, 100),
                head_scale=("uniform", 0.5, 4.0), seed=84),
 ]
@@ -94,6 +94,27 @@ def test_sasa_video_full_size(oracle_mod):
         assert set(bci[brp[row]:brp[row + 1]]) <= set(ci_g[rp_g[row]:rp_g[row + 1]])
     print(f"video: {int(added.sum())} blocks added over {machines} machines to {int((added > 0).sum())} rows, "
           f"mass {mass.sum():.4f}")
+
+
+@pytest.mark.parametrize("w", [SMALL[0], SMALL[1]], ids=lambda w: w.name)
+def test_attention_on_the_augmented_mask(w, oracle_mod):
+    """The augmented mask drives the attention like any mask (at block 64 the paired
+    query blocks walk the union of their augmented lists): every token against the
+    oracle on that mask."""
+    import top_routed_block_b200 as fv
+    from tests.gpu_util import compare_attention
+    Q, K, V = W.generate(w)
+    dQ, dK, dV = to_dev(Q), to_dev(K), to_dev(V)
+    r = fv.fvattn_route_sasa(dQ, dK, w.p, w.bs, 148)
+    fv.check_status(r.dev_status, "fvattn_route_sasa")
+    assert int(r.added.sum().item()) > 0, "choose a case where the plan adds blocks"
+    O, LSE, st = fv.fvattn_sparse_fwd(dQ, dK, dV, r.row_ptr, r.col_idx, w.bs, False)
+    fv.check_status(st, "forward on the augmented mask")
+    rp = r.row_ptr.cpu().numpy()
+    ci = r.col_idx[: int(rp[-1])].cpu().numpy()
+    tokens = np.arange(w.B * w.H * w.N, dtype=np.int64)
+    Oref, Lref = oracle_mod.attn_rows(Q, K, V, w.bs, False, rp, ci, tokens)
+    compare_attention(O, LSE, Oref, Lref, tokens, w.d, w.name)
 
 
 def test_sasa_rejects_bad_machine_counts():
