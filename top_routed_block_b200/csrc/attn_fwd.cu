@@ -60,9 +60,10 @@
 //     2^(e_v - E), E the largest e_v the row has taken so far, so that P <= 256
 //     stays in range; the power of two rides in the exponent argument) and
 //     written four codes per TMEM column; the row sum l uses the unrounded P
-//     (the scaled values summed, then scaled back exactly by 2^(E - e_v)).  When a later block has a larger e_v, O is rescaled by the
-//     exact power of two 2^(E_old - E_new) (together with the maximum rescale).
-//     The epilogue multiplies by 2^E / l.
+//     (the scaled values summed, then scaled back exactly by 2^(E - e_v)).
+//     When a later block has a larger e_v, O is rescaled by the exact power of
+//     two 2^(E_old - E_new) (together with the maximum rescale).  The epilogue
+//     multiplies by 2^E / l.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cstdint>
